@@ -1,0 +1,168 @@
+"""fp64 CPU oracle for multi-scale deformable attention (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never does, and shares no code with it.
+
+The arithmetic lives in ``msda_oracle.c`` (plain C, double precision, direct
+loops over the defining sums); this module only compiles it with gcc, widens
+inputs to float64 and passes pointers.  See the C file's header for the page
+citations and the readings taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "msda_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_build", "libmsda_oracle.so")
+_lib = None
+_lock = threading.Lock()
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("B", "S", "Q", "M", "D", "L", "K")]
+
+
+def build(force: bool = False) -> str:
+    """Compiles the oracle with gcc into oracle/_build (no GPU involved)."""
+    os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + ".%d.tmp" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            D = ctypes.POINTER(_Dims)
+            lib.msda_oracle_forward.argtypes = [D, P, P, P, P, P, P]
+            lib.msda_oracle_backward.argtypes = [D, P, P, P, P, P, P, P, P, P]
+            lib.msda_oracle_sampling_locations.argtypes = [D, P, P, P, P]
+            lib.msda_oracle_softmax.argtypes = [D, P, P]
+            lib.msda_oracle_fused_chain.argtypes = [D, P, P, P, P, P, P, P]
+            for f in ("msda_oracle_forward", "msda_oracle_backward", "msda_oracle_sampling_locations",
+                      "msda_oracle_softmax", "msda_oracle_fused_chain"):
+                getattr(lib, f).restype = None
+            _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _i64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.int64)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dims(value: np.ndarray, loc_like: np.ndarray) -> _Dims:
+    B, S, M, D = value.shape
+    _, Q, M2, L, K = loc_like.shape[:5]
+    assert M2 == M and loc_like.shape[0] == B
+    return _Dims(B, S, Q, M, D, L, K)
+
+
+def forward(value, spatial_shapes, level_start_index, sampling_locations, attention_weights):
+    """out[B,Q,M,D] (float64) of the core operator."""
+    v, sh, st = _f64(value), _i64(spatial_shapes), _i64(level_start_index)
+    loc, a = _f64(sampling_locations), _f64(attention_weights)
+    d = _dims(v, a)
+    out = np.empty((d.B, d.Q, d.M, d.D), np.float64)
+    _load().msda_oracle_forward(ctypes.byref(d), _p(v), _p(sh), _p(st), _p(loc), _p(a), _p(out))
+    return out
+
+
+def backward(value, spatial_shapes, level_start_index, sampling_locations, attention_weights,
+             grad_output):
+    """(grad_value [B,S,M,D], grad_sampling_locations [B,Q,M,L,K,2],
+    grad_attention_weights [B,Q,M,L,K]), float64."""
+    v, sh, st = _f64(value), _i64(spatial_shapes), _i64(level_start_index)
+    loc, a, g = _f64(sampling_locations), _f64(attention_weights), _f64(grad_output)
+    d = _dims(v, a)
+    gv = np.empty_like(v)
+    gl = np.empty_like(loc)
+    ga = np.empty_like(a)
+    _load().msda_oracle_backward(ctypes.byref(d), _p(v), _p(sh), _p(st), _p(loc), _p(a), _p(g),
+                                 _p(gv), _p(gl), _p(ga))
+    return gv, gl, ga
+
+
+def sampling_locations(spatial_shapes, reference_points, sampling_offsets):
+    """loc = ref + off / (W_l, H_l), float64 [B,Q,M,L,K,2]."""
+    sh, ref, off = _i64(spatial_shapes), _f64(reference_points), _f64(sampling_offsets)
+    B, Q, M, L, K, _ = off.shape
+    d = _Dims(B, 0, Q, M, 0, L, K)
+    loc = np.empty_like(off)
+    _load().msda_oracle_sampling_locations(ctypes.byref(d), _p(sh), _p(ref), _p(off), _p(loc))
+    return loc
+
+
+def softmax(attention_logits, L: int, K: int):
+    """Softmax over the L*K logits of each (b,q,m); returns [B,Q,M,L,K] float64."""
+    z = _f64(attention_logits)
+    B, Q, M, n = z.shape
+    assert n == L * K
+    d = _Dims(B, 0, Q, M, 0, L, K)
+    a = np.empty_like(z)
+    _load().msda_oracle_softmax(ctypes.byref(d), _p(z), _p(a))
+    return a.reshape(B, Q, M, L, K)
+
+
+def fused_chain(spatial_shapes, attention_weights, grad_loc, grad_attn, want_ref: bool = True):
+    """(grad_offsets, grad_reference_points or None, grad_logits)."""
+    sh, a, gl, ga = _i64(spatial_shapes), _f64(attention_weights), _f64(grad_loc), _f64(grad_attn)
+    B, Q, M, L, K = a.shape
+    d = _Dims(B, 0, Q, M, 0, L, K)
+    goff = np.empty_like(gl)
+    gref = np.empty((B, Q, 2), np.float64) if want_ref else None
+    glog = np.empty((B, Q, M, L * K), np.float64)
+    _load().msda_oracle_fused_chain(ctypes.byref(d), _p(sh), _p(a), _p(gl), _p(ga), _p(goff),
+                                    _p(gref) if want_ref else None, _p(glog))
+    return goff, gref, glog
+
+
+def fused_forward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
+                  attention_logits):
+    """Fused forward: locations and softmax first, then the core sum.
+
+    Returns (out, attention_weights, sampling_locations), float64."""
+    loc = sampling_locations(spatial_shapes, reference_points, sampling_offsets)
+    L, K = loc.shape[3], loc.shape[4]
+    a = softmax(attention_logits, L, K)
+    return forward(value, spatial_shapes, level_start_index, loc, a), a, loc
+
+
+def fused_backward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
+                   attention_logits, grad_output, want_ref: bool = True):
+    """(grad_value, grad_reference_points, grad_sampling_offsets, grad_attention_logits)."""
+    loc = sampling_locations(spatial_shapes, reference_points, sampling_offsets)
+    L, K = loc.shape[3], loc.shape[4]
+    a = softmax(attention_logits, L, K)
+    gv, gl, ga = backward(value, spatial_shapes, level_start_index, loc, a, grad_output)
+    goff, gref, glog = fused_chain(spatial_shapes, a, gl, ga, want_ref)
+    return gv, gref, goff, glog
+
+
+def pixel_coordinates(spatial_shapes, sampling_locations):
+    """fp64 pixel coordinates (x, y) = (loc_x*W - 0.5, loc_y*H - 0.5) of each
+    sample; tests use them to find samples that sit on a cell edge."""
+    sh = _i64(spatial_shapes)
+    loc = _f64(sampling_locations)
+    W = sh[:, 1].astype(np.float64)[None, None, None, :, None]
+    H = sh[:, 0].astype(np.float64)[None, None, None, :, None]
+    return loc[..., 0] * W - 0.5, loc[..., 1] * H - 0.5

@@ -1,0 +1,100 @@
+"""Planted mistakes in the oracle must fail its pins.
+
+Each case edits a copy of oracle/msda_oracle.c (a dropped term, a wrong sign
+or index, a transposed operand, a wrong pixel convention), builds it into a
+temporary directory, swaps it in for the real oracle and runs the pin checks,
+expecting at least one of them to fail.  Every mutant keeps its memory
+accesses inside the arrays.  CPU only; nothing runs on a GPU.
+"""
+import contextlib
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "msda_oracle.c")
+
+MUTATIONS = {
+    "no_half_pixel_shift": ("double x = lx * (double)W - 0.5;", "double x = lx * (double)W;"),
+    "align_corners_true": ("double x = lx * (double)W - 0.5;", "double x = lx * (double)(W - 1);"),
+    "x_y_swapped_scale": ("double y = ly * (double)H - 0.5;", "double y = ly * (double)W - 0.5;"),
+    "corner_weight_transposed": ("s.w[1] = (1.0 - s.fy) * s.fx;", "s.w[1] = s.fy * (1.0 - s.fx);"),
+    "column_mirrored": ("int64_t key = start_l + cy * W + cx;",
+                        "int64_t key = start_l + cy * W + (W - 1 - cx);"),
+    "level_start_ignored": ("int64_t key = start_l + cy * W + cx;", "int64_t key = cy * W + cx;"),
+    # clamping corners to the border (the other option the pages mention)
+    # instead of masking them to zero; every access stays inside the map
+    "border_clamp_not_zero": ("s.inb[c] = s.cx[c] >= 0 && s.cx[c] < W && s.cy[c] >= 0 && s.cy[c] < H;",
+                              "s.cx[c] = s.cx[c] < 0 ? 0 : (s.cx[c] >= W ? W - 1 : s.cx[c]); "
+                              "s.cy[c] = s.cy[c] < 0 ? 0 : (s.cy[c] >= H ? H - 1 : s.cy[c]); "
+                              "s.inb[c] = 1;"),
+    "grad_x_scale_H": ("grad_loc[2 * p] = (double)W * a * gx;", "grad_loc[2 * p] = (double)H * a * gx;"),
+    "dsdx_sign": ("double dx = (1.0 - s.fy) * (v01 - v00) + s.fy * (v11 - v10);",
+                  "double dx = (1.0 - s.fy) * (v00 - v01) + s.fy * (v11 - v10);"),
+    "dsdy_dropped_term": ("double dy = (1.0 - s.fx) * (v10 - v00) + s.fx * (v11 - v01);",
+                          "double dy = (1.0 - s.fx) * (v10 - v00);"),
+    "grad_value_no_weight": ("gv[ch] += a * s.w[c] * g[ch];", "gv[ch] += a * g[ch];"),
+    "grad_attn_unweighted": ("double samp = s.w[0] * v00 + s.w[1] * v01 + s.w[2] * v10 + s.w[3] * v11;",
+                             "double samp = v00 + v01 + v10 + v11;"),
+    "offset_normalizer_swapped": ("loc[2 * p] = r[0] + off[2 * p] / (double)shapes[2 * l + 1];",
+                                  "loc[2 * p] = r[0] + off[2 * p] / (double)shapes[2 * l];"),
+    "softmax_no_normalize": ("a[j] /= sum;", "a[j] /= 1.0;"),
+    "softmax_jacobian_sign": ("grad_logits[r * n + j] = attn[r * n + j] * (grad_attn[r * n + j] - dot);",
+                              "grad_logits[r * n + j] = attn[r * n + j] * (grad_attn[r * n + j] + dot);"),
+    "grad_off_not_scaled": ("grad_off[2 * p] = grad_loc[2 * p] / (double)shapes[2 * l + 1];",
+                            "grad_off[2 * p] = grad_loc[2 * p];"),
+    "grad_ref_y_from_x": ("grad_ref[2 * (b * d->Q + q) + 1] += grad_loc[2 * p + 1];",
+                          "grad_ref[2 * (b * d->Q + q) + 1] += grad_loc[2 * p];"),
+}
+
+PIN_CHECKS = [
+    pins.test_golden_worked_bilinear,
+    pins.test_golden_worked_two_level_fused,
+    lambda o: pins.test_identity_at_pixel_centres(o, ((5, 7), (3, 11), (1, 1))),
+    pins.test_constant_map,
+    pins.test_linear_map_forward_and_backward,
+    pins.test_backward_matches_central_differences,
+    pins.test_fused_backward_matches_central_differences,
+    pins.test_softmax_closed_forms,
+    lambda o: pins.test_matches_torch_grid_sample(o, "ragged"),
+]
+
+
+@contextlib.contextmanager
+def _swapped(lib_path):
+    oracle._load()
+    saved = oracle._lib
+    lib = ctypes.CDLL(lib_path)
+    for name in ("msda_oracle_forward", "msda_oracle_backward", "msda_oracle_sampling_locations",
+                 "msda_oracle_softmax", "msda_oracle_fused_chain"):
+        f, ref = getattr(lib, name), getattr(saved, name)
+        f.argtypes, f.restype = ref.argtypes, ref.restype
+    oracle._lib = lib
+    try:
+        yield
+    finally:
+        oracle._lib = saved
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    mutated = tmp_path / "mut.c"
+    mutated.write_text(src.replace(old, new))
+    lib_path = str(tmp_path / "libmut.so")
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-o", lib_path,
+                           str(mutated), "-lm"])
+    failures = 0
+    with _swapped(lib_path):
+        for check in PIN_CHECKS:
+            try:
+                check(oracle)
+            except AssertionError:
+                failures += 1
+    assert failures > 0, f"mutation {name} passed every pin"
