@@ -1,0 +1,584 @@
+#!/usr/bin/env python
+"""Throughput of the multi-scale deformable attention core on B200.
+
+One step = one pass of the whole hot path over one batch of the workload:
+msda_fused_forward (location step, softmax over L*K, bilinear gather,
+weighted sum), msda_zero_grads (float32 gradient accumulators) and
+msda_fused_backward (gathers again, gradients of the sample, grad_value
+scatter, chain rule to offsets, reference points and logits).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Prints one JSON line on rank 0.  `value` is G sampled points per second over
+the fwd+bwd step (samples = B*Q*M*L*K per step, all ranks), with inputs
+resident in HBM and L2 flushed between steps; each kernel is timed with CUDA
+events on the stream it is launched on.  Multi-GPU runs (torchrun, one process
+per GPU) give every rank its own batch of the workload (weak scaling; there is
+no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from scale_deformable_attention_msdeformattn_b200 import workloads as wl  # noqa: E402
+
+METRIC = "G sampled points/s and fwd+bwd ms at DETR-encoder shape; % of B200 HBM roofline"
+UNIT = "G samples/s"
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one launch) of
+# the kernels as last captured with ncu, keyed by kernel; each entry records the
+# hash of the CUDA sources it was taken from and is reported only while those
+# sources are unchanged.  Filled from the summaries under profiles/.
+NCU_TRAFFIC = {}
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "scale_deformable_attention_msdeformattn_b200",
+                                           "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="detr_encoder_f32", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="host-core seconds spent timing the oracle for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-nonfused", action="store_true")
+    ap.add_argument("--out", default=None, help="also append the JSON line to this file")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if a.steps < 1:
+        ap.error("--steps must be >= 1")
+    return a
+
+
+# ---------------------------------------------------------------- bytes ----
+
+def algorithmic_bytes(w: wl.Workload) -> dict:
+    """Each tensor of a launch touched once (inputs read, outputs written)."""
+    B, S, Q, M, D, L, K = w.B, w.S, w.num_queries, w.M, w.D, w.L, w.K
+    e = 2 if w.dtype == "bf16" else 4
+    value = B * S * M * D * e
+    rowd = B * Q * M * D * e
+    samples = B * Q * M * L * K
+    loc = samples * 2 * 4
+    attn = samples * 4
+    ref = B * Q * 2 * 4
+    gvalue = B * S * M * D * 4
+    fwd = value + loc + attn + rowd
+    bwd = rowd + value + loc + attn + gvalue + loc + attn
+    fused_fwd = value + loc + attn + ref + rowd             # offsets, logits, ref -> out
+    fused_bwd = rowd + value + loc + attn + ref + gvalue + loc + attn + ref
+    return {"forward": fwd, "backward": bwd, "fused_forward": fused_fwd,
+            "fused_backward": fused_bwd, "zero_grads": gvalue + ref}
+
+
+# --------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """Polls NVML for the SM clock and the clock-event reasons of one GPU."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device: int, period_s: float = 0.005):
+        self.samples = []
+        self.period = period_s
+        self.ok = False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            h = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            except Exception:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = int(vis.split(",")[torch_device]) if vis and vis.split(",")[0].isdigit() else torch_device
+                h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.h = h
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.ok = True
+        except Exception as e:  # NVML missing: report that instead of clocks
+            self.err = repr(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self._reasons_fn(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": "NVML unavailable: " + getattr(self, "err", "")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        reasons = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(mhz), "reasons": reasons, "samples": len(mhz)}
+
+
+# ------------------------------------------------------------- our arm -----
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _to_device(x: wl.Inputs, dev):
+    import torch
+
+    def val(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    t = {
+        "value": val(x.value),
+        "spatial_shapes": torch.from_numpy(x.spatial_shapes).to(dev),
+        "level_start_index": torch.from_numpy(x.level_start_index).to(dev),
+        "reference_points": torch.from_numpy(x.reference_points).to(dev),
+        "sampling_offsets": torch.from_numpy(x.sampling_offsets).to(dev),
+        "attention_logits": torch.from_numpy(x.attention_logits).to(dev),
+        "grad_output": val(x.grad_output),
+    }
+    if x.sampling_locations.size:
+        t["sampling_locations"] = torch.from_numpy(x.sampling_locations).to(dev)
+        t["attention_weights"] = torch.from_numpy(x.attention_weights).to(dev)
+    return t
+
+
+def _pinned(x: wl.Inputs):
+    """Host copies of one step's inputs in pinned memory (for the e2e leg)."""
+    import torch
+
+    def pin(a):
+        if a.dtype == np.uint16:
+            t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(a)
+        return t.pin_memory()
+
+    return {k: pin(v) for k, v in {
+        "value": x.value, "spatial_shapes": x.spatial_shapes,
+        "level_start_index": x.level_start_index, "reference_points": x.reference_points,
+        "sampling_offsets": x.sampling_offsets, "attention_logits": x.attention_logits,
+        "grad_output": x.grad_output}.items()}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import scale_deformable_attention_msdeformattn_b200 as msda
+
+    world, rank, local = _dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    base = wl.WORKLOADS[args.workload]
+    # weak scaling: every rank samples its own batch (its own seed)
+    w = base if rank == 0 else wl.dataclasses.replace(base, index=base.index + 1000 * rank)
+    want_nonfused = not args.no_nonfused and world == 1
+    x = wl.generate(w, with_nonfused=want_nonfused)
+    t = _to_device(x, dev)
+    B, S, Q, M, D, L, K = w.B, w.S, w.num_queries, w.M, w.D, w.L, w.K
+    out = torch.empty((B, Q, M, D), dtype=t["value"].dtype, device=dev)
+    gv = torch.empty((B, S, M, D), dtype=torch.float32, device=dev)
+    gref = torch.empty((B, Q, 2), dtype=torch.float32, device=dev)
+    goff = torch.empty((B, Q, M, L, K, 2), dtype=torch.float32, device=dev)
+    glog = torch.empty((B, Q, M, L * K), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    outputs = {"out": out, "grad_value": gv, "grad_reference_points": gref,
+               "grad_sampling_offsets": goff, "grad_attention_logits": glog}
+
+    def step(ev, tin=None):
+        tin = tin or t
+        ev[0].record(stream)
+        msda.fused_forward(tin["value"], tin["spatial_shapes"], tin["level_start_index"],
+                           tin["reference_points"], tin["sampling_offsets"],
+                           tin["attention_logits"], out=out)
+        ev[1].record(stream)
+        msda.zero_grads(gv, gref)
+        ev[2].record(stream)
+        msda.fused_backward(tin["value"], tin["spatial_shapes"], tin["level_start_index"],
+                            tin["reference_points"], tin["sampling_offsets"],
+                            tin["attention_logits"], tin["grad_output"], accumulate=True,
+                            grad_value=gv, grad_reference_points=gref,
+                            grad_sampling_offsets=goff, grad_attention_logits=glog)
+        ev[3].record(stream)
+        return outputs
+
+    def events(n):
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+
+    warm = events(args.warmup)
+    for i in range(args.warmup):
+        flush.fill_(float(i))
+        step(warm[i])
+    torch.cuda.synchronize()
+    if msda.device_status() != 0:
+        raise SystemExit("kernels reported inconsistent geometry")
+
+    evs = events(args.steps)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(float(i))  # L2 flush, outside the timed events
+        step(evs[i])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    barrier()
+    clocks.stop()
+
+    fwd = [e[0].elapsed_time(e[1]) for e in evs]
+    zero = [e[1].elapsed_time(e[2]) for e in evs]
+    bwd = [e[2].elapsed_time(e[3]) for e in evs]
+    stepms = [e[0].elapsed_time(e[3]) for e in evs]
+    total_ms = float(sum(stepms))
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = tt.item()
+
+    samples_step = w.samples
+    value = world * samples_step * args.steps / (total_ms * 1e-3) / 1e9
+    ms_per_step = total_ms / args.steps
+    nbytes = algorithmic_bytes(w)
+
+    result = None
+    if rank == 0:
+        peaks = _peaks()
+        fwd_ms, bwd_ms, zero_ms = statistics.mean(fwd), statistics.mean(bwd), statistics.mean(zero)
+        dom = "fused_backward" if bwd_ms >= fwd_ms else "fused_forward"
+        dom_ms = bwd_ms if dom == "fused_backward" else fwd_ms
+        achieved = nbytes[dom] / (dom_ms * 1e-3) / 1e9
+        tr = NCU_TRAFFIC.get((dom, w.name))
+        traffic = tr["bytes"] if tr and tr.get("csrc") == csrc_hash() else None
+        step_bytes = nbytes["fused_forward"] + nbytes["fused_backward"]
+        result = {
+            "metric": METRIC,
+            "value": round(value, 4),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32" if w.dtype == "f32" else "bf16 value / f32 accumulate",
+            "data": "synthetic: seeded SplitMix64 + Box-Muller draws of the workload's shapes "
+                    "and distributions (no dataset)",
+            "config": {
+                "workload": w.name, "B": w.B, "levels_HW": [list(l) for l in w.levels],
+                "Q": Q, "M": M, "D": D, "L": L, "K": K,
+                "offset_sigma_px": w.offset_sigma, "logit_sigma": w.logit_sigma,
+                "samples_per_step_per_gpu": samples_step,
+                "step": "msda_fused_forward + msda_zero_grads + msda_fused_backward",
+                "l2": "flushed between steps (256 MiB write outside the timed events)",
+                "parallelism": f"dp{world} (independent batch per GPU)",
+            },
+            "fwd_ms": round(fwd_ms, 5),
+            "zero_ms": round(zero_ms, 5),
+            "bwd_ms": round(bwd_ms, 5),
+            "fwd_gsamples_per_s": round(samples_step / (fwd_ms * 1e-3) / 1e9, 4),
+            "step_ms_p10_p50_p90": [round(float(np.percentile(stepms, p)), 5) for p in (10, 50, 90)],
+            "hbm_frac_step": round(step_bytes / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "roofline": {
+                "kernel": dom,
+                "bound": "hbm",
+                "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"],
+                "peak_source": peaks["source"],
+                "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "bytes_per_launch": nbytes[dom],
+                "traffic": traffic,
+            },
+            "gpu_launches": 3 * args.steps,
+            "host_wall_s": round(wall, 3),
+            "clocks": clocks.summary(),
+        }
+        if want_nonfused:
+            result["nonfused"] = _time_nonfused(msda, t, w, nbytes, flush, min(args.steps, 50))
+        if not args.no_e2e:
+            result["e2e"] = _time_e2e(msda, x, t, w, step, flush, min(args.steps, 50), dev)
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        line = json.dumps(result)
+        print(line, flush=True)
+        if args.out:
+            with open(args.out, "a") as f:
+                f.write(line + "\n")
+    return result
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured (MEASURED_PEAKS.json)"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def _time_nonfused(msda, t, w, nbytes, flush, n):
+    """msda_forward / msda_backward (pre-computed locations and weights) on the
+    same workload: per-launch device times (L2 flushed before each)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    args = (t["value"], t["spatial_shapes"], t["level_start_index"], t["sampling_locations"],
+            t["attention_weights"])
+    out = torch.empty_like(t["grad_output"])
+    gv = torch.empty(t["value"].shape, dtype=torch.float32, device=t["value"].device)
+    gl = torch.empty_like(t["sampling_locations"])
+    ga = torch.empty_like(t["attention_weights"])
+    f, b = [], []
+    for i in range(n + 3):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.fill_(float(i))
+        e[0].record(stream)
+        msda.forward(*args, out=out)
+        e[1].record(stream)
+        msda.zero_grads(gv)
+        flush.fill_(float(i + 1))
+        e[2].record(stream)
+        msda.backward(*args, t["grad_output"], grad_value=gv, grad_sampling_locations=gl,
+                      grad_attention_weights=ga, accumulate=True)
+        e[3].record(stream)
+        if i >= 3:
+            f.append(e)
+    torch.cuda.synchronize()
+    fwd = statistics.mean(e[0].elapsed_time(e[1]) for e in f)
+    bwd = statistics.mean(e[2].elapsed_time(e[3]) for e in f)
+    peak = _peaks()["hbm_gbs"]
+    return {"fwd_ms": round(fwd, 5), "bwd_ms": round(bwd, 5),
+            "fwd_hbm_frac": round(nbytes["forward"] / (fwd * 1e-3) / 1e9 / peak, 4),
+            "bwd_hbm_frac": round(nbytes["backward"] / (bwd * 1e-3) / 1e9 / peak, 4),
+            "fwd_gsamples_per_s": round(w.samples / (fwd * 1e-3) / 1e9, 4), "launches": n}
+
+
+def _time_e2e(msda, x, t, w, step, flush, n, dev):
+    """The same step through the public API with host buffers: every step
+    copies its inputs from pinned host memory and its results back."""
+    import torch
+    stream = torch.cuda.current_stream()
+    hin = _pinned(x)
+    din = {k: torch.empty_like(v, device=dev) for k, v in hin.items()}
+    res_names = ["out", "grad_value", "grad_reference_points", "grad_sampling_offsets",
+                 "grad_attention_logits"]
+    B, S, Q, M, D, L, K = w.B, w.S, w.num_queries, w.M, w.D, w.L, w.K
+    dt = t["value"].dtype
+    hout = {
+        "out": torch.empty((B, Q, M, D), dtype=dt).pin_memory(),
+        "grad_value": torch.empty((B, S, M, D), dtype=torch.float32).pin_memory(),
+        "grad_reference_points": torch.empty((B, Q, 2), dtype=torch.float32).pin_memory(),
+        "grad_sampling_offsets": torch.empty((B, Q, M, L, K, 2), dtype=torch.float32).pin_memory(),
+        "grad_attention_logits": torch.empty((B, Q, M, L * K), dtype=torch.float32).pin_memory(),
+    }
+    h2d = sum(v.numel() * v.element_size() for v in hin.values())
+    d2h = sum(v.numel() * v.element_size() for v in hout.values())
+    times = []
+    for i in range(n + 2):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        flush.fill_(float(i))
+        e0.record(stream)
+        for k in hin:
+            din[k].copy_(hin[k], non_blocking=True)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        outs = step(ev, din)
+        for k in res_names:
+            hout[k].copy_(outs[k], non_blocking=True)
+        e1.record(stream)
+        if i >= 2:
+            times.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in times)
+    return {"value": round(w.samples / (ms * 1e-3) / 1e9, 4), "unit": UNIT,
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": n}
+
+
+# ------------------------------------------------------- the oracle legs --
+
+def _oracle_sample(w: wl.Workload, x: wl.Inputs, stride: int):
+    """Every `stride`-th query of the workload (all levels stay represented),
+    with the full value map: the inputs of a bounded oracle pass."""
+    qs = np.arange(0, w.num_queries, stride)
+    return {
+        "value": x.value_f64(), "grad_output": np.ascontiguousarray(x.grad_output_f64()[:, qs]),
+        "spatial_shapes": x.spatial_shapes, "level_start_index": x.level_start_index,
+        "reference_points": np.ascontiguousarray(x.reference_points[:, qs]),
+        "sampling_offsets": np.ascontiguousarray(x.sampling_offsets[:, qs]),
+        "attention_logits": np.ascontiguousarray(x.attention_logits[:, qs]),
+        "samples": w.B * len(qs) * w.M * w.L * w.K, "queries": len(qs),
+    }
+
+
+def _oracle_step(oracle, smp):
+    oracle.fused_forward(smp["value"], smp["spatial_shapes"], smp["level_start_index"],
+                         smp["reference_points"], smp["sampling_offsets"], smp["attention_logits"])
+    oracle.fused_backward(smp["value"], smp["spatial_shapes"], smp["level_start_index"],
+                          smp["reference_points"], smp["sampling_offsets"],
+                          smp["attention_logits"], smp["grad_output"])
+
+
+def cpu_baseline(w: wl.Workload, x: wl.Inputs, seconds: float) -> dict:
+    """The fp64 oracle (plain C loops, one thread), fused forward + backward on
+    a bounded sample of the workload, timed on this host's cores."""
+    import oracle
+    oracle.build()
+    stride = max(1, int(round(w.num_queries / 2048)))
+    smp = _oracle_sample(w, x, stride)
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        _oracle_step(oracle, smp)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    rate = smp["samples"] * passes / el
+    return {"value": round(rate / 1e9, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"every {stride}th query ({smp['queries']} of {w.num_queries}, "
+                      f"{smp['samples']} samples) x {passes} passes of fused fwd+bwd, "
+                      f"{el:.1f} s", "host_cpus": os.cpu_count(),
+            "full_step_ms_extrapolated": round(w.samples / rate * 1e3, 1)}
+
+
+def run_reference(args):
+    """The reference arm: the oracle, as it stands, on the host cores, each
+    step a bounded sample of the workload (rank 0 only)."""
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    w = wl.WORKLOADS[args.workload]
+    x = wl.generate(w, with_nonfused=False)
+    # size the per-step sample so that warm-up + steps stay within ~2 minutes
+    probe = _oracle_sample(w, x, max(1, w.num_queries // 256))
+    t0 = time.perf_counter()
+    _oracle_step(oracle, probe)
+    per_sample = (time.perf_counter() - t0) / probe["samples"]
+    budget = 120.0 / (args.steps + args.warmup)
+    want = max(64 * w.M * w.L * w.K * w.B, budget / per_sample)
+    stride = max(1, int(np.ceil(w.samples / want)))
+    smp = _oracle_sample(w, x, stride)
+    for _ in range(args.warmup):
+        _oracle_step(oracle, smp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(oracle, smp)
+    el = time.perf_counter() - t0
+    rate = smp["samples"] * args.steps / el
+    value = rate / 1e9
+    sample = (f"every {stride}th query ({smp['queries']} of {w.num_queries}, {smp['samples']} "
+              f"samples) per step, fused fwd+bwd")
+    result = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(w.samples / rate * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded SplitMix64 + Box-Muller draws (no dataset)",
+        "config": {"workload": w.name, "B": w.B, "levels_HW": [list(l) for l in w.levels],
+                   "Q": w.num_queries, "M": w.M, "D": w.D, "L": w.L, "K": w.K,
+                   "step": "oracle fused_forward + fused_backward (fp64 C loops)",
+                   "parallelism": "one host thread"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    line = json.dumps(result)
+    print(line, flush=True)
+    if args.out:
+        with open(args.out, "a") as f:
+            f.write(line + "\n")
+    return result
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+/*
+ * msda.h -- C ABI of the B200 (sm_100a) multi-scale deformable attention core.
+ *
+ * The operator (Deformable DETR's MSDeformAttn without its linear
+ * projections).  For every batch b, query q and head m:
+ *
+ *   out[b,q,m,:] = sum_{l<L} sum_{k<K} A[b,q,m,l,k] * x^l_m( loc[b,q,m,l,k] )
+ *
+ * where x^l_m(p) bilinearly samples head m of level l of the flattened value
+ * map at the normalized point p = (x, y) in [0,1]^2.  Sources (web pages on
+ * the operator, cited by page and section):
+ *   - the multi-scale sum and the level map phi_l:
+ *       discosf.com/news/5175395 §2.2; cf-1.com/news/4799680 §3.1
+ *   - sum over levels and points of A equals 1 (softmax over L*K):
+ *       cf-1.com/news/4799680 §3.1-3.2; x-humanoid.csdn.net MSDA explainer §3
+ *   - the flattened value [B, sum H_l*W_l, M, D] with spatial_shapes (H, W)
+ *     and level_start_index: cf-1.com/news/4799680 §3.3 and §5.3
+ *   - locations = reference_points + offsets / (W_l, H_l), offsets in level
+ *     pixels without a sigmoid: cf-1.com/news/4799680 §3.2
+ *   - bilinear sampling, pixel coordinate x = loc_x * W - 0.5 (grid_sample
+ *     with align_corners=False on grid = 2*loc - 1), out-of-range corners
+ *     masked to zero: cf-1.com/news/4799680 §5.3;
+ *     x-humanoid.csdn.net MSDA explainer §3 note 2;
+ *     discosf.com/news/5175395 §2.1-2.2
+ * Readings taken where the pages are silent: a sample is taken only when
+ * -1 < x < W and -1 < y < H (else it contributes 0 and has zero gradients);
+ * at an integer coordinate the derivative is the one of the cell floor(x);
+ * the backward pass is the exact derivative of the sum above.
+ *
+ * Conventions for every entry point
+ *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *     row-major, each 16-byte aligned.  The library keeps no pointer after
+ *     the call returns and allocates no memory.
+ *   - value, output and grad_output hold value_dtype elements (float32 or
+ *     bfloat16); every other floating-point tensor is float32.  Accumulation
+ *     is float32.
+ *   - Locations and offsets are (x, y) pairs; spatial_shapes rows are (H, W).
+ *   - spatial_shapes [L,2] and level_start_index [L] are int64 device arrays.
+ *     Their consistency (H, W >= 1, start[0] = 0, start[l+1] = start[l] +
+ *     H_l*W_l, sum = S) is checked by the kernels themselves: on a mismatch the
+ *     work is skipped, outputs are left unspecified, and a code is recorded in
+ *     a per-device status word that msda_get_device_status() returns.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream).  The
+ *     host-side checks below run before anything is enqueued; a call that
+ *     returns an error has enqueued nothing.
+ *   - Supported sizes: D (head_dim) in {8, 16, 32, 64, 128, 256};
+ *     1 <= L <= 16; 1 <= K <= 32; L*K <= 128; 1 <= M; S < 2^27;
+ *     B*Q*M*L*K < 2^40; B or Q may be 0 (nothing to sample).
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef MSDA_H_
+#define MSDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSDA_API __attribute__((visibility("default")))
+#else
+#define MSDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; declared here so that callers need
+ * no CUDA header. */
+typedef struct CUstream_st *msda_stream_t;
+
+typedef enum msda_status {
+    MSDA_OK = 0,
+    MSDA_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad size */
+    MSDA_ERR_UNSUPPORTED = 2,   /* valid, but outside the supported sizes */
+    MSDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    MSDA_ERR_DEVICE_CHECK = 4   /* a kernel found inconsistent geometry */
+} msda_status;
+
+typedef enum msda_dtype {
+    MSDA_F32 = 0,
+    MSDA_BF16 = 1
+} msda_dtype;
+
+/* msda_problem.flags */
+#define MSDA_GRAD_VALUE_BF16 (1u << 0) /* backward writes grad_value as bf16;
+                                          needs a float32 workspace */
+#define MSDA_ACCUMULATE_GRADS (1u << 1) /* backward adds into grad_value (and
+                                          grad_reference_points) instead of
+                                          zeroing them first; float32 only */
+
+/* Sizes of one call.  S = sum_l H_l * W_l. */
+typedef struct msda_problem {
+    int64_t batch;        /* B */
+    int64_t num_keys;     /* S */
+    int64_t num_queries;  /* Q */
+    int32_t num_heads;    /* M */
+    int32_t head_dim;     /* D */
+    int32_t num_levels;   /* L */
+    int32_t num_points;   /* K */
+    int32_t value_dtype;  /* msda_dtype of value, output, grad_output */
+    uint32_t flags;       /* MSDA_* flags above */
+} msda_problem;
+
+/*
+ * Forward of the core operator (discosf.com/news/5175395 §2.2;
+ * cf-1.com/news/4799680 §3.1 and the argument list of §5.3).
+ *   value               [B, S, M, D]        value_dtype
+ *   spatial_shapes      [L, 2] int64        (H_l, W_l)
+ *   level_start_index   [L]    int64
+ *   sampling_locations  [B, Q, M, L, K, 2]  float32, normalized (x, y)
+ *   attention_weights   [B, Q, M, L, K]     float32 (used as given; the
+ *                                            operator does not renormalize)
+ *   output              [B, Q, M, D]        value_dtype, overwritten
+ */
+MSDA_API msda_status msda_forward(const msda_problem *problem, const void *value,
+                         const int64_t *spatial_shapes, const int64_t *level_start_index,
+                         const float *sampling_locations, const float *attention_weights,
+                         void *output, msda_stream_t stream);
+
+/*
+ * Backward of the core operator: the exact derivative of msda_forward
+ * (bilinear sampling is differentiable in the coordinates,
+ * discosf.com/news/5175395 §2.1).  Inputs as msda_forward plus
+ *   grad_output              [B, Q, M, D]       value_dtype
+ * Outputs, all overwritten:
+ *   grad_value               [B, S, M, D]       float32 (bf16 with
+ *                                               MSDA_GRAD_VALUE_BF16)
+ *   grad_sampling_locations  [B, Q, M, L, K, 2] float32
+ *   grad_attention_weights   [B, Q, M, L, K]    float32
+ * grad_value is zeroed and then accumulated with float32 atomics, so its
+ * summation order (and its last bits) vary from run to run.  With
+ * MSDA_ACCUMULATE_GRADS the zero-fill is skipped and the gradients are added to
+ * what grad_value holds (not allowed together with MSDA_GRAD_VALUE_BF16).
+ * workspace: with MSDA_GRAD_VALUE_BF16, at least msda_backward_workspace_size()
+ * bytes of device memory that the call may overwrite; otherwise ignored (may
+ * be NULL).
+ */
+MSDA_API msda_status msda_backward(const msda_problem *problem, const void *value,
+                          const int64_t *spatial_shapes, const int64_t *level_start_index,
+                          const float *sampling_locations, const float *attention_weights,
+                          const void *grad_output, void *grad_value,
+                          float *grad_sampling_locations, float *grad_attention_weights,
+                          void *workspace, size_t workspace_bytes, msda_stream_t stream);
+
+/*
+ * Fused forward: computes the sampling locations and the attention softmax
+ * inside the kernel (cf-1.com/news/4799680 §3.2):
+ *   loc[b,q,m,l,k] = reference_points[b,q] + sampling_offsets[b,q,m,l,k] / (W_l, H_l)
+ *   A[b,q,m,:]     = softmax(attention_logits[b,q,m,:])   over the L*K points
+ * then the forward sum.
+ *   reference_points    [B, Q, 2]          float32, normalized (x, y), shared
+ *                                          by every level and head
+ *   sampling_offsets    [B, Q, M, L, K, 2] float32, pixels of level l
+ *   attention_logits    [B, Q, M, L*K]     float32
+ *   output              [B, Q, M, D]       value_dtype, overwritten
+ *   attention_weights_out [B, Q, M, L, K]  float32 or NULL: the softmax, if
+ *                                          the caller wants it
+ */
+MSDA_API msda_status msda_fused_forward(const msda_problem *problem, const void *value,
+                               const int64_t *spatial_shapes, const int64_t *level_start_index,
+                               const float *reference_points, const float *sampling_offsets,
+                               const float *attention_logits, void *output,
+                               float *attention_weights_out, msda_stream_t stream);
+
+/*
+ * Fused backward: msda_backward followed by the chain rule through the
+ * location and softmax steps of msda_fused_forward:
+ *   grad_sampling_offsets = grad_loc / (W_l, H_l)
+ *   grad_reference_points = sum over (m, l, k) of grad_loc   (NULL: skipped)
+ *   grad_attention_logits = A * (grad_A - sum_j A_j grad_A_j)
+ * Inputs as msda_fused_forward plus grad_output [B, Q, M, D] (value_dtype).
+ * Outputs (overwritten): grad_value as in msda_backward, grad_reference_points
+ * [B, Q, 2], grad_sampling_offsets [B, Q, M, L, K, 2], grad_attention_logits
+ * [B, Q, M, L*K], all float32 except grad_value with MSDA_GRAD_VALUE_BF16.
+ * grad_reference_points is accumulated with atomics over the M heads; like
+ * grad_value it is zeroed first unless MSDA_ACCUMULATE_GRADS is set.
+ */
+MSDA_API msda_status msda_fused_backward(const msda_problem *problem, const void *value,
+                                const int64_t *spatial_shapes, const int64_t *level_start_index,
+                                const float *reference_points, const float *sampling_offsets,
+                                const float *attention_logits, const void *grad_output,
+                                void *grad_value, float *grad_reference_points,
+                                float *grad_sampling_offsets, float *grad_attention_logits,
+                                void *workspace, size_t workspace_bytes, msda_stream_t stream);
+
+/*
+ * Zeroes the float32 accumulators of a backward call: grad_value
+ * [B, S, M, D] and, if not NULL, grad_reference_points [B, Q, 2].  Together
+ * with MSDA_ACCUMULATE_GRADS this splits the zero-fill from the backward
+ * kernel (e.g. to accumulate several backward calls into one buffer).
+ */
+MSDA_API msda_status msda_zero_grads(const msda_problem *problem, float *grad_value,
+                                     float *grad_reference_points, msda_stream_t stream);
+
+/* Bytes of workspace msda_backward / msda_fused_backward need for `problem`
+ * (0 unless MSDA_GRAD_VALUE_BF16 is set).  Host only; enqueues nothing. */
+MSDA_API msda_status msda_backward_workspace_size(const msda_problem *problem, size_t *bytes);
+
+/*
+ * Synchronizes `stream`, then returns in *code the status the kernels recorded
+ * on the current device since the last call (MSDA_OK or
+ * MSDA_ERR_DEVICE_CHECK), and clears it.  Returns MSDA_ERR_CUDA if the
+ * synchronization or the read fails.
+ */
+MSDA_API msda_status msda_get_device_status(msda_stream_t stream, int32_t *code);
+
+/* Static English description of a status code. */
+MSDA_API const char *msda_status_string(msda_status status);
+
+/* Library version, e.g. "0.1.0". */
+MSDA_API const char *msda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSDA_H_ */

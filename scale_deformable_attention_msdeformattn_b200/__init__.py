@@ -1,0 +1,21 @@
+"""B200-native (sm_100a) multi-scale deformable attention core.
+
+The operator runs in libmsda.so (hand-written CUDA kernels behind the C ABI of
+include/msda.h); this package is its Python binding.  PyTorch only provides
+device memory and the current stream.
+"""
+from .binding import (  # noqa: F401
+    MsdaError,
+    MSDeformAttnFunction,
+    MSDeformAttnFusedFunction,
+    backward,
+    device_status,
+    forward,
+    fused_backward,
+    fused_forward,
+    ms_deform_attn,
+    version,
+    zero_grads,
+)
+
+__version__ = "0.1.0"

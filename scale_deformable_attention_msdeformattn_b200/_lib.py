@@ -1,0 +1,82 @@
+"""ctypes view of libmsda.so (include/msda.h).  Argument marshalling only."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmsda.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "msda.h")
+
+MSDA_OK = 0
+MSDA_ERR_INVALID_ARG = 1
+MSDA_ERR_UNSUPPORTED = 2
+MSDA_ERR_CUDA = 3
+MSDA_ERR_DEVICE_CHECK = 4
+
+MSDA_F32 = 0
+MSDA_BF16 = 1
+
+MSDA_GRAD_VALUE_BF16 = 1 << 0
+MSDA_ACCUMULATE_GRADS = 1 << 1
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("num_keys", ctypes.c_int64),
+        ("num_queries", ctypes.c_int64),
+        ("num_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("num_levels", ctypes.c_int32),
+        ("num_points", ctypes.c_int32),
+        ("value_dtype", ctypes.c_int32),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
+_P = ctypes.c_void_p
+_PROB = ctypes.POINTER(Problem)
+_SIGNATURES = {
+    "msda_forward": [_PROB, _P, _P, _P, _P, _P, _P, _P],
+    "msda_backward": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "msda_fused_forward": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "msda_fused_backward": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "msda_backward_workspace_size": [_PROB, ctypes.POINTER(ctypes.c_size_t)],
+    "msda_zero_grads": [_PROB, _P, _P, _P],
+    "msda_get_device_status": [_P, ctypes.POINTER(ctypes.c_int32)],
+    "msda_status_string": [ctypes.c_int],
+    "msda_version": [],
+}
+
+_lib = None
+_lock = threading.Lock()
+
+
+def declared_functions(header: str = HEADER):
+    """Names of the functions include/msda.h declares."""
+    text = open(header).read()
+    return sorted(set(re.findall(r"^\s*MSDA_API\s+(?:const\s+)?[a-z_]+\s*\*?\s*(msda_[a-z_0-9]+)\s*\(", text, re.M)))
+
+
+def load(path: str = LIB_PATH):
+    """Loads libmsda.so; raises if it was not built (there is no fallback)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                "libmsda.so is missing (%s): build it with "
+                "`python -m scale_deformable_attention_msdeformattn_b200.build`" % path)
+        lib = ctypes.CDLL(path)
+        for name, args in _SIGNATURES.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        lib.msda_status_string.restype = ctypes.c_char_p
+        lib.msda_version.restype = ctypes.c_char_p
+        _lib = lib
+        return lib

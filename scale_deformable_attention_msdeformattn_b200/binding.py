@@ -1,0 +1,326 @@
+"""Python binding of the C-ABI: torch tensors in, libmsda.so calls, tensors out.
+
+Only argument marshalling happens here (shape and dtype checks, output
+allocation through PyTorch, pointer and stream hand-off).  Every step of the
+operator runs in the CUDA kernels of libmsda.so; there is no CPU or PyTorch
+fallback, and a missing library raises.
+
+Layouts follow the operator's conventional argument list (cf-1.com/news/4799680
+§5.3, x-humanoid.csdn.net MSDA explainer §3):
+  value               [B, S, M, D]        float32 or bfloat16
+  spatial_shapes      [L, 2]  int64 (H, W)
+  level_start_index   [L]     int64
+  sampling_locations  [B, Q, M, L, K, 2]  float32, normalized (x, y)
+  attention_weights   [B, Q, M, L, K]     float32
+  reference_points    [B, Q, 2]           float32 (fused variant)
+  sampling_offsets    [B, Q, M, L, K, 2]  float32, level pixels (fused variant)
+  attention_logits    [B, Q, M, L*K] or [B, Q, M, L, K] float32 (fused variant)
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+
+class MsdaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _lib.load()
+        msg = lib.msda_status_string(status).decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != _lib.MSDA_OK:
+        raise MsdaError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr()) if t.numel() > 0 else None
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+_DTYPES = {torch.float32: _lib.MSDA_F32, torch.bfloat16: _lib.MSDA_BF16}
+
+
+def _problem(value: torch.Tensor, Q: int, L: int, K: int, flags: int = 0) -> _lib.Problem:
+    if value.dim() != 4:
+        raise ValueError("value must be [B, S, M, D]")
+    if value.dtype not in _DTYPES:
+        raise TypeError("value must be float32 or bfloat16")
+    B, S, M, D = value.shape
+    return _lib.Problem(B, S, Q, M, D, L, K, _DTYPES[value.dtype], flags)
+
+
+def _geometry(value, spatial_shapes, level_start_index):
+    _need(spatial_shapes, "spatial_shapes", torch.int64, device=value.device)
+    if spatial_shapes.dim() != 2 or spatial_shapes.shape[1] != 2:
+        raise ValueError("spatial_shapes must be [L, 2]")
+    L = spatial_shapes.shape[0]
+    _need(level_start_index, "level_start_index", torch.int64, (L,), device=value.device)
+    return L
+
+
+def forward(value: torch.Tensor, spatial_shapes: torch.Tensor, level_start_index: torch.Tensor,
+            sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
+            out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """msda_forward: returns out [B, Q, M, D] in value's dtype."""
+    _need(value, "value", None)
+    L = _geometry(value, spatial_shapes, level_start_index)
+    B, S, M, D = value.shape
+    if sampling_locations.dim() != 6:
+        raise ValueError("sampling_locations must be [B, Q, M, L, K, 2]")
+    Q, K = sampling_locations.shape[1], sampling_locations.shape[4]
+    _need(sampling_locations, "sampling_locations", torch.float32, (B, Q, M, L, K, 2), value.device)
+    _need(attention_weights, "attention_weights", torch.float32, (B, Q, M, L, K), value.device)
+    if out is None:
+        out = torch.empty((B, Q, M, D), dtype=value.dtype, device=value.device)
+    _need(out, "out", value.dtype, (B, Q, M, D), value.device)
+    prob = _problem(value, Q, L, K)
+    st = _lib.load().msda_forward(ctypes.byref(prob), _ptr(value), _ptr(spatial_shapes),
+                                  _ptr(level_start_index), _ptr(sampling_locations),
+                                  _ptr(attention_weights), _ptr(out), _stream())
+    _check(st, "msda_forward")
+    return out
+
+
+def backward(value, spatial_shapes, level_start_index, sampling_locations, attention_weights,
+             grad_output, grad_value_dtype=torch.float32,
+             grad_value: Optional[torch.Tensor] = None,
+             grad_sampling_locations: Optional[torch.Tensor] = None,
+             grad_attention_weights: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None,
+             accumulate: bool = False) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """msda_backward: (grad_value, grad_sampling_locations, grad_attention_weights).
+
+    accumulate=True adds into the given float32 grad_value instead of
+    overwriting it (MSDA_ACCUMULATE_GRADS)."""
+    _need(value, "value", None)
+    L = _geometry(value, spatial_shapes, level_start_index)
+    B, S, M, D = value.shape
+    Q, K = sampling_locations.shape[1], sampling_locations.shape[4]
+    dev = value.device
+    _need(sampling_locations, "sampling_locations", torch.float32, (B, Q, M, L, K, 2), dev)
+    _need(attention_weights, "attention_weights", torch.float32, (B, Q, M, L, K), dev)
+    _need(grad_output, "grad_output", value.dtype, (B, Q, M, D), dev)
+    flags = _lib.MSDA_GRAD_VALUE_BF16 if grad_value_dtype == torch.bfloat16 else 0
+    if grad_value_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("grad_value_dtype must be float32 or bfloat16")
+    if accumulate:
+        if grad_value is None:
+            raise ValueError("accumulate=True needs the grad_value buffer to add into")
+        flags |= _lib.MSDA_ACCUMULATE_GRADS
+    if grad_value is None:
+        grad_value = torch.empty((B, S, M, D), dtype=grad_value_dtype, device=dev)
+    if grad_sampling_locations is None:
+        grad_sampling_locations = torch.empty((B, Q, M, L, K, 2), dtype=torch.float32, device=dev)
+    if grad_attention_weights is None:
+        grad_attention_weights = torch.empty((B, Q, M, L, K), dtype=torch.float32, device=dev)
+    _need(grad_value, "grad_value", grad_value_dtype, (B, S, M, D), dev)
+    prob = _problem(value, Q, L, K, flags)
+    lib = _lib.load()
+    ws_bytes = ctypes.c_size_t(0)
+    _check(lib.msda_backward_workspace_size(ctypes.byref(prob), ctypes.byref(ws_bytes)),
+           "msda_backward_workspace_size")
+    if ws_bytes.value and workspace is None:
+        workspace = torch.empty(ws_bytes.value, dtype=torch.uint8, device=dev)
+    st = lib.msda_backward(ctypes.byref(prob), _ptr(value), _ptr(spatial_shapes),
+                           _ptr(level_start_index), _ptr(sampling_locations),
+                           _ptr(attention_weights), _ptr(grad_output), _ptr(grad_value),
+                           _ptr(grad_sampling_locations), _ptr(grad_attention_weights),
+                           _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                           _stream())
+    _check(st, "msda_backward")
+    return grad_value, grad_sampling_locations, grad_attention_weights
+
+
+def _logits(attention_logits, B, Q, M, L, K, dev):
+    if attention_logits.dim() == 5:
+        attention_logits = attention_logits.reshape(B, Q, M, L * K)
+    return _need(attention_logits, "attention_logits", torch.float32, (B, Q, M, L * K), dev)
+
+
+def fused_forward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
+                  attention_logits, return_attention_weights: bool = False,
+                  out: Optional[torch.Tensor] = None):
+    """msda_fused_forward: out [B, Q, M, D] (and the softmax weights if asked)."""
+    _need(value, "value", None)
+    L = _geometry(value, spatial_shapes, level_start_index)
+    B, S, M, D = value.shape
+    if sampling_offsets.dim() != 6:
+        raise ValueError("sampling_offsets must be [B, Q, M, L, K, 2]")
+    Q, K = sampling_offsets.shape[1], sampling_offsets.shape[4]
+    dev = value.device
+    _need(reference_points, "reference_points", torch.float32, (B, Q, 2), dev)
+    _need(sampling_offsets, "sampling_offsets", torch.float32, (B, Q, M, L, K, 2), dev)
+    attention_logits = _logits(attention_logits, B, Q, M, L, K, dev)
+    if out is None:
+        out = torch.empty((B, Q, M, D), dtype=value.dtype, device=dev)
+    _need(out, "out", value.dtype, (B, Q, M, D), dev)
+    attn = torch.empty((B, Q, M, L, K), dtype=torch.float32, device=dev) if return_attention_weights else None
+    prob = _problem(value, Q, L, K)
+    st = _lib.load().msda_fused_forward(ctypes.byref(prob), _ptr(value), _ptr(spatial_shapes),
+                                        _ptr(level_start_index), _ptr(reference_points),
+                                        _ptr(sampling_offsets), _ptr(attention_logits), _ptr(out),
+                                        _ptr(attn), _stream())
+    _check(st, "msda_fused_forward")
+    return (out, attn) if return_attention_weights else out
+
+
+def fused_backward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
+                   attention_logits, grad_output, grad_value_dtype=torch.float32,
+                   want_grad_reference_points: bool = True,
+                   grad_value: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
+                   accumulate: bool = False,
+                   grad_reference_points: Optional[torch.Tensor] = None,
+                   grad_sampling_offsets: Optional[torch.Tensor] = None,
+                   grad_attention_logits: Optional[torch.Tensor] = None):
+    """msda_fused_backward: (grad_value, grad_reference_points or None,
+    grad_sampling_offsets, grad_attention_logits [B, Q, M, L*K]).
+
+    accumulate=True adds into the given float32 grad_value (and
+    grad_reference_points) instead of overwriting them."""
+    _need(value, "value", None)
+    L = _geometry(value, spatial_shapes, level_start_index)
+    B, S, M, D = value.shape
+    Q, K = sampling_offsets.shape[1], sampling_offsets.shape[4]
+    dev = value.device
+    _need(reference_points, "reference_points", torch.float32, (B, Q, 2), dev)
+    _need(sampling_offsets, "sampling_offsets", torch.float32, (B, Q, M, L, K, 2), dev)
+    attention_logits = _logits(attention_logits, B, Q, M, L, K, dev)
+    _need(grad_output, "grad_output", value.dtype, (B, Q, M, D), dev)
+    if grad_value_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("grad_value_dtype must be float32 or bfloat16")
+    flags = _lib.MSDA_GRAD_VALUE_BF16 if grad_value_dtype == torch.bfloat16 else 0
+    if accumulate:
+        if grad_value is None or (want_grad_reference_points and grad_reference_points is None):
+            raise ValueError("accumulate=True needs the buffers to add into")
+        flags |= _lib.MSDA_ACCUMULATE_GRADS
+    if grad_value is None:
+        grad_value = torch.empty((B, S, M, D), dtype=grad_value_dtype, device=dev)
+    _need(grad_value, "grad_value", grad_value_dtype, (B, S, M, D), dev)
+    gref = None
+    if want_grad_reference_points:
+        gref = grad_reference_points if grad_reference_points is not None else \
+            torch.empty((B, Q, 2), dtype=torch.float32, device=dev)
+        _need(gref, "grad_reference_points", torch.float32, (B, Q, 2), dev)
+    goff = grad_sampling_offsets if grad_sampling_offsets is not None else \
+        torch.empty((B, Q, M, L, K, 2), dtype=torch.float32, device=dev)
+    _need(goff, "grad_sampling_offsets", torch.float32, (B, Q, M, L, K, 2), dev)
+    glog = grad_attention_logits if grad_attention_logits is not None else \
+        torch.empty((B, Q, M, L * K), dtype=torch.float32, device=dev)
+    _need(glog, "grad_attention_logits", torch.float32, (B, Q, M, L * K), dev)
+    prob = _problem(value, Q, L, K, flags)
+    lib = _lib.load()
+    ws_bytes = ctypes.c_size_t(0)
+    _check(lib.msda_backward_workspace_size(ctypes.byref(prob), ctypes.byref(ws_bytes)),
+           "msda_backward_workspace_size")
+    if ws_bytes.value and workspace is None:
+        workspace = torch.empty(ws_bytes.value, dtype=torch.uint8, device=dev)
+    st = lib.msda_fused_backward(ctypes.byref(prob), _ptr(value), _ptr(spatial_shapes),
+                                 _ptr(level_start_index), _ptr(reference_points),
+                                 _ptr(sampling_offsets), _ptr(attention_logits), _ptr(grad_output),
+                                 _ptr(grad_value), _ptr(gref), _ptr(goff), _ptr(glog),
+                                 _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                 _stream())
+    _check(st, "msda_fused_backward")
+    return grad_value, gref, goff, glog
+
+
+def zero_grads(grad_value: torch.Tensor, grad_reference_points: Optional[torch.Tensor] = None,
+               num_queries: int = 0, num_levels: int = 1, num_points: int = 1):
+    """msda_zero_grads: zeroes float32 grad_value [B, S, M, D] (and
+    grad_reference_points [B, Q, 2]) in a library kernel."""
+    _need(grad_value, "grad_value", torch.float32)
+    B, S, M, D = grad_value.shape
+    Q = grad_reference_points.shape[1] if grad_reference_points is not None else num_queries
+    if grad_reference_points is not None:
+        _need(grad_reference_points, "grad_reference_points", torch.float32, (B, Q, 2), grad_value.device)
+    prob = _lib.Problem(B, S, Q, M, D, num_levels, num_points, _lib.MSDA_F32, 0)
+    st = _lib.load().msda_zero_grads(ctypes.byref(prob), _ptr(grad_value), _ptr(grad_reference_points),
+                                     _stream())
+    _check(st, "msda_zero_grads")
+
+
+def device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronizes the stream and returns (and clears) the kernels' status word."""
+    s = ctypes.c_void_p((stream or torch.cuda.current_stream()).cuda_stream)
+    code = ctypes.c_int32(0)
+    _check(_lib.load().msda_get_device_status(s, ctypes.byref(code)), "msda_get_device_status")
+    return code.value
+
+
+def version() -> str:
+    return _lib.load().msda_version().decode()
+
+
+class MSDeformAttnFunction(torch.autograd.Function):
+    """Autograd wrapper over msda_forward / msda_backward (grad_value in the
+    value's dtype)."""
+
+    @staticmethod
+    def forward(ctx, value, spatial_shapes, level_start_index, sampling_locations, attention_weights):
+        ctx.save_for_backward(value, spatial_shapes, level_start_index, sampling_locations,
+                              attention_weights)
+        return forward(value, spatial_shapes, level_start_index, sampling_locations,
+                       attention_weights)
+
+    @staticmethod
+    def backward(ctx, grad_output):
+        value, shapes, starts, loc, attn = ctx.saved_tensors
+        gv, gl, ga = backward(value, shapes, starts, loc, attn, grad_output.contiguous(),
+                              grad_value_dtype=value.dtype)
+        return gv, None, None, gl, ga
+
+
+class MSDeformAttnFusedFunction(torch.autograd.Function):
+    """Autograd wrapper over msda_fused_forward / msda_fused_backward."""
+
+    @staticmethod
+    def forward(ctx, value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
+                attention_logits):
+        ctx.save_for_backward(value, spatial_shapes, level_start_index, reference_points,
+                              sampling_offsets, attention_logits)
+        return fused_forward(value, spatial_shapes, level_start_index, reference_points,
+                             sampling_offsets, attention_logits)
+
+    @staticmethod
+    def backward(ctx, grad_output):
+        value, shapes, starts, ref, off, logits = ctx.saved_tensors
+        gv, gref, goff, glog = fused_backward(value, shapes, starts, ref, off, logits,
+                                              grad_output.contiguous(), grad_value_dtype=value.dtype)
+        return gv, None, None, gref, goff, glog.reshape(logits.shape)
+
+
+def ms_deform_attn(value, spatial_shapes, level_start_index, sampling_locations, attention_weights):
+    """Differentiable core operator; output [B, Q, M*D] like the module's
+    reshape before output_proj."""
+    out = MSDeformAttnFunction.apply(value, spatial_shapes, level_start_index, sampling_locations,
+                                     attention_weights)
+    return out.flatten(2)

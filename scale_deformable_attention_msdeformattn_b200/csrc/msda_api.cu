@@ -1,0 +1,475 @@
+// msda_api.cu -- the C ABI declared in include/msda.h: argument checks, kernel
+// selection by (value dtype, head_dim), launch shapes, device status word.
+//
+// Launch shape.  Every compute kernel runs as one persistent wave: the grid is
+// (SM count) x (resident CTAs per SM, from the occupancy calculator), each CTA
+// owning a contiguous range of row tiles.  CTAs have up to 8 warps; fewer when
+// the shared-memory records of the L*K samples of each row would exceed the
+// per-CTA budget.
+#include "msda.h"
+#include "msda_kernels.cuh"
+
+#include <mutex>
+
+namespace {
+
+using msda::KernelArgs;
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kCtaSmemBudget = 96 * 1024;   // keeps >= 2 CTAs per SM
+constexpr size_t kForwardRecordBytes = sizeof(msda::Record);
+constexpr size_t kBackwardRecordBytes = sizeof(msda::Record) + 3 * sizeof(float);
+
+bool is_supported_head_dim(int d)
+{
+    return d == 8 || d == 16 || d == 32 || d == 64 || d == 128 || d == 256;
+}
+
+size_t elem_bytes(int32_t dtype) { return dtype == MSDA_BF16 ? 2 : 4; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A pointer may be null only when its tensor is empty.
+bool ptr_ok(const void *p, int64_t numel)
+{
+    if (numel == 0)
+        return p == nullptr || aligned16(p);
+    return p != nullptr && aligned16(p);
+}
+
+msda_status check_problem(const msda_problem *p)
+{
+    if (!p)
+        return MSDA_ERR_INVALID_ARG;
+    if (p->batch < 0 || p->num_queries < 0 || p->num_keys < 1 || p->num_heads < 1 ||
+        p->num_levels < 1 || p->num_points < 1 || p->head_dim < 1)
+        return MSDA_ERR_INVALID_ARG;
+    if (p->value_dtype != MSDA_F32 && p->value_dtype != MSDA_BF16)
+        return MSDA_ERR_INVALID_ARG;
+    if (p->flags & ~(uint32_t)(MSDA_GRAD_VALUE_BF16 | MSDA_ACCUMULATE_GRADS))
+        return MSDA_ERR_INVALID_ARG;
+    if ((p->flags & MSDA_GRAD_VALUE_BF16) && (p->flags & MSDA_ACCUMULATE_GRADS))
+        return MSDA_ERR_INVALID_ARG;
+    if (p->num_levels > msda::kMaxLevels || p->num_points > 32 ||
+        p->num_levels * p->num_points > 128)
+        return MSDA_ERR_UNSUPPORTED;
+    if (!is_supported_head_dim(p->head_dim))
+        return MSDA_ERR_UNSUPPORTED;
+    if (p->num_keys >= (int64_t(1) << 27))
+        return MSDA_ERR_UNSUPPORTED;
+    if ((int64_t)p->num_heads * p->head_dim * (int64_t)elem_bytes(p->value_dtype) >= (int64_t(1) << 31))
+        return MSDA_ERR_UNSUPPORTED;
+    // B * Q * M * L * K < 2^40, evaluated without overflow
+    const double samples = (double)p->batch * (double)p->num_queries * p->num_heads *
+                           p->num_levels * p->num_points;
+    if (samples >= 1099511627776.0)
+        return MSDA_ERR_UNSUPPORTED;
+    const double values = (double)p->batch * (double)p->num_keys * p->num_heads * p->head_dim;
+    if (values >= 9.0e18)
+        return MSDA_ERR_UNSUPPORTED;
+    return MSDA_OK;
+}
+
+struct DeviceInfo {
+    int sm_count = 0;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+
+msda_status current_device(int &dev, int &sm_count)
+{
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return MSDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_devices[dev].sm_count == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            return MSDA_ERR_CUDA;
+        g_devices[dev].sm_count = n;
+    }
+    sm_count = g_devices[dev].sm_count;
+    return MSDA_OK;
+}
+
+// Resident CTAs per SM of `kernel` for (threads, smem), cached per device.
+struct OccEntry {
+    const void *kernel;
+    int dev, threads;
+    size_t smem;
+    int blocks;
+};
+constexpr int kOccCache = 256;
+OccEntry g_occ[kOccCache];
+int g_occ_n = 0;
+
+msda_status occupancy(const void *kernel, int dev, int threads, size_t smem, int &blocks)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    for (int i = 0; i < g_occ_n; ++i) {
+        const OccEntry &e = g_occ[i];
+        if (e.kernel == kernel && e.dev == dev && e.threads == threads && e.smem == smem) {
+            blocks = e.blocks;
+            return MSDA_OK;
+        }
+    }
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, threads, smem) != cudaSuccess || b < 1)
+        return MSDA_ERR_CUDA;
+    if (g_occ_n < kOccCache)
+        g_occ[g_occ_n++] = OccEntry{kernel, dev, threads, smem, b};
+    blocks = b;
+    return MSDA_OK;
+}
+
+template <typename T, int D> constexpr int rows_per_warp() { return msda::Layout<T, D>::kRowsPerWarp; }
+
+// Launches one compute kernel over all rows as a persistent wave.
+msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, KernelArgs &a,
+                        cudaStream_t stream)
+{
+    int dev = 0, sms = 0;
+    msda_status st = current_device(dev, sms);
+    if (st != MSDA_OK)
+        return st;
+    const int P = a.L * a.K;
+    const size_t per_warp = (size_t)rpw * P * record_bytes;
+    int warps = (int)(kCtaSmemBudget / per_warp);
+    warps = warps < 1 ? 1 : (warps > msda::kMaxWarpsPerCta ? msda::kMaxWarpsPerCta : warps);
+    const size_t smem = per_warp * warps;
+    const int threads = warps * 32;
+    int blocks_per_sm = 0;
+    st = occupancy(kernel, dev, threads, smem, blocks_per_sm);
+    if (st != MSDA_OK)
+        return st;
+    a.rows_per_tile = (int64_t)warps * rpw;
+    a.ntiles = (a.rows + a.rows_per_tile - 1) / a.rows_per_tile;
+    int64_t ctas = (int64_t)sms * blocks_per_sm;
+    if (ctas > a.ntiles)
+        ctas = a.ntiles;
+    a.tiles_per_cta = (a.ntiles + ctas - 1) / ctas;
+    ctas = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+    void *params[] = {&a};
+    if (cudaLaunchKernel(kernel, dim3((unsigned)ctas), dim3(threads), params, smem, stream) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    return MSDA_OK;
+}
+
+msda_status launch_zero(float *a, int64_t na, float *b, int64_t nb, cudaStream_t stream)
+{
+    if (na == 0 && nb == 0)
+        return MSDA_OK;
+    int dev = 0, sms = 0;
+    msda_status st = current_device(dev, sms);
+    if (st != MSDA_OK)
+        return st;
+    int64_t work = na / 4 > nb ? na / 4 : nb;
+    int64_t blocks = (work + 255) / 256;
+    if (blocks > (int64_t)sms * 8)
+        blocks = (int64_t)sms * 8;
+    if (blocks < 1)
+        blocks = 1;
+    msda::zero_kernel<<<(unsigned)blocks, 256, 0, stream>>>(reinterpret_cast<float4 *>(a), na / 4, b, nb);
+    return cudaGetLastError() == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
+}
+
+msda_status launch_to_bf16(const float *src, void *dst, int64_t n, cudaStream_t stream)
+{
+    if (n == 0)
+        return MSDA_OK;
+    int dev = 0, sms = 0;
+    msda_status st = current_device(dev, sms);
+    if (st != MSDA_OK)
+        return st;
+    int64_t n8 = n / 8;
+    int64_t blocks = (n8 + 255) / 256;
+    if (blocks > (int64_t)sms * 8)
+        blocks = (int64_t)sms * 8;
+    msda::f32_to_bf16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        reinterpret_cast<const float4 *>(src), reinterpret_cast<uint4 *>(dst), n8);
+    return cudaGetLastError() == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
+}
+
+// Kernel selection -----------------------------------------------------------
+
+template <bool FUSED>
+msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
+{
+#define MSDA_FWD_CASE(T, DD)                                                                      \
+    case DD:                                                                                       \
+        return launch_rows((const void *)msda::forward_kernel<T, DD, FUSED>, rows_per_warp<T, DD>(), \
+                           kForwardRecordBytes, a, s);
+    if (p->value_dtype == MSDA_F32) {
+        switch (p->head_dim) {
+            MSDA_FWD_CASE(float, 8) MSDA_FWD_CASE(float, 16) MSDA_FWD_CASE(float, 32)
+            MSDA_FWD_CASE(float, 64) MSDA_FWD_CASE(float, 128) MSDA_FWD_CASE(float, 256)
+        }
+    } else {
+        switch (p->head_dim) {
+            MSDA_FWD_CASE(__nv_bfloat16, 8) MSDA_FWD_CASE(__nv_bfloat16, 16)
+            MSDA_FWD_CASE(__nv_bfloat16, 32) MSDA_FWD_CASE(__nv_bfloat16, 64)
+            MSDA_FWD_CASE(__nv_bfloat16, 128) MSDA_FWD_CASE(__nv_bfloat16, 256)
+        }
+    }
+#undef MSDA_FWD_CASE
+    return MSDA_ERR_UNSUPPORTED;
+}
+
+template <bool FUSED>
+msda_status launch_backward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
+{
+#define MSDA_BWD_CASE(T, DD)                                                                       \
+    case DD:                                                                                        \
+        return launch_rows((const void *)msda::backward_kernel<T, DD, FUSED>, rows_per_warp<T, DD>(), \
+                           kBackwardRecordBytes, a, s);
+    if (p->value_dtype == MSDA_F32) {
+        switch (p->head_dim) {
+            MSDA_BWD_CASE(float, 8) MSDA_BWD_CASE(float, 16) MSDA_BWD_CASE(float, 32)
+            MSDA_BWD_CASE(float, 64) MSDA_BWD_CASE(float, 128) MSDA_BWD_CASE(float, 256)
+        }
+    } else {
+        switch (p->head_dim) {
+            MSDA_BWD_CASE(__nv_bfloat16, 8) MSDA_BWD_CASE(__nv_bfloat16, 16)
+            MSDA_BWD_CASE(__nv_bfloat16, 32) MSDA_BWD_CASE(__nv_bfloat16, 64)
+            MSDA_BWD_CASE(__nv_bfloat16, 128) MSDA_BWD_CASE(__nv_bfloat16, 256)
+        }
+    }
+#undef MSDA_BWD_CASE
+    return MSDA_ERR_UNSUPPORTED;
+}
+
+KernelArgs base_args(const msda_problem *p, const void *value, const int64_t *shapes,
+                     const int64_t *starts)
+{
+    KernelArgs a = {};
+    a.value = value;
+    a.shapes = shapes;
+    a.starts = starts;
+    a.rows = p->batch * p->num_queries * p->num_heads;
+    a.S = p->num_keys;
+    a.Q = (int)p->num_queries;
+    a.M = p->num_heads;
+    a.L = p->num_levels;
+    a.K = p->num_points;
+    return a;
+}
+
+struct Sizes {
+    int64_t value, samples, rows_d, queries;
+};
+
+Sizes sizes_of(const msda_problem *p)
+{
+    Sizes z;
+    z.value = p->batch * p->num_keys * p->num_heads * p->head_dim;
+    z.samples = p->batch * p->num_queries * p->num_heads * p->num_levels * p->num_points;
+    z.rows_d = p->batch * p->num_queries * p->num_heads * p->head_dim;
+    z.queries = p->batch * p->num_queries;
+    return z;
+}
+
+bool geometry_ptrs_ok(const msda_problem *p, const int64_t *shapes, const int64_t *starts)
+{
+    (void)p;
+    return shapes != nullptr && starts != nullptr && aligned16(shapes) && aligned16(starts);
+}
+
+// Shared tail of both backward entry points: zero, run, convert.
+template <bool FUSED>
+msda_status run_backward(const msda_problem *p, KernelArgs &a, void *grad_value, void *workspace,
+                         size_t workspace_bytes, cudaStream_t s)
+{
+    const Sizes z = sizes_of(p);
+    const bool to_bf16 = (p->flags & MSDA_GRAD_VALUE_BF16) != 0;
+    float *acc = static_cast<float *>(grad_value);
+    if (to_bf16) {
+        if (workspace_bytes < (size_t)z.value * sizeof(float) || !ptr_ok(workspace, z.value))
+            return MSDA_ERR_INVALID_ARG;
+        acc = static_cast<float *>(workspace);
+    }
+    a.grad_value = acc;
+    msda_status st = MSDA_OK;
+    if (!(p->flags & MSDA_ACCUMULATE_GRADS)) {
+        st = launch_zero(acc, z.value, FUSED ? a.grad_ref : nullptr,
+                         (FUSED && a.grad_ref) ? z.queries * 2 : 0, s);
+        if (st != MSDA_OK)
+            return st;
+    }
+    if (a.rows > 0) {
+        st = launch_backward<FUSED>(p, a, s);
+        if (st != MSDA_OK)
+            return st;
+    }
+    if (to_bf16)
+        return launch_to_bf16(acc, grad_value, z.value, s);
+    return MSDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+msda_status msda_forward(const msda_problem *problem, const void *value,
+                         const int64_t *spatial_shapes, const int64_t *level_start_index,
+                         const float *sampling_locations, const float *attention_weights,
+                         void *output, msda_stream_t stream)
+{
+    msda_status st = check_problem(problem);
+    if (st != MSDA_OK)
+        return st;
+    const Sizes z = sizes_of(problem);
+    if (!ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
+        !ptr_ok(sampling_locations, z.samples * 2) || !ptr_ok(attention_weights, z.samples) ||
+        !ptr_ok(output, z.rows_d))
+        return MSDA_ERR_INVALID_ARG;
+    KernelArgs a = base_args(problem, value, spatial_shapes, level_start_index);
+    if (a.rows == 0)
+        return MSDA_OK;
+    a.loc = sampling_locations;
+    a.attn = attention_weights;
+    a.out = output;
+    return launch_forward<false>(problem, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_backward(const msda_problem *problem, const void *value,
+                          const int64_t *spatial_shapes, const int64_t *level_start_index,
+                          const float *sampling_locations, const float *attention_weights,
+                          const void *grad_output, void *grad_value,
+                          float *grad_sampling_locations, float *grad_attention_weights,
+                          void *workspace, size_t workspace_bytes, msda_stream_t stream)
+{
+    msda_status st = check_problem(problem);
+    if (st != MSDA_OK)
+        return st;
+    const Sizes z = sizes_of(problem);
+    if (!ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
+        !ptr_ok(sampling_locations, z.samples * 2) || !ptr_ok(attention_weights, z.samples) ||
+        !ptr_ok(grad_output, z.rows_d) || !ptr_ok(grad_value, z.value) ||
+        !ptr_ok(grad_sampling_locations, z.samples * 2) || !ptr_ok(grad_attention_weights, z.samples))
+        return MSDA_ERR_INVALID_ARG;
+    KernelArgs a = base_args(problem, value, spatial_shapes, level_start_index);
+    a.loc = sampling_locations;
+    a.attn = attention_weights;
+    a.grad_out = grad_output;
+    a.grad_loc = grad_sampling_locations;
+    a.grad_attn = grad_attention_weights;
+    return run_backward<false>(problem, a, grad_value, workspace, workspace_bytes,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_fused_forward(const msda_problem *problem, const void *value,
+                               const int64_t *spatial_shapes, const int64_t *level_start_index,
+                               const float *reference_points, const float *sampling_offsets,
+                               const float *attention_logits, void *output,
+                               float *attention_weights_out, msda_stream_t stream)
+{
+    msda_status st = check_problem(problem);
+    if (st != MSDA_OK)
+        return st;
+    const Sizes z = sizes_of(problem);
+    if (!ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
+        !ptr_ok(reference_points, z.queries * 2) || !ptr_ok(sampling_offsets, z.samples * 2) ||
+        !ptr_ok(attention_logits, z.samples) || !ptr_ok(output, z.rows_d) ||
+        (attention_weights_out && !aligned16(attention_weights_out)))
+        return MSDA_ERR_INVALID_ARG;
+    KernelArgs a = base_args(problem, value, spatial_shapes, level_start_index);
+    if (a.rows == 0)
+        return MSDA_OK;
+    a.ref = reference_points;
+    a.off = sampling_offsets;
+    a.logits = attention_logits;
+    a.out = output;
+    a.attn_out = attention_weights_out;
+    return launch_forward<true>(problem, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_fused_backward(const msda_problem *problem, const void *value,
+                                const int64_t *spatial_shapes, const int64_t *level_start_index,
+                                const float *reference_points, const float *sampling_offsets,
+                                const float *attention_logits, const void *grad_output,
+                                void *grad_value, float *grad_reference_points,
+                                float *grad_sampling_offsets, float *grad_attention_logits,
+                                void *workspace, size_t workspace_bytes, msda_stream_t stream)
+{
+    msda_status st = check_problem(problem);
+    if (st != MSDA_OK)
+        return st;
+    const Sizes z = sizes_of(problem);
+    if (!ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
+        !ptr_ok(reference_points, z.queries * 2) || !ptr_ok(sampling_offsets, z.samples * 2) ||
+        !ptr_ok(attention_logits, z.samples) || !ptr_ok(grad_output, z.rows_d) ||
+        !ptr_ok(grad_value, z.value) || !ptr_ok(grad_sampling_offsets, z.samples * 2) ||
+        !ptr_ok(grad_attention_logits, z.samples) ||
+        (grad_reference_points && !aligned16(grad_reference_points)))
+        return MSDA_ERR_INVALID_ARG;
+    KernelArgs a = base_args(problem, value, spatial_shapes, level_start_index);
+    a.ref = reference_points;
+    a.off = sampling_offsets;
+    a.logits = attention_logits;
+    a.grad_out = grad_output;
+    a.grad_ref = grad_reference_points;
+    a.grad_off = grad_sampling_offsets;
+    a.grad_logits = grad_attention_logits;
+    return run_backward<true>(problem, a, grad_value, workspace, workspace_bytes,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_zero_grads(const msda_problem *problem, float *grad_value,
+                            float *grad_reference_points, msda_stream_t stream)
+{
+    msda_status st = check_problem(problem);
+    if (st != MSDA_OK)
+        return st;
+    const Sizes z = sizes_of(problem);
+    if (!ptr_ok(grad_value, z.value) || (grad_reference_points && !aligned16(grad_reference_points)))
+        return MSDA_ERR_INVALID_ARG;
+    return launch_zero(grad_value, z.value, grad_reference_points,
+                       grad_reference_points ? z.queries * 2 : 0,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_backward_workspace_size(const msda_problem *problem, size_t *bytes)
+{
+    msda_status st = check_problem(problem);
+    if (st != MSDA_OK)
+        return st;
+    if (!bytes)
+        return MSDA_ERR_INVALID_ARG;
+    *bytes = (problem->flags & MSDA_GRAD_VALUE_BF16) ? (size_t)sizes_of(problem).value * sizeof(float) : 0;
+    return MSDA_OK;
+}
+
+msda_status msda_get_device_status(msda_stream_t stream, int32_t *code)
+{
+    if (!code)
+        return MSDA_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, msda::g_device_status, sizeof(int)) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(msda::g_device_status, &zero, sizeof(int)) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    *code = v;
+    return MSDA_OK;
+}
+
+const char *msda_status_string(msda_status status)
+{
+    switch (status) {
+    case MSDA_OK: return "success";
+    case MSDA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or bad size)";
+    case MSDA_ERR_UNSUPPORTED: return "sizes outside the supported range";
+    case MSDA_ERR_CUDA: return "CUDA runtime error";
+    case MSDA_ERR_DEVICE_CHECK: return "kernel found inconsistent spatial_shapes / level_start_index";
+    }
+    return "unknown status";
+}
+
+const char *msda_version(void) { return "0.1.0"; }
+
+}  // extern "C"

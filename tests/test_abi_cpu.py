@@ -1,0 +1,108 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+function include/msda.h declares, and its host-side argument checks reject bad
+calls before any CUDA call is made (no compute happens here)."""
+import ctypes
+
+import pytest
+
+from scale_deformable_attention_msdeformattn_b200 import _lib
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from scale_deformable_attention_msdeformattn_b200 import build
+    build.build()
+    return _lib.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _lib.declared_functions()
+    assert {"msda_forward", "msda_backward", "msda_fused_forward", "msda_fused_backward",
+            "msda_zero_grads", "msda_backward_workspace_size", "msda_get_device_status",
+            "msda_status_string", "msda_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(_lib._SIGNATURES) >= set(names)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.msda_version().decode() == "0.1.0"
+    for code in range(5):
+        assert lib.msda_status_string(code)
+    assert b"unknown" in lib.msda_status_string(99)
+
+
+FAKE = ctypes.c_void_p(0x100000)       # 16-byte aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p(0x100004)
+
+
+def _prob(**kw):
+    d = dict(batch=1, num_keys=80, num_queries=16, num_heads=2, head_dim=8, num_levels=2,
+             num_points=2, value_dtype=_lib.MSDA_F32, flags=0)
+    d.update(kw)
+    return _lib.Problem(**d)
+
+
+def _fwd(lib, prob, **ptrs):
+    p = dict(value=FAKE, shapes=FAKE, starts=FAKE, loc=FAKE, attn=FAKE, out=FAKE)
+    p.update(ptrs)
+    return lib.msda_forward(ctypes.byref(prob) if prob is not None else None, p["value"],
+                            p["shapes"], p["starts"], p["loc"], p["attn"], p["out"], None)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(head_dim=24), _lib.MSDA_ERR_UNSUPPORTED),
+    (dict(head_dim=512), _lib.MSDA_ERR_UNSUPPORTED),
+    (dict(num_levels=17), _lib.MSDA_ERR_UNSUPPORTED),
+    (dict(num_points=33), _lib.MSDA_ERR_UNSUPPORTED),
+    (dict(num_levels=16, num_points=9), _lib.MSDA_ERR_UNSUPPORTED),
+    (dict(num_keys=1 << 27), _lib.MSDA_ERR_UNSUPPORTED),
+    (dict(num_keys=0), _lib.MSDA_ERR_INVALID_ARG),
+    (dict(num_heads=0), _lib.MSDA_ERR_INVALID_ARG),
+    (dict(batch=-1), _lib.MSDA_ERR_INVALID_ARG),
+    (dict(num_queries=-3), _lib.MSDA_ERR_INVALID_ARG),
+    (dict(value_dtype=7), _lib.MSDA_ERR_INVALID_ARG),
+    (dict(flags=1 << 5), _lib.MSDA_ERR_INVALID_ARG),
+    (dict(flags=_lib.MSDA_GRAD_VALUE_BF16 | _lib.MSDA_ACCUMULATE_GRADS), _lib.MSDA_ERR_INVALID_ARG),
+])
+def test_problem_checks(lib, bad, code):
+    assert _fwd(lib, _prob(**bad)) == code
+
+
+def test_pointer_checks(lib):
+    assert _fwd(lib, None) == _lib.MSDA_ERR_INVALID_ARG
+    for k in ("value", "shapes", "starts", "loc", "attn", "out"):
+        assert _fwd(lib, _prob(), **{k: None}) == _lib.MSDA_ERR_INVALID_ARG, k
+        assert _fwd(lib, _prob(), **{k: MISALIGNED}) == _lib.MSDA_ERR_INVALID_ARG, k
+
+
+def test_backward_checks(lib):
+    prob = _prob(flags=_lib.MSDA_GRAD_VALUE_BF16)
+    n = ctypes.c_size_t(0)
+    assert lib.msda_backward_workspace_size(ctypes.byref(prob), ctypes.byref(n)) == 0
+    assert n.value == 1 * 80 * 2 * 8 * 4
+    prob32 = _prob()
+    assert lib.msda_backward_workspace_size(ctypes.byref(prob32), ctypes.byref(n)) == 0
+    assert n.value == 0
+    # bf16 grad_value without a big enough workspace
+    st = lib.msda_backward(ctypes.byref(prob), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                           FAKE, 16, None)
+    assert st == _lib.MSDA_ERR_INVALID_ARG
+    st = lib.msda_fused_backward(ctypes.byref(_prob()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 None, FAKE, FAKE, FAKE, None, 0, None)
+    assert st == _lib.MSDA_ERR_INVALID_ARG
+    assert lib.msda_zero_grads(ctypes.byref(_prob()), None, None, None) == _lib.MSDA_ERR_INVALID_ARG
+    assert lib.msda_get_device_status(None, None) == _lib.MSDA_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_oracle_import():
+    """The package (binding + library) never imports the oracle."""
+    import os
+    import re
+    pkg = os.path.dirname(_lib.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
+                assert "msda_oracle" not in text, f
