@@ -48,11 +48,13 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, out: str = LIB, defines=()) -> str:
+    """Compiles the library to `out`; `defines` are extra -D tuning knobs."""
+    if not force and out == LIB and not defines and up_to_date():
         return LIB
-    tmp = LIB + ".%d.tmp" % os.getpid()
-    cmd = [nvcc()] + ARCH + FLAGS + ["-I", INCLUDE, "-I", CSRC, "-o", tmp] + sources()
+    tmp = out + ".%d.tmp" % os.getpid()
+    cmd = [nvcc()] + ARCH + FLAGS + ["-D" + d for d in defines] + \
+        ["-I", INCLUDE, "-I", CSRC, "-o", tmp] + sources()
     if verbose:
         cmd += ["-Xptxas", "-v"]
         print(" ".join(cmd))
@@ -62,8 +64,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         sys.stderr.write(res.stderr)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed (exit %d)" % res.returncode)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

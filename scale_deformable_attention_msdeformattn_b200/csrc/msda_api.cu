@@ -2,8 +2,8 @@
 // selection by (value dtype, head_dim), launch shapes, device status word.
 //
 // Launch shape.  Every compute kernel runs as one persistent wave: the grid is
-// (SM count) x (resident CTAs per SM, from the occupancy calculator), each CTA
-// owning a contiguous range of row tiles.  CTAs have up to 8 warps; fewer when
+// (SM count) x (resident CTAs per SM, from the occupancy calculator), walking
+// the row tiles band by band (see the scheduling notes in msda_kernels.cuh).  CTAs have up to 8 warps; fewer when
 // the shared-memory records of the L*K samples of each row would exceed the
 // per-CTA budget.
 #include "msda.h"
@@ -17,8 +17,11 @@ using msda::KernelArgs;
 
 constexpr int kMaxDevices = 64;
 constexpr size_t kCtaSmemBudget = 96 * 1024;   // keeps >= 2 CTAs per SM
-constexpr size_t kForwardRecordBytes = sizeof(msda::Record);
-constexpr size_t kBackwardRecordBytes = sizeof(msda::Record) + 3 * sizeof(float);
+// shared-memory bytes per sample slot of a row: two 16-byte records, plus the
+// saved grad_A of the fused backward
+constexpr size_t kForwardRecordBytes = 32;
+constexpr size_t kBackwardRecordBytes = 32;
+constexpr size_t kFusedBackwardRecordBytes = 36;
 
 bool is_supported_head_dim(int d)
 {
@@ -59,6 +62,10 @@ msda_status check_problem(const msda_problem *p)
         return MSDA_ERR_UNSUPPORTED;
     if ((int64_t)p->num_heads * p->head_dim * (int64_t)elem_bytes(p->value_dtype) >= (int64_t(1) << 31))
         return MSDA_ERR_UNSUPPORTED;
+    // corner offsets are int32 counts of 16-byte vectors within one batch entry
+    if (p->num_keys * (int64_t)p->num_heads * p->head_dim * (int64_t)elem_bytes(p->value_dtype) / 16 >=
+        (int64_t(1) << 31))
+        return MSDA_ERR_UNSUPPORTED;
     // B * Q * M * L * K < 2^40, evaluated without overflow
     const double samples = (double)p->batch * (double)p->num_queries * p->num_heads *
                            p->num_levels * p->num_points;
@@ -93,15 +100,42 @@ msda_status current_device(int &dev, int &sm_count)
 }
 
 // Resident CTAs per SM of `kernel` for (threads, smem), cached per device.
+// The kernel's dynamic shared-memory limit is raised once, to the device's
+// opt-in maximum, so that launches of one kernel with different record sizes
+// never see a limit set for a smaller one.
 struct OccEntry {
     const void *kernel;
     int dev, threads;
     size_t smem;
     int blocks;
 };
-constexpr int kOccCache = 256;
+struct AttrEntry {
+    const void *kernel;
+    int dev;
+};
+constexpr int kOccCache = 512;
 OccEntry g_occ[kOccCache];
 int g_occ_n = 0;
+AttrEntry g_attr[kOccCache];
+int g_attr_n = 0;
+
+msda_status raise_smem_limit(const void *kernel, int dev)
+{
+    for (int i = 0; i < g_attr_n; ++i)
+        if (g_attr[i].kernel == kernel && g_attr[i].dev == dev)
+            return MSDA_OK;
+    int optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, kernel) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - (int)fa.sharedSizeBytes) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    if (g_attr_n < kOccCache)
+        g_attr[g_attr_n++] = AttrEntry{kernel, dev};
+    return MSDA_OK;
+}
 
 msda_status occupancy(const void *kernel, int dev, int threads, size_t smem, int &blocks)
 {
@@ -113,9 +147,9 @@ msda_status occupancy(const void *kernel, int dev, int threads, size_t smem, int
             return MSDA_OK;
         }
     }
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return MSDA_ERR_CUDA;
+    msda_status st = raise_smem_limit(kernel, dev);
+    if (st != MSDA_OK)
+        return st;
     int b = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, threads, smem) != cudaSuccess || b < 1)
         return MSDA_ERR_CUDA;
@@ -136,7 +170,7 @@ msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, Kernel
     if (st != MSDA_OK)
         return st;
     const int P = a.L * a.K;
-    const size_t per_warp = (size_t)rpw * P * record_bytes;
+    const size_t per_warp = (size_t)rpw * msda::record_stride(P) * record_bytes;
     int warps = (int)(kCtaSmemBudget / per_warp);
     warps = warps < 1 ? 1 : (warps > msda::kMaxWarpsPerCta ? msda::kMaxWarpsPerCta : warps);
     const size_t smem = per_warp * warps;
@@ -147,11 +181,11 @@ msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, Kernel
         return st;
     a.rows_per_tile = (int64_t)warps * rpw;
     a.ntiles = (a.rows + a.rows_per_tile - 1) / a.rows_per_tile;
+    // one resident wave, but no more CTAs than there are band slices of work
     int64_t ctas = (int64_t)sms * blocks_per_sm;
-    if (ctas > a.ntiles)
-        ctas = a.ntiles;
-    a.tiles_per_cta = (a.ntiles + ctas - 1) / ctas;
-    ctas = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+    const int64_t slices = (a.ntiles + MSDA_BAND_TILES - 1) / MSDA_BAND_TILES;
+    if (ctas > slices)
+        ctas = slices;
     void *params[] = {&a};
     if (cudaLaunchKernel(kernel, dim3((unsigned)ctas), dim3(threads), params, smem, stream) != cudaSuccess)
         return MSDA_ERR_CUDA;
@@ -224,7 +258,7 @@ msda_status launch_backward(const msda_problem *p, KernelArgs &a, cudaStream_t s
 #define MSDA_BWD_CASE(T, DD)                                                                       \
     case DD:                                                                                        \
         return launch_rows((const void *)msda::backward_kernel<T, DD, FUSED>, rows_per_warp<T, DD>(), \
-                           kBackwardRecordBytes, a, s);
+                           FUSED ? kFusedBackwardRecordBytes : kBackwardRecordBytes, a, s);
     if (p->value_dtype == MSDA_F32) {
         switch (p->head_dim) {
             MSDA_BWD_CASE(float, 8) MSDA_BWD_CASE(float, 16) MSDA_BWD_CASE(float, 32)

@@ -39,9 +39,33 @@
 
 namespace msda {
 
+// Tuning knobs (compile-time): samples whose corner loads a forward lane keeps
+// in flight, and the resident CTAs per SM the register allocation targets.
+#ifndef MSDA_FWD_SAMPLES_IN_FLIGHT
+#define MSDA_FWD_SAMPLES_IN_FLIGHT 4
+#endif
+#ifndef MSDA_FWD_MIN_CTAS
+#define MSDA_FWD_MIN_CTAS 2
+#endif
+#ifndef MSDA_BWD_MIN_CTAS
+#define MSDA_BWD_MIN_CTAS 2
+#endif
+// Row tiles a CTA walks contiguously before the grid moves to the next band.
+#ifndef MSDA_BAND_TILES
+#define MSDA_BAND_TILES 8
+#endif
+// 1: rows are processed head-major (all queries of head 0, then head 1, ...)
+// so that the lane groups of a warp hold neighbouring queries of one head.
+#ifndef MSDA_HEAD_MAJOR
+#define MSDA_HEAD_MAJOR 1
+#endif
+// 1: streaming inputs and outputs carry an L2 evict-first policy.
+#ifndef MSDA_STREAM_HINTS
+#define MSDA_STREAM_HINTS 1
+#endif
+
 constexpr int kMaxLevels = 16;
 constexpr int kMaxWarpsPerCta = 8;
-constexpr int kKeyBias = 1 << 27;  // keys are stored biased into 28 bits
 
 // Per-device status word; kernels record inconsistent geometry here.
 __device__ int g_device_status;
@@ -67,7 +91,6 @@ struct KernelArgs {
     int64_t rows;           // B * Q * M
     int64_t rows_per_tile;  // warps per CTA * rows per warp
     int64_t ntiles;         // ceil(rows / rows_per_tile)
-    int64_t tiles_per_cta;
     int64_t S;
     int Q, M, L, K;
 };
@@ -184,46 +207,124 @@ __device__ __forceinline__ float group_max(float v)
     return v;
 }
 
+// ------------------------------------------------------------ cache hints --
+//
+// Arrays touched once per call (locations, offsets, logits, weights,
+// reference points, grad_output and the per-sample gradients) are read and
+// written with an L2 evict-first policy, so that they do not push value and
+// the grad_value accumulator out of L2.
+
+__device__ __forceinline__ uint64_t stream_policy()
+{
+    uint64_t p = 0;
+#if MSDA_STREAM_HINTS
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+#endif
+    return p;
+}
+
+__device__ __forceinline__ float ld_stream(const float *ptr, uint64_t pol)
+{
+#if MSDA_STREAM_HINTS
+    float v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.f32 %0, [%1], %2;"
+                 : "=f"(v) : "l"(ptr), "l"(pol));
+    return v;
+#else
+    (void)pol;
+    return __ldg(ptr);
+#endif
+}
+
+__device__ __forceinline__ float2 ld_stream2(const float2 *ptr, uint64_t pol)
+{
+#if MSDA_STREAM_HINTS
+    float2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;"
+                 : "=f"(v.x), "=f"(v.y) : "l"(ptr), "l"(pol));
+    return v;
+#else
+    (void)pol;
+    return __ldg(ptr);
+#endif
+}
+
+__device__ __forceinline__ void st_stream(float *ptr, float v, uint64_t pol)
+{
+#if MSDA_STREAM_HINTS
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" :: "l"(ptr), "f"(v), "l"(pol) : "memory");
+#else
+    (void)pol;
+    *ptr = v;
+#endif
+}
+
+__device__ __forceinline__ void st_stream2(float2 *ptr, float2 v, uint64_t pol)
+{
+#if MSDA_STREAM_HINTS
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;"
+                 :: "l"(ptr), "f"(v.x), "f"(v.y), "l"(pol) : "memory");
+#else
+    (void)pol;
+    *ptr = v;
+#endif
+}
+
+// 16-byte grad_output vector, read once per row.
+template <typename Raw>
+__device__ __forceinline__ Raw ld_stream_vec(const Raw *ptr, uint64_t pol)
+{
+#if MSDA_STREAM_HINTS
+    uint4 u;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "l"(ptr), "l"(pol));
+    return *reinterpret_cast<Raw *>(&u);
+#else
+    (void)pol;
+    return __ldg(ptr);
+#endif
+}
+
+// ------------------------------------------------------------- scheduling --
+//
+// Persistent grid, banded: the tiles are cut into bands of gridDim.x *
+// MSDA_BAND_TILES tiles; inside a band CTA c walks its own MSDA_BAND_TILES
+// consecutive tiles.  The whole GPU therefore sweeps the queries band by band
+// (the L2 working set is one band's footprint) while each CTA reuses its L1
+// across neighbouring tiles.
+//
+// Processing row p maps to memory row (b * Q + q) * M + m; head-major order
+// takes p = (m * B + b) * Q + q.
+
+__device__ __forceinline__ int64_t memory_row(const KernelArgs &a, int64_t p)
+{
+#if MSDA_HEAD_MAJOR
+    const int64_t BQ = a.rows / a.M;
+    const int64_t m = p / BQ;
+    const int64_t bq = p - m * BQ;
+    return bq * a.M + m;
+#else
+    (void)a;
+    return p;
+#endif
+}
+
 // ----------------------------------------------------------------- set-up --
+//
+// Each sample of a row becomes a 32-byte record in shared memory, stored as
+// two 16-byte arrays (structure of arrays) with an odd row stride so that the
+// lane groups of a warp read distinct banks:
+//   forward   wa  = {A*w00, A*w01, A*w10, A*w11}  (0 for corners outside the map)
+//             off = {o00, o01, o10, o11}          vector offsets of the corners
+//                                                 (o00 = -1: sample skipped)
+//   backward  fa  = {fx (-1: sample skipped), fy, A, W | H << 16}
+//             off = {o00, o01, o10, o11}          bit 31 set: corner outside
+// Corner c = (y0 + c/2, x0 + c%2).  A corner outside the map is redirected to
+// an in-map corner of the same sample (clamping its column / row), so every
+// issued load is in bounds and no per-corner predicate is needed; its weight
+// is exactly zero (forward) or its dot product is discarded (backward).
 
-// One sample's record: fractional parts, attention weight, and the biased key
-// of its top-left corner (start_l + y0 * W + x0) with the four corner in-map
-// bits in the top nibble (bit c: corner c = (y0 + c/2, x0 + c%2) is inside).
-struct Record {
-    float fx, fy, A;
-    uint32_t packed;
-};
-
-__device__ __forceinline__ Record make_record(double x, double y, int H, int W, int start, float A)
-{
-    Record r;
-    r.A = A;
-    bool valid = (x > -1.0) && (x < (double)W) && (y > -1.0) && (y < (double)H);
-    if (!valid) {
-        r.fx = 0.f;
-        r.fy = 0.f;
-        r.packed = (uint32_t)kKeyBias;  // mask 0: nothing is read
-        return r;
-    }
-    double x0d = floor(x), y0d = floor(y);
-    int x0 = (int)x0d, y0 = (int)y0d;  // x0 in [-1, W-1], y0 in [-1, H-1]
-    r.fx = (float)(x - x0d);
-    r.fy = (float)(y - y0d);
-    uint32_t mask = 0;
-    bool left = x0 >= 0, right = x0 + 1 < W, top = y0 >= 0, bottom = y0 + 1 < H;
-    mask |= (top && left) ? 1u : 0u;
-    mask |= (top && right) ? 2u : 0u;
-    mask |= (bottom && left) ? 4u : 0u;
-    mask |= (bottom && right) ? 8u : 0u;
-    int key = start + y0 * W + x0;
-    r.packed = (uint32_t)(key + kKeyBias) | (mask << 28);
-    return r;
-}
-
-__device__ __forceinline__ int record_key(uint32_t packed)
-{
-    return (int)(packed & 0x0fffffffu) - kKeyBias;
-}
+__host__ __device__ __forceinline__ int record_stride(int P) { return (P & 1) ? P + 2 : P + 1; }
 
 // Non-fused: x = loc_x * W - 0.5 in float64 (the product of a float32 and an
 // integer below 2^16 is exact, so this equals the double-precision formula).
@@ -245,71 +346,166 @@ __device__ __forceinline__ void pixel_from_offset(float rx, float ry, float ox, 
     y = __dsub_rn(__dmul_rn(ly, (double)H), 0.5);
 }
 
-// Level of flattened sample s = l * K + k.
-__device__ __forceinline__ int level_of(int s, int K) { return s / K; }
+// Corner geometry of one sample at pixel coordinate (x, y) of a level.
+struct Corners {
+    bool valid;          // -1 < x < W and -1 < y < H
+    float fx, fy;
+    int key[4];          // flattened keys, redirected into the map
+    bool in[4];          // corner lies inside the map
+};
 
-// Builds the records of one row into rec[0 .. P-1]; lane `gl` of the group
-// does samples gl, gl + G, ...  For the fused kernels the softmax over the
-// row's logits is taken here as well (max-subtracted, float32).
-template <int G, bool FUSED>
-__device__ __forceinline__ void setup_row(const KernelArgs &a, const Geometry &geo, int64_t row,
-                                          bool active, int gl, Record *rec, float *attn_out)
+__device__ __forceinline__ Corners corners_of(double x, double y, int H, int W, int start)
+{
+    Corners c;
+    c.valid = (x > -1.0) && (x < (double)W) && (y > -1.0) && (y < (double)H);
+    if (!c.valid) {
+        c.fx = c.fy = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            c.key[i] = start;
+            c.in[i] = false;
+        }
+        return c;
+    }
+    const double x0d = floor(x), y0d = floor(y);
+    const int x0 = (int)x0d, y0 = (int)y0d;  // x0 in [-1, W-1], y0 in [-1, H-1]
+    c.fx = (float)(x - x0d);
+    c.fy = (float)(y - y0d);
+    const bool left = x0 >= 0, right = x0 + 1 < W, top = y0 >= 0, bottom = y0 + 1 < H;
+    const int xl = left ? x0 : x0 + 1, xr = right ? x0 + 1 : x0;
+    const int yt = top ? y0 : y0 + 1, yb = bottom ? y0 + 1 : y0;
+    c.key[0] = start + yt * W + xl;
+    c.key[1] = start + yt * W + xr;
+    c.key[2] = start + yb * W + xl;
+    c.key[3] = start + yb * W + xr;
+    c.in[0] = top && left;
+    c.in[1] = top && right;
+    c.in[2] = bottom && left;
+    c.in[3] = bottom && right;
+    return c;
+}
+
+// Row prologue of the fused kernels: softmax statistics of the row's L*K
+// logits (max-subtracted, float32) and the row's reference point.  Every lane
+// of the warp takes part in the shuffles; inactive groups use dummy values.
+template <int G>
+__device__ __forceinline__ void fused_row_stats(const KernelArgs &a, int64_t row, bool active, int gl,
+                                                float &mx, float &inv_sum, float &rx, float &ry)
 {
     const int P = a.L * a.K;
     const int64_t base = row * P;
-    float mx = -INFINITY, inv_sum = 0.f;
-    float rx = 0.f, ry = 0.f;
-    if (FUSED) {
-        // softmax statistics of the row (every lane of the warp takes part in
-        // the shuffles, inactive groups on dummy values)
-        if (active)
-            for (int s = gl; s < P; s += G)
-                mx = fmaxf(mx, __ldg(a.logits + base + s));
-        mx = group_max<G>(mx);
-        float sum = 0.f;
-        if (active)
-            for (int s = gl; s < P; s += G)
-                sum += expf(__ldg(a.logits + base + s) - mx);
-        sum = group_sum<G>(sum);
-        inv_sum = 1.0f / sum;
-        if (active) {
-            int64_t bq = row / a.M;
-            rx = __ldg(a.ref + 2 * bq);
-            ry = __ldg(a.ref + 2 * bq + 1);
-        }
+    mx = -INFINITY;
+    if (active)
+        for (int s = gl; s < P; s += G)
+            mx = fmaxf(mx, __ldg(a.logits + base + s));
+    mx = group_max<G>(mx);
+    float sum = 0.f;
+    if (active)
+        for (int s = gl; s < P; s += G)
+            sum += expf(__ldg(a.logits + base + s) - mx);
+    sum = group_sum<G>(sum);
+    inv_sum = 1.0f / sum;
+    rx = ry = 0.f;
+    if (active) {
+        const int64_t bq = row / a.M;
+        const float2 r = __ldg(reinterpret_cast<const float2 *>(a.ref) + bq);
+        rx = r.x;
+        ry = r.y;
     }
+}
+
+// Pixel coordinate and attention weight of sample s of a row.
+template <bool FUSED>
+__device__ __forceinline__ void sample_input(const KernelArgs &a, int64_t base, int s, int H, int W,
+                                             float mx, float inv_sum, float rx, float ry,
+                                             uint64_t pol, double &x, double &y, float &A)
+{
+    if (FUSED) {
+        const float2 o = ld_stream2(reinterpret_cast<const float2 *>(a.off) + base + s, pol);
+        pixel_from_offset(rx, ry, o.x, o.y, H, W, x, y);
+        // last read of the logits: the softmax statistics pass read them first
+        A = expf(ld_stream(a.logits + base + s, pol) - mx) * inv_sum;
+    } else {
+        const float2 p = ld_stream2(reinterpret_cast<const float2 *>(a.loc) + base + s, pol);
+        pixel_from_location(p.x, p.y, H, W, x, y);
+        A = ld_stream(a.attn + base + s, pol);
+    }
+}
+
+// Builds the forward records of one row; lane gl of the group does samples
+// gl, gl + G, ...  `vpp` is the number of value vectors per key (M * D / EPV).
+template <int G, bool FUSED>
+__device__ __forceinline__ void setup_forward_row(const KernelArgs &a, const Geometry &geo,
+                                                  int64_t row, bool active, int gl, int vpp,
+                                                  uint64_t pol, float4 *wa, int4 *off)
+{
+    const int P = a.L * a.K;
+    const int64_t base = row * P;
+    float mx = 0.f, inv_sum = 0.f, rx = 0.f, ry = 0.f;
+    if (FUSED)
+        fused_row_stats<G>(a, row, active, gl, mx, inv_sum, rx, ry);
     if (!active)
         return;
     for (int s = gl; s < P; s += G) {
-        const int l = level_of(s, a.K);
+        const int l = s / a.K;
         const int H = geo.H[l], W = geo.W[l];
         double x, y;
         float A;
-        if (FUSED) {
-            const float2 o = __ldg(reinterpret_cast<const float2 *>(a.off) + base + s);
-            pixel_from_offset(rx, ry, o.x, o.y, H, W, x, y);
-            A = expf(__ldg(a.logits + base + s) - mx) * inv_sum;
-            if (attn_out)
-                attn_out[base + s] = A;
-        } else {
-            const float2 p = __ldg(reinterpret_cast<const float2 *>(a.loc) + base + s);
-            pixel_from_location(p.x, p.y, H, W, x, y);
-            A = __ldg(a.attn + base + s);
-        }
-        rec[s] = make_record(x, y, H, W, geo.start[l], A);
+        sample_input<FUSED>(a, base, s, H, W, mx, inv_sum, rx, ry, pol, x, y, A);
+        if (FUSED && a.attn_out)
+            st_stream(a.attn_out + base + s, A, pol);
+        const Corners c = corners_of(x, y, H, W, geo.start[l]);
+        const float ay1 = A * c.fy, ay0 = A - ay1;
+        float4 w;
+        w.x = c.in[0] ? ay0 * (1.f - c.fx) : 0.f;
+        w.y = c.in[1] ? ay0 * c.fx : 0.f;
+        w.z = c.in[2] ? ay1 * (1.f - c.fx) : 0.f;
+        w.w = c.in[3] ? ay1 * c.fx : 0.f;
+        wa[s] = w;
+        off[s] = c.valid ? make_int4(c.key[0] * vpp, c.key[1] * vpp, c.key[2] * vpp, c.key[3] * vpp)
+                         : make_int4(-1, 0, 0, 0);
+    }
+}
+
+// Builds the backward records of one row (same lane split as the forward).
+template <int G, bool FUSED>
+__device__ __forceinline__ void setup_backward_row(const KernelArgs &a, const Geometry &geo,
+                                                   int64_t row, bool active, int gl, int vpp,
+                                                   uint64_t pol, float4 *fa, int4 *off)
+{
+    const int P = a.L * a.K;
+    const int64_t base = row * P;
+    float mx = 0.f, inv_sum = 0.f, rx = 0.f, ry = 0.f;
+    if (FUSED)
+        fused_row_stats<G>(a, row, active, gl, mx, inv_sum, rx, ry);
+    if (!active)
+        return;
+    for (int s = gl; s < P; s += G) {
+        const int l = s / a.K;
+        const int H = geo.H[l], W = geo.W[l];
+        double x, y;
+        float A;
+        sample_input<FUSED>(a, base, s, H, W, mx, inv_sum, rx, ry, pol, x, y, A);
+        const Corners c = corners_of(x, y, H, W, geo.start[l]);
+        fa[s] = make_float4(c.valid ? c.fx : -1.f, c.fy, A, __uint_as_float((unsigned)W | ((unsigned)H << 16)));
+        int o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            o[i] = (c.key[i] * vpp) | (c.in[i] ? 0 : (int)0x80000000);
+        off[s] = make_int4(o[0], o[1], o[2], o[3]);
     }
 }
 
 // ---------------------------------------------------------------- forward --
 
 template <typename T, int D, bool FUSED>
-__global__ void __launch_bounds__(kMaxWarpsPerCta * 32)
+__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, MSDA_FWD_MIN_CTAS)
 forward_kernel(const KernelArgs a)
 {
     using Lay = Layout<T, D>;
     using Raw = typename Vec<T>::Raw;
-    constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems;
-    constexpr int UNROLL = 4;
+    constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Vec<T>::kElems;
+    constexpr int U = MSDA_FWD_SAMPLES_IN_FLIGHT;  // samples in flight per lane (4 corners each)
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ Geometry geo;
@@ -318,77 +514,73 @@ forward_kernel(const KernelArgs a)
         return;
 
     const int P = a.L * a.K;
+    const int stride = record_stride(P);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int grp = lane / G, gl = lane % G;
-    Record *rec = reinterpret_cast<Record *>(smem_raw) + (warp * Lay::kRowsPerWarp + grp) * P;
-    const int64_t rows_per_tile = a.rows_per_tile;
-    const int64_t MD = (int64_t)a.M * D;
+    const int slot = warp * Lay::kRowsPerWarp + grp;
+    float4 *wa = reinterpret_cast<float4 *>(smem_raw) + slot * stride;
+    int4 *off = reinterpret_cast<int4 *>(smem_raw) + a.rows_per_tile * stride + slot * stride;
+    const int vpp = a.M * (D / EPV);
+    const uint64_t pol = stream_policy();
 
-    const int64_t t0 = (int64_t)blockIdx.x * a.tiles_per_cta;
-    const int64_t t1 = min(t0 + a.tiles_per_cta, a.ntiles);
-    for (int64_t tile = t0; tile < t1; ++tile) {
-        const int64_t row = tile * rows_per_tile + warp * Lay::kRowsPerWarp + grp;
-        const bool active = row < a.rows;
-        setup_row<G, FUSED>(a, geo, row, active, gl, rec, a.attn_out);
+    const int64_t band = (int64_t)gridDim.x * MSDA_BAND_TILES;
+    for (int64_t tile0 = (int64_t)blockIdx.x * MSDA_BAND_TILES; tile0 < a.ntiles; tile0 += band)
+    for (int64_t tile = tile0; tile < min(tile0 + MSDA_BAND_TILES, a.ntiles); ++tile) {
+        const int64_t prow = tile * a.rows_per_tile + slot;
+        const bool active = prow < a.rows;
+        const int64_t row = active ? memory_row(a, prow) : prow;
+        setup_forward_row<G, FUSED>(a, geo, row, active, gl, vpp, pol, wa, off);
         __syncwarp();
         if (active) {
             const int64_t bq = row / a.M;
             const int m = (int)(row - bq * a.M);
             const int64_t b = bq / a.Q;
-            // this lane's first vector of head m of batch b, key 0
             const Raw *vbase = reinterpret_cast<const Raw *>(static_cast<const T *>(a.value) +
                                                              (b * a.S * a.M + m) * D) + gl;
             float acc[E];
 #pragma unroll
             for (int e = 0; e < E; ++e)
                 acc[e] = 0.f;
-            for (int l = 0; l < a.L; ++l) {
-                const int64_t row_step = (int64_t)geo.W[l] * MD / Vec<T>::kElems;  // vectors
-                const int64_t col_step = MD / Vec<T>::kElems;
-                for (int k0 = 0; k0 < a.K; k0 += UNROLL) {
-                    Raw v[UNROLL][4][CH];
-                    float w[UNROLL][4];
+            for (int s0 = 0; s0 < P; s0 += U) {
+                Raw v[U][4][CH];
+                float4 w[U];
+                bool ok[U];
 #pragma unroll
-                    for (int u = 0; u < UNROLL; ++u) {
-                        const bool in = k0 + u < a.K;
-                        const Record r = in ? rec[l * a.K + k0 + u] : Record{0.f, 0.f, 0.f, (uint32_t)kKeyBias};
-                        const uint32_t mask = r.packed >> 28;
-                        const float ay1 = r.A * r.fy, ay0 = r.A - ay1;
-                        w[u][0] = ay0 - ay0 * r.fx;
-                        w[u][1] = ay0 * r.fx;
-                        w[u][2] = ay1 - ay1 * r.fx;
-                        w[u][3] = ay1 * r.fx;
-                        const Raw *p0 = vbase + (int64_t)record_key(r.packed) * col_step;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const Raw *pc = p0 + ((c >> 1) ? row_step : 0) + ((c & 1) ? col_step : 0);
-#pragma unroll
-                            for (int j = 0; j < CH; ++j) {
-                                if (mask & (1u << c))
-                                    v[u][c][j] = load_value<T>(pc + j * G);
-                                else
-                                    v[u][c][j] = Raw{};
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < UNROLL; ++u)
+                for (int u = 0; u < U; ++u) {
+                    const int s = s0 + u;
+                    const int4 o = s < P ? off[s] : make_int4(-1, 0, 0, 0);
+                    w[u] = s < P ? wa[s] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    ok[u] = o.x >= 0;
+                    const int oc[4] = {o.x, o.y, o.z, o.w};
+                    if (ok[u]) {
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
 #pragma unroll
-                            for (int j = 0; j < CH; ++j) {
-                                float f[Vec<T>::kElems];
-                                Vec<T>::widen(v[u][c][j], f);
+                            for (int j = 0; j < CH; ++j)
+                                v[u][c][j] = load_value<T>(vbase + oc[c] + j * G);
+                    }
+                }
 #pragma unroll
-                                for (int e = 0; e < Vec<T>::kElems; ++e)
-                                    acc[j * Vec<T>::kElems + e] = fmaf(w[u][c], f[e], acc[j * Vec<T>::kElems + e]);
-                            }
+                for (int u = 0; u < U; ++u) {
+                    if (!ok[u])
+                        continue;
+                    const float wc[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int j = 0; j < CH; ++j) {
+                            float f[EPV];
+                            Vec<T>::widen(v[u][c][j], f);
+#pragma unroll
+                            for (int e = 0; e < EPV; ++e)
+                                acc[j * EPV + e] = fmaf(wc[c], f[e], acc[j * EPV + e]);
+                        }
                 }
             }
             Raw *obase = reinterpret_cast<Raw *>(static_cast<T *>(a.out) + row * D) + gl;
 #pragma unroll
             for (int j = 0; j < CH; ++j)
-                obase[j * G] = Vec<T>::narrow(acc + j * Vec<T>::kElems);
+                obase[j * G] = Vec<T>::narrow(acc + j * EPV);
         }
         __syncwarp();
     }
@@ -396,13 +588,42 @@ forward_kernel(const KernelArgs a)
 
 // --------------------------------------------------------------- backward --
 
+// Reduce-scatter of C samples x 3 partial sums over the G lanes of a group:
+// afterwards v[0][0..2] of lane gl holds the group totals of chunk sample
+// gl % C (halving exchange over the sample index for C lanes, then a plain
+// butterfly over the remaining G / C lanes).  Every lane of the warp must call.
+template <int G, int C>
+__device__ __forceinline__ void reduce_scatter3(float (&v)[C][3], int gl)
+{
+#pragma unroll
+    for (int o = C / 2; o >= 1; o >>= 1) {
+        const bool hi = (gl & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i)
+#pragma unroll
+            for (int t = 0; t < 3; ++t) {
+                const float lo_v = v[i][t], hi_v = v[i + o][t];
+                const float send = hi ? lo_v : hi_v;
+                const float keep = hi ? hi_v : lo_v;
+                v[i][t] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+    }
+#pragma unroll
+    for (int o = C; o < G; o <<= 1)
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+            v[0][t] += __shfl_xor_sync(0xffffffffu, v[0][t], o);
+}
+
 template <typename T, int D, bool FUSED>
-__global__ void __launch_bounds__(kMaxWarpsPerCta * 32)
+__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, MSDA_BWD_MIN_CTAS)
 backward_kernel(const KernelArgs a)
 {
     using Lay = Layout<T, D>;
     using Raw = typename Vec<T>::Raw;
     constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Vec<T>::kElems;
+    constexpr int C = G < 8 ? G : 8;  // samples per reduce-scatter chunk
+    constexpr int F4 = EPV / 4;       // float4 of grad_value per value vector
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ Geometry geo;
@@ -411,137 +632,127 @@ backward_kernel(const KernelArgs a)
         return;
 
     const int P = a.L * a.K;
+    const int stride = record_stride(P);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int grp = lane / G, gl = lane % G;
-    const int row_slot = warp * Lay::kRowsPerWarp + grp;
-    const int rows_per_cta = (int)a.rows_per_tile;
-    Record *rec = reinterpret_cast<Record *>(smem_raw) + row_slot * P;
-    // per-sample results of the row: (grad_x, grad_y, grad_A)
-    float *res = reinterpret_cast<float *>(reinterpret_cast<Record *>(smem_raw) + rows_per_cta * P)
-                 + row_slot * P * 3;
-    const int64_t MD = (int64_t)a.M * D;
+    const int slot = warp * Lay::kRowsPerWarp + grp;
+    float4 *fa = reinterpret_cast<float4 *>(smem_raw) + slot * stride;
+    int4 *off = reinterpret_cast<int4 *>(smem_raw) + a.rows_per_tile * stride + slot * stride;
+    // fused: grad_A of each sample, kept for the softmax Jacobian
+    float *gA = reinterpret_cast<float *>(reinterpret_cast<int4 *>(smem_raw) + 2 * a.rows_per_tile * stride)
+                + slot * stride;
+    const int vpp = a.M * (D / EPV);
+    const uint64_t pol = stream_policy();
 
-    const int64_t t0 = (int64_t)blockIdx.x * a.tiles_per_cta;
-    const int64_t t1 = min(t0 + a.tiles_per_cta, a.ntiles);
-    for (int64_t tile = t0; tile < t1; ++tile) {
-        const int64_t row = tile * rows_per_cta + row_slot;
-        const bool active = row < a.rows;
-        setup_row<G, FUSED>(a, geo, row, active, gl, rec, nullptr);
+    const int64_t band = (int64_t)gridDim.x * MSDA_BAND_TILES;
+    for (int64_t tile0 = (int64_t)blockIdx.x * MSDA_BAND_TILES; tile0 < a.ntiles; tile0 += band)
+    for (int64_t tile = tile0; tile < min(tile0 + MSDA_BAND_TILES, a.ntiles); ++tile) {
+        const int64_t prow = tile * a.rows_per_tile + slot;
+        const bool active = prow < a.rows;
+        const int64_t row = active ? memory_row(a, prow) : prow;
+        setup_backward_row<G, FUSED>(a, geo, row, active, gl, vpp, pol, fa, off);
         __syncwarp();
         const int64_t bq = active ? row / a.M : 0;
         const int m = active ? (int)(row - bq * a.M) : 0;
         const int64_t b = bq / a.Q;
         const Raw *vbase = reinterpret_cast<const Raw *>(static_cast<const T *>(a.value) +
                                                          (b * a.S * a.M + m) * D) + gl;
-        float4 *gvbase = reinterpret_cast<float4 *>(a.grad_value + (b * a.S * a.M + m) * D) + gl * (EPV / 4);
-        // grad_output chunk of this lane, widened
+        float4 *gvbase = reinterpret_cast<float4 *>(a.grad_value + (b * a.S * a.M + m) * D) + gl * F4;
         float g[E];
         if (active) {
             const Raw *gp = reinterpret_cast<const Raw *>(static_cast<const T *>(a.grad_out) + row * D) + gl;
 #pragma unroll
             for (int j = 0; j < CH; ++j)
-                Vec<T>::widen(__ldg(gp + j * G), g + j * EPV);
+                Vec<T>::widen(ld_stream_vec(gp + j * G, pol), g + j * EPV);
         } else {
 #pragma unroll
             for (int e = 0; e < E; ++e)
                 g[e] = 0.f;
         }
-        float ref_gx = 0.f, ref_gy = 0.f;  // fused: sum over the row of grad_loc
-        for (int l = 0; l < a.L; ++l) {
-            const int W = geo.W[l], H = geo.H[l];
-            const int64_t row_step = (int64_t)W * MD / EPV;
-            const int64_t col_step = MD / EPV;
-            for (int k = 0; k < a.K; ++k) {
-                const int s = l * a.K + k;
-                const Record r = active ? rec[s] : Record{0.f, 0.f, 0.f, (uint32_t)kKeyBias};
-                const uint32_t mask = r.packed >> 28;
-                const Raw *p0 = vbase + (int64_t)record_key(r.packed) * col_step;
+        const int64_t base = row * P;
+        float dot = 0.f, ref_gx = 0.f, ref_gy = 0.f;  // fused: per-owner partial sums
+        for (int c0 = 0; c0 < P; c0 += C) {
+            float part[C][3];
+#pragma unroll
+            for (int i = 0; i < C; ++i) {
+                const int s = c0 + i;
+                const bool in = active && s < P;
+                const float4 r = in ? fa[s] : make_float4(-1.f, 0.f, 0.f, 0.f);
+                const int4 o = in ? off[s] : make_int4(0, 0, 0, 0);
+                const bool ok = r.x >= 0.f;
+                const int oc[4] = {o.x, o.y, o.z, o.w};
                 float d[4] = {0.f, 0.f, 0.f, 0.f};  // partial <g, v_c>
+                if (ok) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int64_t coff = ((c >> 1) ? row_step : 0) + ((c & 1) ? col_step : 0);
+                    for (int c = 0; c < 4; ++c) {
 #pragma unroll
-                    for (int j = 0; j < CH; ++j) {
-                        if (mask & (1u << c)) {
+                        for (int j = 0; j < CH; ++j) {
                             float f[EPV];
-                            Vec<T>::widen(load_value<T>(p0 + coff + j * G), f);
+                            Vec<T>::widen(load_value<T>(vbase + (oc[c] & 0x7fffffff) + j * G), f);
 #pragma unroll
                             for (int e = 0; e < EPV; ++e)
                                 d[c] = fmaf(g[j * EPV + e], f[e], d[c]);
                         }
+                        d[c] = oc[c] < 0 ? 0.f : d[c];
                     }
                 }
-                const float fx = r.fx, fy = r.fy;
-                const float w00 = (1.f - fx) * (1.f - fy), w01 = fx * (1.f - fy);
-                const float w10 = (1.f - fx) * fy, w11 = fx * fy;
-                float ga = w00 * d[0] + w01 * d[1] + w10 * d[2] + w11 * d[3];
-                float gx = (1.f - fy) * (d[1] - d[0]) + fy * (d[3] - d[2]);
-                float gy = (1.f - fx) * (d[2] - d[0]) + fx * (d[3] - d[1]);
-                ga = group_sum<G>(ga);
-                gx = group_sum<G>(gx);
-                gy = group_sum<G>(gy);
-                if (active && mask) {
-                    // scatter A * w_c * g into grad_value
-                    const float wc[4] = {r.A * w00, r.A * w01, r.A * w10, r.A * w11};
-                    float4 *q0 = gvbase + (int64_t)record_key(r.packed) * (MD / 4);
+                const float fx = ok ? r.x : 0.f, fy = r.y, A = r.z;
+                const float ex = 1.f - fx, ey = 1.f - fy;
+                const float w[4] = {ex * ey, fx * ey, ex * fy, fx * fy};
+                part[i][0] = w[0] * d[0] + w[1] * d[1] + w[2] * d[2] + w[3] * d[3];
+                part[i][1] = A * (ey * (d[1] - d[0]) + fy * (d[3] - d[2]));
+                part[i][2] = A * (ex * (d[2] - d[0]) + fx * (d[3] - d[1]));
+                if (ok) {
+                    // scatter A * w_c * g into grad_value (in-map corners only)
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        if (!(mask & (1u << c)))
+                        if (oc[c] < 0)
                             continue;
-                        float4 *qc = q0 + ((c >> 1) ? (int64_t)W * MD / 4 : 0) + ((c & 1) ? MD / 4 : 0);
+                        const float aw = A * w[c];
+                        float4 *q = gvbase + (int64_t)oc[c] * F4;
 #pragma unroll
                         for (int j = 0; j < CH; ++j)
 #pragma unroll
-                            for (int h = 0; h < EPV / 4; ++h) {
+                            for (int h = 0; h < F4; ++h) {
                                 const float *gg = g + j * EPV + 4 * h;
-                                atomicAdd(qc + j * G * (EPV / 4) + h,
-                                          make_float4(wc[c] * gg[0], wc[c] * gg[1], wc[c] * gg[2], wc[c] * gg[3]));
+                                atomicAdd(q + j * G * F4 + h,
+                                          make_float4(aw * gg[0], aw * gg[1], aw * gg[2], aw * gg[3]));
                             }
                     }
                 }
-                // gradients w.r.t. the pixel coordinate, scaled to the caller's units
-                const float gxA = r.A * gx, gyA = r.A * gy;
-                if (active && gl == (s % G)) {
-                    if (FUSED) {
-                        res[3 * s] = gxA;         // grad offset (level pixels)
-                        res[3 * s + 1] = gyA;
-                    } else {
-                        res[3 * s] = (float)W * gxA;   // grad location (normalized)
-                        res[3 * s + 1] = (float)H * gyA;
-                    }
-                    res[3 * s + 2] = ga;
-                }
+            }
+            reduce_scatter3<G, C>(part, gl);
+            const int s = c0 + gl;
+            if (active && gl < C && s < P) {
+                const float4 r = fa[s];
+                const unsigned wh = __float_as_uint(r.w);
+                const float W = (float)(wh & 0xffffu), H = (float)(wh >> 16);
                 if (FUSED) {
-                    ref_gx += (float)W * gxA;
-                    ref_gy += (float)H * gyA;
+                    st_stream2(reinterpret_cast<float2 *>(a.grad_off) + base + s,
+                               make_float2(part[0][1], part[0][2]), pol);
+                    gA[s] = part[0][0];
+                    dot += r.z * part[0][0];
+                    ref_gx += W * part[0][1];
+                    ref_gy += H * part[0][2];
+                } else {
+                    st_stream2(reinterpret_cast<float2 *>(a.grad_loc) + base + s,
+                               make_float2(W * part[0][1], H * part[0][2]), pol);
+                    st_stream(a.grad_attn + base + s, part[0][0], pol);
                 }
             }
         }
-        __syncwarp();
-        // softmax Jacobian: grad_z_j = A_j (gA_j - sum_i A_i gA_i); every lane
-        // of the warp takes part in the shuffles
-        float dot = 0.f;
         if (FUSED) {
-            if (active)
-                for (int s = gl; s < P; s += G)
-                    dot += rec[s].A * res[3 * s + 2];
+            // softmax Jacobian: grad_z_j = A_j (gA_j - sum_i A_i gA_i)
             dot = group_sum<G>(dot);
-        }
-        if (active) {
-            const int64_t base = row * P;
-            if (FUSED) {
-                for (int s = gl; s < P; s += G) {
-                    a.grad_logits[base + s] = rec[s].A * (res[3 * s + 2] - dot);
-                    reinterpret_cast<float2 *>(a.grad_off)[base + s] = make_float2(res[3 * s], res[3 * s + 1]);
-                }
+            ref_gx = group_sum<G>(ref_gx);
+            ref_gy = group_sum<G>(ref_gy);
+            __syncwarp();
+            if (active && gl < C) {
+                for (int s = gl; s < P; s += C)
+                    st_stream(a.grad_logits + base + s, fa[s].z * (gA[s] - dot), pol);
                 if (a.grad_ref && gl == 0) {
                     atomicAdd(a.grad_ref + 2 * bq, ref_gx);
                     atomicAdd(a.grad_ref + 2 * bq + 1, ref_gy);
-                }
-            } else {
-                for (int s = gl; s < P; s += G) {
-                    reinterpret_cast<float2 *>(a.grad_loc)[base + s] = make_float2(res[3 * s], res[3 * s + 1]);
-                    a.grad_attn[base + s] = res[3 * s + 2];
                 }
             }
         }
