@@ -29,8 +29,9 @@
  *
  * Conventions for every entry point
  *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous,
- *     row-major, each 16-byte aligned.  The library keeps no pointer after
- *     the call returns and allocates no memory.
+ *     row-major, each 16-byte aligned; value and output 32-byte aligned (they
+ *     move in 32-byte vectors).  The library keeps no pointer after the call
+ *     returns and allocates no memory.
  *   - value, output and grad_output hold value_dtype elements (float32 or
  *     bfloat16); every other floating-point tensor is float32.  Accumulation
  *     is float32.
@@ -44,7 +45,7 @@
  *     host-side checks below run before anything is enqueued; a call that
  *     returns an error has enqueued nothing.
  *   - Supported sizes: D (head_dim) in {8, 16, 32, 64, 128, 256};
- *     1 <= L <= 16; 1 <= K <= 32; L*K <= 128; 1 <= M; S < 2^27;
+ *     1 <= L <= 16; 1 <= K <= 32; L*K <= 128; 1 <= M; S < 2^27; S*M < 2^31;
  *     B*Q*M*L*K < 2^40; B or Q may be 0 (nothing to sample).
  *   - No C++ exception crosses this boundary.
  */

@@ -17,11 +17,11 @@ using msda::KernelArgs;
 
 constexpr int kMaxDevices = 64;
 constexpr size_t kCtaSmemBudget = 96 * 1024;   // keeps >= 2 CTAs per SM
-// shared-memory bytes per sample slot of a row: two 16-byte records, plus the
-// saved grad_A of the fused backward
+// shared-memory bytes per sample slot of a row: two 16-byte records, plus
+// grad_A and A in the fused backward
 constexpr size_t kForwardRecordBytes = 32;
 constexpr size_t kBackwardRecordBytes = 32;
-constexpr size_t kFusedBackwardRecordBytes = 36;
+constexpr size_t kFusedBackwardRecordBytes = 40;
 
 bool is_supported_head_dim(int d)
 {
@@ -31,6 +31,7 @@ bool is_supported_head_dim(int d)
 size_t elem_bytes(int32_t dtype) { return dtype == MSDA_BF16 ? 2 : 4; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // A pointer may be null only when its tensor is empty.
 bool ptr_ok(const void *p, int64_t numel)
@@ -39,6 +40,9 @@ bool ptr_ok(const void *p, int64_t numel)
         return p == nullptr || aligned16(p);
     return p != nullptr && aligned16(p);
 }
+
+// value and output are read / written with 32-byte vectors
+bool vec_ptr_ok(const void *p, int64_t numel) { return ptr_ok(p, numel) && aligned32(p); }
 
 msda_status check_problem(const msda_problem *p)
 {
@@ -62,9 +66,8 @@ msda_status check_problem(const msda_problem *p)
         return MSDA_ERR_UNSUPPORTED;
     if ((int64_t)p->num_heads * p->head_dim * (int64_t)elem_bytes(p->value_dtype) >= (int64_t(1) << 31))
         return MSDA_ERR_UNSUPPORTED;
-    // corner offsets are int32 counts of 16-byte vectors within one batch entry
-    if (p->num_keys * (int64_t)p->num_heads * p->head_dim * (int64_t)elem_bytes(p->value_dtype) / 16 >=
-        (int64_t(1) << 31))
+    // corner offsets are int32 (key, head) row indices within one batch entry
+    if (p->num_keys * (int64_t)p->num_heads >= (int64_t(1) << 31))
         return MSDA_ERR_UNSUPPORTED;
     // B * Q * M * L * K < 2^40, evaluated without overflow
     const double samples = (double)p->batch * (double)p->num_queries * p->num_heads *
@@ -159,18 +162,17 @@ msda_status occupancy(const void *kernel, int dev, int threads, size_t smem, int
     return MSDA_OK;
 }
 
-template <typename T, int D> constexpr int rows_per_warp() { return msda::Layout<T, D>::kRowsPerWarp; }
 
-// Launches one compute kernel over all rows as a persistent wave.
-msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, KernelArgs &a,
-                        cudaStream_t stream)
+// Launches one compute kernel over all rows as a persistent wave; the row
+// records hold `padded_samples` slots.
+msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, int padded_samples,
+                        KernelArgs &a, cudaStream_t stream)
 {
     int dev = 0, sms = 0;
     msda_status st = current_device(dev, sms);
     if (st != MSDA_OK)
         return st;
-    const int P = a.L * a.K;
-    const size_t per_warp = (size_t)rpw * msda::record_stride(P) * record_bytes;
+    const size_t per_warp = (size_t)rpw * msda::record_stride(padded_samples) * record_bytes;
     int warps = (int)(kCtaSmemBudget / per_warp);
     warps = warps < 1 ? 1 : (warps > msda::kMaxWarpsPerCta ? msda::kMaxWarpsPerCta : warps);
     const size_t smem = per_warp * warps;
@@ -234,8 +236,9 @@ msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 {
 #define MSDA_FWD_CASE(T, DD)                                                                      \
     case DD:                                                                                       \
-        return launch_rows((const void *)msda::forward_kernel<T, DD, FUSED>, rows_per_warp<T, DD>(), \
-                           kForwardRecordBytes, a, s);
+        return launch_rows((const void *)msda::forward_kernel<T, DD, FUSED>,                     \
+                           msda::forward_rows_per_warp<T, DD>(),                                 \
+                           kForwardRecordBytes, a.L * a.K, a, s);
     if (p->value_dtype == MSDA_F32) {
         switch (p->head_dim) {
             MSDA_FWD_CASE(float, 8) MSDA_FWD_CASE(float, 16) MSDA_FWD_CASE(float, 32)
@@ -257,8 +260,10 @@ msda_status launch_backward(const msda_problem *p, KernelArgs &a, cudaStream_t s
 {
 #define MSDA_BWD_CASE(T, DD)                                                                       \
     case DD:                                                                                        \
-        return launch_rows((const void *)msda::backward_kernel<T, DD, FUSED>, rows_per_warp<T, DD>(), \
-                           FUSED ? kFusedBackwardRecordBytes : kBackwardRecordBytes, a, s);
+        return launch_rows((const void *)msda::backward_kernel<T, DD, FUSED>,                    \
+                           msda::backward_rows_per_warp<T, DD>(),                                \
+                           FUSED ? kFusedBackwardRecordBytes : kBackwardRecordBytes,             \
+                           msda::backward_padded_samples<T, DD>(a.L * a.K), a, s);
     if (p->value_dtype == MSDA_F32) {
         switch (p->head_dim) {
             MSDA_BWD_CASE(float, 8) MSDA_BWD_CASE(float, 16) MSDA_BWD_CASE(float, 32)
@@ -355,9 +360,9 @@ msda_status msda_forward(const msda_problem *problem, const void *value,
     if (st != MSDA_OK)
         return st;
     const Sizes z = sizes_of(problem);
-    if (!ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
+    if (!vec_ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
         !ptr_ok(sampling_locations, z.samples * 2) || !ptr_ok(attention_weights, z.samples) ||
-        !ptr_ok(output, z.rows_d))
+        !vec_ptr_ok(output, z.rows_d))
         return MSDA_ERR_INVALID_ARG;
     KernelArgs a = base_args(problem, value, spatial_shapes, level_start_index);
     if (a.rows == 0)
@@ -379,7 +384,7 @@ msda_status msda_backward(const msda_problem *problem, const void *value,
     if (st != MSDA_OK)
         return st;
     const Sizes z = sizes_of(problem);
-    if (!ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
+    if (!vec_ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
         !ptr_ok(sampling_locations, z.samples * 2) || !ptr_ok(attention_weights, z.samples) ||
         !ptr_ok(grad_output, z.rows_d) || !ptr_ok(grad_value, z.value) ||
         !ptr_ok(grad_sampling_locations, z.samples * 2) || !ptr_ok(grad_attention_weights, z.samples))
@@ -404,9 +409,9 @@ msda_status msda_fused_forward(const msda_problem *problem, const void *value,
     if (st != MSDA_OK)
         return st;
     const Sizes z = sizes_of(problem);
-    if (!ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
+    if (!vec_ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
         !ptr_ok(reference_points, z.queries * 2) || !ptr_ok(sampling_offsets, z.samples * 2) ||
-        !ptr_ok(attention_logits, z.samples) || !ptr_ok(output, z.rows_d) ||
+        !ptr_ok(attention_logits, z.samples) || !vec_ptr_ok(output, z.rows_d) ||
         (attention_weights_out && !aligned16(attention_weights_out)))
         return MSDA_ERR_INVALID_ARG;
     KernelArgs a = base_args(problem, value, spatial_shapes, level_start_index);
@@ -432,7 +437,7 @@ msda_status msda_fused_backward(const msda_problem *problem, const void *value,
     if (st != MSDA_OK)
         return st;
     const Sizes z = sizes_of(problem);
-    if (!ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
+    if (!vec_ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
         !ptr_ok(reference_points, z.queries * 2) || !ptr_ok(sampling_offsets, z.samples * 2) ||
         !ptr_ok(attention_logits, z.samples) || !ptr_ok(grad_output, z.rows_d) ||
         !ptr_ok(grad_value, z.value) || !ptr_ok(grad_sampling_offsets, z.samples * 2) ||

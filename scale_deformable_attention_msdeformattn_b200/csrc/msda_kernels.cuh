@@ -1,29 +1,29 @@
 // msda_kernels.cuh -- sm_100a kernels of the multi-scale deformable attention
-// core: forward, backward and their fused variants (location + softmax in the
-// kernel), plus the zero-fill and float32 -> bf16 conversion helpers.
+// core: forward, backward and their fused variants (location step + softmax
+// over the L*K points inside the kernel), plus zero-fill and float32 -> bf16
+// conversion helpers.
 //
-// Work decomposition.  A "row" is one (b, q, m) triple, rows are numbered
-// r = (b * Q + q) * M + m, so consecutive rows are the heads of one query and
-// consecutive queries follow.  A group of G lanes owns one row; each lane owns
-// one 16-byte vector (4 float32 or 8 bf16 channels) of the head_dim axis, so a
-// corner of a sample is one fully used 16*G-byte row segment of `value`
-// (128 bytes for D = 32 float32).  A warp carries 32 / G rows, a CTA up to 8
-// warps (fewer when the per-row shared-memory records would not fit).
-// Each CTA walks a contiguous range of row tiles (persistent grid, one wave),
-// so neighbouring queries -- which sample neighbouring pixels -- stay on one SM
-// and share its L1.
+// Work decomposition.  A "row" is one (b, q, m) triple; rows are numbered
+// r = (b * Q + q) * M + m.  A group of G lanes owns one row; each lane owns
+// one vector of VB bytes (16 or 32: 4 or 8 float32, 8 or 16 bf16 channels) of
+// the head_dim axis, so a corner of a sample is one fully used G*VB-byte row
+// segment of `value` (128 bytes for D = 32 float32).  A warp carries 32 / G
+// rows, a CTA up to 8 warps (fewer when the per-row shared-memory records
+// would not fit).
 //
-// Per tile there are two phases:
-//   1. set-up: the group's lanes turn the row's L*K samples into 16-byte
-//      records {fx, fy, A, key|mask} in shared memory (pixel coordinate, floor,
-//      the four corner in-map bits, the attention weight -- in the fused
-//      kernels also the location step and the softmax over the L*K logits);
+// Per tile of rows there are two phases:
+//   1. set-up: the group's lanes turn the row's L*K samples into records in
+//      shared memory (pixel coordinate, floor, corner in-map bits, corner
+//      offsets, attention weight; in the fused kernels also the location step
+//      and the softmax over the row's logits);
 //   2. gather: every lane of the group reads each record (a shared-memory
 //      broadcast) and issues the four corner loads for its vector; the forward
 //      accumulates A * w_c * v_c in float32 registers, the backward forms the
 //      four partial dot products <g, v_c>, reduces the three gradient terms over
-//      the group with butterfly shuffles and scatters A * w_c * g into
-//      grad_value with 16-byte vector float32 reductions (red.global.add.v4.f32).
+//      the group with a reduce-scatter of shuffles (each lane ends up owning
+//      one sample's results), and scatters A * w_c * g into the float32
+//      grad_value with 16-byte vector reductions (red.global.add.v4.f32), laid
+//      out so that every reduction fills whole 32-byte L2 sectors.
 //
 // Floor decisions.  The pixel coordinate x = loc_x * W - 0.5 and its floor are
 // taken in float64 with the same operations, in the same order, as the
@@ -39,28 +39,41 @@
 
 namespace msda {
 
-// Tuning knobs (compile-time): samples whose corner loads a forward lane keeps
-// in flight, and the resident CTAs per SM the register allocation targets.
-#ifndef MSDA_FWD_SAMPLES_IN_FLIGHT
-#define MSDA_FWD_SAMPLES_IN_FLIGHT 4
+// Tuning knobs (compile-time).  The forward gathers float32 rows with 32-byte
+// lane vectors, one sample in flight per lane and 3 CTAs per SM, and bf16
+// rows with 16-byte vectors and four samples in flight; the backward uses
+// 16-byte vectors (whole-sector grad_value reductions, more rows per warp).
+#ifndef MSDA_FWD_VB_F32
+#define MSDA_FWD_VB_F32 32
 #endif
-#ifndef MSDA_FWD_MIN_CTAS
-#define MSDA_FWD_MIN_CTAS 2
+#ifndef MSDA_FWD_INFLIGHT_F32
+#define MSDA_FWD_INFLIGHT_F32 1
+#endif
+#ifndef MSDA_FWD_MIN_CTAS_F32
+#define MSDA_FWD_MIN_CTAS_F32 3
+#endif
+#ifndef MSDA_FWD_VB_BF16
+#define MSDA_FWD_VB_BF16 16
+#endif
+#ifndef MSDA_FWD_INFLIGHT_BF16
+#define MSDA_FWD_INFLIGHT_BF16 4
+#endif
+#ifndef MSDA_FWD_MIN_CTAS_BF16
+#define MSDA_FWD_MIN_CTAS_BF16 2
+#endif
+#ifndef MSDA_BWD_VB
+#define MSDA_BWD_VB 16
 #endif
 #ifndef MSDA_BWD_MIN_CTAS
 #define MSDA_BWD_MIN_CTAS 2
 #endif
-// Row tiles a CTA walks contiguously before the grid moves to the next band.
-#ifndef MSDA_BAND_TILES
-#define MSDA_BAND_TILES 8
+#ifndef MSDA_BAND_TILES              // row tiles a CTA walks before the grid moves on
+#define MSDA_BAND_TILES 1
 #endif
-// 1: rows are processed head-major (all queries of head 0, then head 1, ...)
-// so that the lane groups of a warp hold neighbouring queries of one head.
-#ifndef MSDA_HEAD_MAJOR
-#define MSDA_HEAD_MAJOR 1
+#ifndef MSDA_HEAD_MAJOR              // 1: process rows head-major
+#define MSDA_HEAD_MAJOR 0
 #endif
-// 1: streaming inputs and outputs carry an L2 evict-first policy.
-#ifndef MSDA_STREAM_HINTS
+#ifndef MSDA_STREAM_HINTS            // 1: L2 evict-first on streaming arrays
 #define MSDA_STREAM_HINTS 1
 #endif
 
@@ -133,61 +146,96 @@ __device__ __forceinline__ bool load_geometry(const KernelArgs &a, Geometry &geo
 
 // ---------------------------------------------------------------- vectors --
 
-template <typename T> struct Vec;
-
-template <> struct Vec<float> {
-    static constexpr int kElems = 4;
-    using Raw = float4;
-    __device__ __forceinline__ static void widen(const Raw &r, float *f)
-    {
-        f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w;
-    }
-    __device__ __forceinline__ static Raw narrow(const float *f)
-    {
-        return make_float4(f[0], f[1], f[2], f[3]);
-    }
+struct alignas(32) U8 {
+    uint32_t w[8];
 };
 
-template <> struct Vec<__nv_bfloat16> {
-    static constexpr int kElems = 8;
-    using Raw = uint4;
-    // bf16 -> f32 is exact: the bf16 bits are the top half of the float.
-    __device__ __forceinline__ static void widen(const Raw &r, float *f)
+template <int VB> struct RawOf;
+template <> struct RawOf<16> { using type = uint4; };
+template <> struct RawOf<32> { using type = U8; };
+
+// Read-only vector load of `value` (L1-cached).
+__device__ __forceinline__ uint4 ld_vec(const uint4 *p) { return __ldg(p); }
+__device__ __forceinline__ U8 ld_vec(const U8 *p)
+{
+    U8 r;
+    asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]), "=r"(r.w[5]),
+                   "=r"(r.w[6]), "=r"(r.w[7])
+                 : "l"(p));
+    return r;
+}
+__device__ __forceinline__ void st_vec(uint4 *p, const uint4 &v) { *p = v; }
+__device__ __forceinline__ void st_vec(U8 *p, const U8 &v)
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :: "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]),
+                    "r"(v.w[6]), "r"(v.w[7])
+                 : "memory");
+}
+
+// Element type traits: widening of stored words to float32 and back.
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static constexpr int kBytes = 4;
+    template <int NW> __device__ __forceinline__ static void widen(const uint32_t *u, float *f)
     {
-        const uint32_t u[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < NW; ++i)
+            f[i] = __uint_as_float(u[i]);
+    }
+    template <int NW> __device__ __forceinline__ static void narrow(const float *f, uint32_t *u)
+    {
+#pragma unroll
+        for (int i = 0; i < NW; ++i)
+            u[i] = __float_as_uint(f[i]);
+    }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static constexpr int kBytes = 2;
+    // bf16 -> f32 is exact: the bf16 bits are the top half of the float.
+    template <int NW> __device__ __forceinline__ static void widen(const uint32_t *u, float *f)
+    {
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
             f[2 * i] = __uint_as_float(u[i] << 16);
             f[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
         }
     }
-    __device__ __forceinline__ static Raw narrow(const float *f)
+    template <int NW> __device__ __forceinline__ static void narrow(const float *f, uint32_t *u)
     {
-        uint32_t u[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < NW; ++i) {
             __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
             u[i] = *reinterpret_cast<uint32_t *>(&h);
         }
-        return make_uint4(u[0], u[1], u[2], u[3]);
     }
 };
 
-template <typename T, int D> struct Layout {
-    static constexpr int kEpv = Vec<T>::kElems;              // channels per vector
+// Lane layout of one row of D channels with VB-byte lane vectors.
+template <typename T, int D, int VB> struct Layout {
+    static constexpr int kVB = (D * Elem<T>::kBytes < VB) ? D * Elem<T>::kBytes : VB;
+    using Raw = typename RawOf<kVB>::type;
+    static constexpr int kWords = kVB / 4;                   // 32-bit words per vector
+    static constexpr int kEpv = kVB / Elem<T>::kBytes;       // channels per vector
     static constexpr int kNvec = D / kEpv;                   // vectors per row
     static constexpr int kG = kNvec < 32 ? kNvec : 32;       // lanes per row
     static constexpr int kCh = kNvec / kG;                   // vectors per lane
     static constexpr int kRowsPerWarp = 32 / kG;
     static constexpr int kLaneElems = kCh * kEpv;            // channels per lane
+    static_assert(kVB == 16 || kVB == 32, "vector size");
     static_assert(kNvec >= 1 && kNvec % kG == 0, "unsupported head_dim");
+    __device__ __forceinline__ static void widen(const Raw &r, float *f)
+    {
+        Elem<T>::template widen<kWords>(reinterpret_cast<const uint32_t *>(&r), f);
+    }
+    __device__ __forceinline__ static Raw narrow(const float *f)
+    {
+        Raw r;
+        Elem<T>::template narrow<kWords>(f, reinterpret_cast<uint32_t *>(&r));
+        return r;
+    }
 };
-
-template <typename T>
-__device__ __forceinline__ typename Vec<T>::Raw load_value(const typename Vec<T>::Raw *p)
-{
-    return __ldg(p);
-}
 
 template <int G>
 __device__ __forceinline__ float group_sum(float v)
@@ -205,6 +253,25 @@ __device__ __forceinline__ float group_max(float v)
     for (int o = G / 2; o > 0; o >>= 1)
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
+}
+
+// Packed float32 pair arithmetic (one instruction for two lanes of work).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(*reinterpret_cast<unsigned long long *>(&d))
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)),
+          "l"(*reinterpret_cast<unsigned long long *>(&c)));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;"
+        : "=l"(*reinterpret_cast<unsigned long long *>(&d))
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)));
+    return d;
 }
 
 // ------------------------------------------------------------ cache hints --
@@ -249,6 +316,32 @@ __device__ __forceinline__ float2 ld_stream2(const float2 *ptr, uint64_t pol)
 #endif
 }
 
+__device__ __forceinline__ uint2 ld_stream_u2(const uint2 *ptr, uint64_t pol)
+{
+#if MSDA_STREAM_HINTS
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;"
+                 : "=r"(v.x), "=r"(v.y) : "l"(ptr), "l"(pol));
+    return v;
+#else
+    (void)pol;
+    return __ldg(ptr);
+#endif
+}
+
+__device__ __forceinline__ uint4 ld_stream_u4(const uint4 *ptr, uint64_t pol)
+{
+#if MSDA_STREAM_HINTS
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(ptr), "l"(pol));
+    return v;
+#else
+    (void)pol;
+    return __ldg(ptr);
+#endif
+}
+
 __device__ __forceinline__ void st_stream(float *ptr, float v, uint64_t pol)
 {
 #if MSDA_STREAM_HINTS
@@ -270,28 +363,31 @@ __device__ __forceinline__ void st_stream2(float2 *ptr, float2 v, uint64_t pol)
 #endif
 }
 
-// 16-byte grad_output vector, read once per row.
-template <typename Raw>
-__device__ __forceinline__ Raw ld_stream_vec(const Raw *ptr, uint64_t pol)
+// 4 consecutive grad_output channels starting at element `e` of a row,
+// widened to float32.
+template <typename T>
+__device__ __forceinline__ float4 ld_grad4(const T *row, int e, uint64_t pol);
+template <>
+__device__ __forceinline__ float4 ld_grad4<float>(const float *row, int e, uint64_t pol)
 {
-#if MSDA_STREAM_HINTS
-    uint4 u;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
-                 : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "l"(ptr), "l"(pol));
-    return *reinterpret_cast<Raw *>(&u);
-#else
-    (void)pol;
-    return __ldg(ptr);
-#endif
+    const uint4 u = ld_stream_u4(reinterpret_cast<const uint4 *>(row + e), pol);
+    return make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+}
+template <>
+__device__ __forceinline__ float4 ld_grad4<__nv_bfloat16>(const __nv_bfloat16 *row, int e, uint64_t pol)
+{
+    const uint2 u = ld_stream_u2(reinterpret_cast<const uint2 *>(row + e), pol);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
 }
 
 // ------------------------------------------------------------- scheduling --
 //
 // Persistent grid, banded: the tiles are cut into bands of gridDim.x *
 // MSDA_BAND_TILES tiles; inside a band CTA c walks its own MSDA_BAND_TILES
-// consecutive tiles.  The whole GPU therefore sweeps the queries band by band
-// (the L2 working set is one band's footprint) while each CTA reuses its L1
-// across neighbouring tiles.
+// consecutive tiles (1: a plain grid-stride walk, so that the whole GPU sweeps
+// neighbouring queries together and the L2 working set stays one band's
+// footprint).
 //
 // Processing row p maps to memory row (b * Q + q) * M + m; head-major order
 // takes p = (m * B + b) * Q + q.
@@ -315,14 +411,15 @@ __device__ __forceinline__ int64_t memory_row(const KernelArgs &a, int64_t p)
 // two 16-byte arrays (structure of arrays) with an odd row stride so that the
 // lane groups of a warp read distinct banks:
 //   forward   wa  = {A*w00, A*w01, A*w10, A*w11}  (0 for corners outside the map)
-//             off = {o00, o01, o10, o11}          vector offsets of the corners
-//                                                 (o00 = -1: sample skipped)
-//   backward  fa  = {fx (-1: sample skipped), fy, A, W | H << 16}
-//             off = {o00, o01, o10, o11}          bit 31 set: corner outside
+//             off = {o00, o01, o10, o11}          corner rows (key * M) relative to
+//                                                 the row's (b, m) base; o00 = -1:
+//                                                 sample skipped
+//   backward  fa  = {fx (-1: sample skipped), fy, A, level | in-map bits << 8}
+//             off = {o00, o01, o10, o11}
 // Corner c = (y0 + c/2, x0 + c%2).  A corner outside the map is redirected to
-// an in-map corner of the same sample (clamping its column / row), so every
-// issued load is in bounds and no per-corner predicate is needed; its weight
-// is exactly zero (forward) or its dot product is discarded (backward).
+// an in-map corner of the same sample (its column / row clamped into the map),
+// so every issued load is in bounds; its weight is exactly zero (forward) or
+// its dot product and reduction are dropped (backward).
 
 __host__ __device__ __forceinline__ int record_stride(int P) { return (P & 1) ? P + 2 : P + 1; }
 
@@ -433,11 +530,11 @@ __device__ __forceinline__ void sample_input(const KernelArgs &a, int64_t base, 
 }
 
 // Builds the forward records of one row; lane gl of the group does samples
-// gl, gl + G, ...  `vpp` is the number of value vectors per key (M * D / EPV).
+// gl, gl + G, ...
 template <int G, bool FUSED>
 __device__ __forceinline__ void setup_forward_row(const KernelArgs &a, const Geometry &geo,
-                                                  int64_t row, bool active, int gl, int vpp,
-                                                  uint64_t pol, float4 *wa, int4 *off)
+                                                  int64_t row, bool active, int gl, uint64_t pol,
+                                                  float4 *wa, int4 *off)
 {
     const int P = a.L * a.K;
     const int64_t base = row * P;
@@ -462,50 +559,68 @@ __device__ __forceinline__ void setup_forward_row(const KernelArgs &a, const Geo
         w.z = c.in[2] ? ay1 * (1.f - c.fx) : 0.f;
         w.w = c.in[3] ? ay1 * c.fx : 0.f;
         wa[s] = w;
-        off[s] = c.valid ? make_int4(c.key[0] * vpp, c.key[1] * vpp, c.key[2] * vpp, c.key[3] * vpp)
+        off[s] = c.valid ? make_int4(c.key[0] * a.M, c.key[1] * a.M, c.key[2] * a.M, c.key[3] * a.M)
                          : make_int4(-1, 0, 0, 0);
     }
 }
 
-// Builds the backward records of one row (same lane split as the forward).
+// Builds the backward records of one row, padded to Pp >= P samples with
+// inert records (no load, no reduction); lane gl of the group does samples
+// gl, gl + G, ...  For an inactive row every record is inert.  Record of
+// sample s: fa = {fx, fy, A, in-map bits of the four corners}, off = corner
+// rows (key * M) with off.x = -1 when the sample is skipped.
 template <int G, bool FUSED>
 __device__ __forceinline__ void setup_backward_row(const KernelArgs &a, const Geometry &geo,
-                                                   int64_t row, bool active, int gl, int vpp,
-                                                   uint64_t pol, float4 *fa, int4 *off)
+                                                   int64_t row, bool active, int gl, uint64_t pol,
+                                                   int Pp, float4 *fa, int4 *off, float *As)
 {
     const int P = a.L * a.K;
     const int64_t base = row * P;
     float mx = 0.f, inv_sum = 0.f, rx = 0.f, ry = 0.f;
     if (FUSED)
         fused_row_stats<G>(a, row, active, gl, mx, inv_sum, rx, ry);
-    if (!active)
-        return;
-    for (int s = gl; s < P; s += G) {
+    for (int s = gl; s < Pp; s += G) {
+        if (!active || s >= P) {
+            fa[s] = make_float4(0.f, 0.f, 0.f, 0.f);
+            off[s] = make_int4(-1, 0, 0, 0);
+            continue;
+        }
         const int l = s / a.K;
         const int H = geo.H[l], W = geo.W[l];
         double x, y;
         float A;
         sample_input<FUSED>(a, base, s, H, W, mx, inv_sum, rx, ry, pol, x, y, A);
         const Corners c = corners_of(x, y, H, W, geo.start[l]);
-        fa[s] = make_float4(c.valid ? c.fx : -1.f, c.fy, A, __uint_as_float((unsigned)W | ((unsigned)H << 16)));
-        int o[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            o[i] = (c.key[i] * vpp) | (c.in[i] ? 0 : (int)0x80000000);
-        off[s] = make_int4(o[0], o[1], o[2], o[3]);
+        const unsigned bits = (c.in[0] ? 1u : 0u) | (c.in[1] ? 2u : 0u) | (c.in[2] ? 4u : 0u) |
+                              (c.in[3] ? 8u : 0u);
+        fa[s] = make_float4(c.fx, c.fy, A, __uint_as_float(bits));
+        off[s] = c.valid ? make_int4(c.key[0] * a.M, c.key[1] * a.M, c.key[2] * a.M, c.key[3] * a.M)
+                         : make_int4(-1, 0, 0, 0);
+        if (FUSED)
+            As[s] = A;
     }
 }
 
 // ---------------------------------------------------------------- forward --
 
+template <typename T> struct FwdTune;
+template <> struct FwdTune<float> {
+    static constexpr int kVB = MSDA_FWD_VB_F32, kInFlight = MSDA_FWD_INFLIGHT_F32,
+                         kMinCtas = MSDA_FWD_MIN_CTAS_F32;
+};
+template <> struct FwdTune<__nv_bfloat16> {
+    static constexpr int kVB = MSDA_FWD_VB_BF16, kInFlight = MSDA_FWD_INFLIGHT_BF16,
+                         kMinCtas = MSDA_FWD_MIN_CTAS_BF16;
+};
+
 template <typename T, int D, bool FUSED>
-__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, MSDA_FWD_MIN_CTAS)
+__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, FwdTune<T>::kMinCtas)
 forward_kernel(const KernelArgs a)
 {
-    using Lay = Layout<T, D>;
-    using Raw = typename Vec<T>::Raw;
-    constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Vec<T>::kElems;
-    constexpr int U = MSDA_FWD_SAMPLES_IN_FLIGHT;  // samples in flight per lane (4 corners each)
+    using Lay = Layout<T, D, FwdTune<T>::kVB>;
+    using Raw = typename Lay::Raw;
+    constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Lay::kEpv;
+    constexpr int U = FwdTune<T>::kInFlight;  // samples in flight per lane (4 corners each)
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ Geometry geo;
@@ -520,7 +635,6 @@ forward_kernel(const KernelArgs a)
     const int slot = warp * Lay::kRowsPerWarp + grp;
     float4 *wa = reinterpret_cast<float4 *>(smem_raw) + slot * stride;
     int4 *off = reinterpret_cast<int4 *>(smem_raw) + a.rows_per_tile * stride + slot * stride;
-    const int vpp = a.M * (D / EPV);
     const uint64_t pol = stream_policy();
 
     const int64_t band = (int64_t)gridDim.x * MSDA_BAND_TILES;
@@ -529,12 +643,14 @@ forward_kernel(const KernelArgs a)
         const int64_t prow = tile * a.rows_per_tile + slot;
         const bool active = prow < a.rows;
         const int64_t row = active ? memory_row(a, prow) : prow;
-        setup_forward_row<G, FUSED>(a, geo, row, active, gl, vpp, pol, wa, off);
+        setup_forward_row<G, FUSED>(a, geo, row, active, gl, pol, wa, off);
         __syncwarp();
         if (active) {
             const int64_t bq = row / a.M;
             const int m = (int)(row - bq * a.M);
             const int64_t b = bq / a.Q;
+            // this lane's first vector of head m of batch b, key 0; corner rows
+            // are D channels apart
             const Raw *vbase = reinterpret_cast<const Raw *>(static_cast<const T *>(a.value) +
                                                              (b * a.S * a.M + m) * D) + gl;
             float acc[E];
@@ -557,7 +673,7 @@ forward_kernel(const KernelArgs a)
                         for (int c = 0; c < 4; ++c)
 #pragma unroll
                             for (int j = 0; j < CH; ++j)
-                                v[u][c][j] = load_value<T>(vbase + oc[c] + j * G);
+                                v[u][c][j] = ld_vec(vbase + (int64_t)oc[c] * Lay::kNvec + j * G);
                     }
                 }
 #pragma unroll
@@ -570,7 +686,7 @@ forward_kernel(const KernelArgs a)
 #pragma unroll
                         for (int j = 0; j < CH; ++j) {
                             float f[EPV];
-                            Vec<T>::widen(v[u][c][j], f);
+                            Lay::widen(v[u][c][j], f);
 #pragma unroll
                             for (int e = 0; e < EPV; ++e)
                                 acc[j * EPV + e] = fmaf(wc[c], f[e], acc[j * EPV + e]);
@@ -580,7 +696,7 @@ forward_kernel(const KernelArgs a)
             Raw *obase = reinterpret_cast<Raw *>(static_cast<T *>(a.out) + row * D) + gl;
 #pragma unroll
             for (int j = 0; j < CH; ++j)
-                obase[j * G] = Vec<T>::narrow(acc + j * EPV);
+                st_vec(obase + j * G, Lay::narrow(acc + j * EPV));
         }
         __syncwarp();
     }
@@ -615,15 +731,23 @@ __device__ __forceinline__ void reduce_scatter3(float (&v)[C][3], int gl)
             v[0][t] += __shfl_xor_sync(0xffffffffu, v[0][t], o);
 }
 
+// Samples per backward reduce-scatter chunk for G lanes per row.
+template <int G> struct BwdChunk { static constexpr int kC = G < 4 ? G : 4; };
+
 template <typename T, int D, bool FUSED>
 __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, MSDA_BWD_MIN_CTAS)
 backward_kernel(const KernelArgs a)
 {
-    using Lay = Layout<T, D>;
-    using Raw = typename Vec<T>::Raw;
-    constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Vec<T>::kElems;
-    constexpr int C = G < 8 ? G : 8;  // samples per reduce-scatter chunk
-    constexpr int F4 = EPV / 4;       // float4 of grad_value per value vector
+    using Lay = Layout<T, D, MSDA_BWD_VB>;
+    using Raw = typename Lay::Raw;
+    constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Lay::kEpv;
+    constexpr int C = BwdChunk<G>::kC;
+    // grad_value reductions: a float32 row is D / 4 chunks of 16 bytes;
+    // reduction h of lane gl covers chunk h * G + gl, so each reduction
+    // instruction of a group fills whole sectors
+    constexpr int NR = D / 4 / G;
+    static_assert(NR >= 1 && (D / 4) % G == 0, "reduction layout");
+    static_assert(EPV % 2 == 0, "pairs");
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ Geometry geo;
@@ -632,16 +756,19 @@ backward_kernel(const KernelArgs a)
         return;
 
     const int P = a.L * a.K;
-    const int stride = record_stride(P);
+    const int Pp = (P + C - 1) / C * C;
+    const int stride = record_stride(Pp);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int grp = lane / G, gl = lane % G;
     const int slot = warp * Lay::kRowsPerWarp + grp;
+    const int64_t arr = a.rows_per_tile * stride;  // one record array, in 16-byte units
     float4 *fa = reinterpret_cast<float4 *>(smem_raw) + slot * stride;
-    int4 *off = reinterpret_cast<int4 *>(smem_raw) + a.rows_per_tile * stride + slot * stride;
-    // fused: grad_A of each sample, kept for the softmax Jacobian
-    float *gA = reinterpret_cast<float *>(reinterpret_cast<int4 *>(smem_raw) + 2 * a.rows_per_tile * stride)
-                + slot * stride;
-    const int vpp = a.M * (D / EPV);
+    int4 *off = reinterpret_cast<int4 *>(reinterpret_cast<float4 *>(smem_raw) + arr) + slot * stride;
+    // fused: grad_A and A of each sample, kept for the softmax Jacobian.
+    // Layout in floats: fa, off: 4 * arr each; gA, As: arr each (10 * arr
+    // floats = 40 bytes per record slot, as the host sizes it).
+    float *gA = reinterpret_cast<float *>(reinterpret_cast<float4 *>(smem_raw) + 2 * arr) + slot * stride;
+    float *As = gA + arr;
     const uint64_t pol = stream_policy();
 
     const int64_t band = (int64_t)gridDim.x * MSDA_BAND_TILES;
@@ -650,88 +777,101 @@ backward_kernel(const KernelArgs a)
         const int64_t prow = tile * a.rows_per_tile + slot;
         const bool active = prow < a.rows;
         const int64_t row = active ? memory_row(a, prow) : prow;
-        setup_backward_row<G, FUSED>(a, geo, row, active, gl, vpp, pol, fa, off);
+        setup_backward_row<G, FUSED>(a, geo, row, active, gl, pol, Pp, fa, off, As);
         __syncwarp();
         const int64_t bq = active ? row / a.M : 0;
         const int m = active ? (int)(row - bq * a.M) : 0;
         const int64_t b = bq / a.Q;
-        const Raw *vbase = reinterpret_cast<const Raw *>(static_cast<const T *>(a.value) +
-                                                         (b * a.S * a.M + m) * D) + gl;
-        float4 *gvbase = reinterpret_cast<float4 *>(a.grad_value + (b * a.S * a.M + m) * D) + gl * F4;
-        float g[E];
+        const int64_t rbase = b * a.S * a.M + m;  // (b, key 0, m) row
+        const Raw *vbase = reinterpret_cast<const Raw *>(static_cast<const T *>(a.value) + rbase * D) + gl;
+        float4 *gvbase = reinterpret_cast<float4 *>(a.grad_value + rbase * D) + gl;
+        // grad_output of the row: pairs in the load layout (dot products) and
+        // float4s in the reduction layout (scatter)
+        float2 g2[E / 2];
+        float4 gr[NR];
         if (active) {
-            const Raw *gp = reinterpret_cast<const Raw *>(static_cast<const T *>(a.grad_out) + row * D) + gl;
+            const T *grow = static_cast<const T *>(a.grad_out) + row * D;
 #pragma unroll
             for (int j = 0; j < CH; ++j)
-                Vec<T>::widen(ld_stream_vec(gp + j * G, pol), g + j * EPV);
+#pragma unroll
+                for (int q4 = 0; q4 < EPV / 4; ++q4) {
+                    const float4 t4 = ld_grad4<T>(grow, (j * G + gl) * EPV + 4 * q4, pol);
+                    g2[(j * EPV + 4 * q4) / 2] = make_float2(t4.x, t4.y);
+                    g2[(j * EPV + 4 * q4) / 2 + 1] = make_float2(t4.z, t4.w);
+                }
+#pragma unroll
+            for (int h = 0; h < NR; ++h)
+                gr[h] = ld_grad4<T>(grow, (h * G + gl) * 4, pol);
         } else {
 #pragma unroll
-            for (int e = 0; e < E; ++e)
-                g[e] = 0.f;
+            for (int e = 0; e < E / 2; ++e)
+                g2[e] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int h = 0; h < NR; ++h)
+                gr[h] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         const int64_t base = row * P;
         float dot = 0.f, ref_gx = 0.f, ref_gy = 0.f;  // fused: per-owner partial sums
-        for (int c0 = 0; c0 < P; c0 += C) {
+        for (int c0 = 0; c0 < Pp; c0 += C) {
             float part[C][3];
 #pragma unroll
             for (int i = 0; i < C; ++i) {
                 const int s = c0 + i;
-                const bool in = active && s < P;
-                const float4 r = in ? fa[s] : make_float4(-1.f, 0.f, 0.f, 0.f);
-                const int4 o = in ? off[s] : make_int4(0, 0, 0, 0);
-                const bool ok = r.x >= 0.f;
-                const int oc[4] = {o.x, o.y, o.z, o.w};
+                const int4 o = off[s];
                 float d[4] = {0.f, 0.f, 0.f, 0.f};  // partial <g, v_c>
-                if (ok) {
+                if (o.x >= 0) {
+                    const int oc[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
+                        float2 dp = make_float2(0.f, 0.f);
 #pragma unroll
                         for (int j = 0; j < CH; ++j) {
                             float f[EPV];
-                            Vec<T>::widen(load_value<T>(vbase + (oc[c] & 0x7fffffff) + j * G), f);
+                            Lay::widen(ld_vec(vbase + (int64_t)oc[c] * Lay::kNvec + j * G), f);
 #pragma unroll
-                            for (int e = 0; e < EPV; ++e)
-                                d[c] = fmaf(g[j * EPV + e], f[e], d[c]);
+                            for (int e = 0; e < EPV; e += 2)
+                                dp = fma2(g2[(j * EPV + e) / 2], make_float2(f[e], f[e + 1]), dp);
                         }
-                        d[c] = oc[c] < 0 ? 0.f : d[c];
+                        d[c] = dp.x + dp.y;
                     }
                 }
-                const float fx = ok ? r.x : 0.f, fy = r.y, A = r.z;
-                const float ex = 1.f - fx, ey = 1.f - fy;
+                const float4 r = fa[s];
+                const unsigned inm = __float_as_uint(r.w);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    d[c] = (inm & (1u << c)) ? d[c] : 0.f;  // corners outside the map read 0
+                const float fx = r.x, fy = r.y, A = r.z, ex = 1.f - fx, ey = 1.f - fy;
                 const float w[4] = {ex * ey, fx * ey, ex * fy, fx * fy};
                 part[i][0] = w[0] * d[0] + w[1] * d[1] + w[2] * d[2] + w[3] * d[3];
                 part[i][1] = A * (ey * (d[1] - d[0]) + fy * (d[3] - d[2]));
                 part[i][2] = A * (ex * (d[2] - d[0]) + fx * (d[3] - d[1]));
-                if (ok) {
-                    // scatter A * w_c * g into grad_value (in-map corners only)
+                // scatter A * w_c * g into grad_value (in-map corners of taken
+                // samples; skipped samples have no in-map bits)
+                const int ocs[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        if (oc[c] < 0)
-                            continue;
-                        const float aw = A * w[c];
-                        float4 *q = gvbase + (int64_t)oc[c] * F4;
+                for (int c = 0; c < 4; ++c) {
+                    if (!(inm & (1u << c)))
+                        continue;
+                    const float awc = A * w[c];
+                    float4 *q = gvbase + (int64_t)ocs[c] * (D / 4);
+                    const float2 ww = make_float2(awc, awc);
 #pragma unroll
-                        for (int j = 0; j < CH; ++j)
-#pragma unroll
-                            for (int h = 0; h < F4; ++h) {
-                                const float *gg = g + j * EPV + 4 * h;
-                                atomicAdd(q + j * G * F4 + h,
-                                          make_float4(aw * gg[0], aw * gg[1], aw * gg[2], aw * gg[3]));
-                            }
+                    for (int h = 0; h < NR; ++h) {
+                        const float2 lo = mul2(ww, make_float2(gr[h].x, gr[h].y));
+                        const float2 hi = mul2(ww, make_float2(gr[h].z, gr[h].w));
+                        atomicAdd(q + h * G, make_float4(lo.x, lo.y, hi.x, hi.y));
                     }
                 }
             }
             reduce_scatter3<G, C>(part, gl);
             const int s = c0 + gl;
             if (active && gl < C && s < P) {
-                const float4 r = fa[s];
-                const unsigned wh = __float_as_uint(r.w);
-                const float W = (float)(wh & 0xffffu), H = (float)(wh >> 16);
+                const int l = s / a.K;
+                const float W = (float)geo.W[l], H = (float)geo.H[l];
                 if (FUSED) {
                     st_stream2(reinterpret_cast<float2 *>(a.grad_off) + base + s,
                                make_float2(part[0][1], part[0][2]), pol);
                     gA[s] = part[0][0];
-                    dot += r.z * part[0][0];
                     ref_gx += W * part[0][1];
                     ref_gy += H * part[0][2];
                 } else {
@@ -743,13 +883,15 @@ backward_kernel(const KernelArgs a)
         }
         if (FUSED) {
             // softmax Jacobian: grad_z_j = A_j (gA_j - sum_i A_i gA_i)
+            if (active && gl < C)
+                for (int s = gl; s < P; s += C)
+                    dot += As[s] * gA[s];
             dot = group_sum<G>(dot);
             ref_gx = group_sum<G>(ref_gx);
             ref_gy = group_sum<G>(ref_gy);
-            __syncwarp();
             if (active && gl < C) {
                 for (int s = gl; s < P; s += C)
-                    st_stream(a.grad_logits + base + s, fa[s].z * (gA[s] - dot), pol);
+                    st_stream(a.grad_logits + base + s, As[s] * (gA[s] - dot), pol);
                 if (a.grad_ref && gl == 0) {
                     atomicAdd(a.grad_ref + 2 * bq, ref_gx);
                     atomicAdd(a.grad_ref + 2 * bq + 1, ref_gy);
@@ -779,8 +921,20 @@ __global__ void f32_to_bf16_kernel(const float4 *src, uint4 *dst, int64_t n8)
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
         const float4 x = src[2 * i], y = src[2 * i + 1];
         const float f[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
-        dst[i] = Vec<__nv_bfloat16>::narrow(f);
+        uint4 r;
+        Elem<__nv_bfloat16>::narrow<4>(f, reinterpret_cast<uint32_t *>(&r));
+        dst[i] = r;
     }
+}
+
+// Rows per warp of each kernel (the host sizes CTAs and shared memory by it).
+template <typename T, int D> constexpr int forward_rows_per_warp() { return Layout<T, D, FwdTune<T>::kVB>::kRowsPerWarp; }
+template <typename T, int D> constexpr int backward_rows_per_warp() { return Layout<T, D, MSDA_BWD_VB>::kRowsPerWarp; }
+// Record slots of a backward row: L*K rounded up to the reduce-scatter chunk.
+template <typename T, int D> inline int backward_padded_samples(int P)
+{
+    constexpr int C = BwdChunk<Layout<T, D, MSDA_BWD_VB>::kG>::kC;
+    return (P + C - 1) / C * C;
 }
 
 }  // namespace msda
