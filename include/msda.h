@@ -193,6 +193,37 @@ MSDA_API msda_status msda_fused_backward(const msda_problem *problem, const void
 MSDA_API msda_status msda_zero_grads(const msda_problem *problem, float *grad_value,
                                      float *grad_reference_points, msda_stream_t stream);
 
+/*
+ * msda_backward with grad_value written as bf16, for callers that cannot
+ * allocate device memory at call time (a host framework that gives an
+ * extension only its input and output tensors and no workspace, or a
+ * serving process whose device memory is fixed once it has started).  The
+ * pages on the operator have no counterpart of this entry point; it is an
+ * interface convenience of this library.
+ *   Arguments: as msda_backward, without the workspace; grad_value is
+ *   [B, S, M, D] bf16 (overwritten).  problem->flags may be 0 or
+ *   MSDA_GRAD_VALUE_BF16 (the output is bf16 either way).
+ *   Scratch: the float32 sums are kept in one buffer owned by the library,
+ *   4 Mi floats (16 MiB) per GPU, held until the process exits.  Problems with
+ *   B*S*M*D > 4 * 2^20 are rejected with MSDA_ERR_UNSUPPORTED before anything
+ *   is enqueued.  Nothing is allocated: no cudaMalloc, no cudaFree, no
+ *   allocating library routine.
+ *   The first call on a device looks up the buffer's device address (a CUDA
+ *   runtime query, once per device, with that device current); make that
+ *   first call before any stream capture.
+ *   Every call on a device shares the one buffer and clears it before use:
+ *   calls that overlap on the GPU (different streams, no ordering between
+ *   them) race on it and give wrong results.  Serialize them.
+ */
+MSDA_API msda_status msda_backward_noalloc(const msda_problem *problem, const void *value,
+                                           const int64_t *spatial_shapes,
+                                           const int64_t *level_start_index,
+                                           const float *sampling_locations,
+                                           const float *attention_weights,
+                                           const void *grad_output, void *grad_value,
+                                           float *grad_sampling_locations,
+                                           float *grad_attention_weights, msda_stream_t stream);
+
 /* Bytes of workspace msda_backward / msda_fused_backward need for `problem`
  * (0 unless MSDA_GRAD_VALUE_BF16 is set).  Host only; enqueues nothing. */
 MSDA_API msda_status msda_backward_workspace_size(const msda_problem *problem, size_t *bytes);

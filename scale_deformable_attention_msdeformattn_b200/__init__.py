@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     MSDeformAttnFunction,
     MSDeformAttnFusedFunction,
     backward,
+    backward_noalloc,
     device_status,
     forward,
     fused_backward,

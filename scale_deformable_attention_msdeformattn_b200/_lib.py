@@ -46,6 +46,7 @@ _SIGNATURES = {
     "msda_fused_backward": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "msda_backward_workspace_size": [_PROB, ctypes.POINTER(ctypes.c_size_t)],
     "msda_zero_grads": [_PROB, _P, _P, _P],
+    "msda_backward_noalloc": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "msda_get_device_status": [_P, ctypes.POINTER(ctypes.c_int32)],
     "msda_status_string": [ctypes.c_int],
     "msda_version": [],

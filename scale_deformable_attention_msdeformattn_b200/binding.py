@@ -253,6 +253,39 @@ def fused_backward(value, spatial_shapes, level_start_index, reference_points, s
     return grad_value, gref, goff, glog
 
 
+def backward_noalloc(value, spatial_shapes, level_start_index, sampling_locations,
+                     attention_weights, grad_output, grad_value: Optional[torch.Tensor] = None,
+                     grad_sampling_locations: Optional[torch.Tensor] = None,
+                     grad_attention_weights: Optional[torch.Tensor] = None):
+    """msda_backward_noalloc: backward with grad_value written as bf16, using
+    the library's own float32 scratch buffer instead of a workspace (for
+    callers that cannot allocate device memory when they run the backward).
+    Pass preallocated outputs to keep this call itself allocation-free."""
+    _need(value, "value", None)
+    L = _geometry(value, spatial_shapes, level_start_index)
+    B, S, M, D = value.shape
+    Q, K = sampling_locations.shape[1], sampling_locations.shape[4]
+    dev = value.device
+    _need(sampling_locations, "sampling_locations", torch.float32, (B, Q, M, L, K, 2), dev)
+    _need(attention_weights, "attention_weights", torch.float32, (B, Q, M, L, K), dev)
+    _need(grad_output, "grad_output", value.dtype, (B, Q, M, D), dev)
+    if grad_value is None:
+        grad_value = torch.empty((B, S, M, D), dtype=torch.bfloat16, device=dev)
+    if grad_sampling_locations is None:
+        grad_sampling_locations = torch.empty((B, Q, M, L, K, 2), dtype=torch.float32, device=dev)
+    if grad_attention_weights is None:
+        grad_attention_weights = torch.empty((B, Q, M, L, K), dtype=torch.float32, device=dev)
+    _need(grad_value, "grad_value", torch.bfloat16, (B, S, M, D), dev)
+    prob = _problem(value, Q, L, K, _lib.MSDA_GRAD_VALUE_BF16)
+    st = _lib.load().msda_backward_noalloc(ctypes.byref(prob), _ptr(value), _ptr(spatial_shapes),
+                                           _ptr(level_start_index), _ptr(sampling_locations),
+                                           _ptr(attention_weights), _ptr(grad_output),
+                                           _ptr(grad_value), _ptr(grad_sampling_locations),
+                                           _ptr(grad_attention_weights), _stream())
+    _check(st, "msda_backward_noalloc")
+    return grad_value, grad_sampling_locations, grad_attention_weights
+
+
 def zero_grads(grad_value: torch.Tensor, grad_reference_points: Optional[torch.Tensor] = None,
                num_queries: int = 0, num_levels: int = 1, num_points: int = 1):
     """msda_zero_grads: zeroes float32 grad_value [B, S, M, D] (and

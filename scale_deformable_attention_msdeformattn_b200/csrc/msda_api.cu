@@ -347,6 +347,36 @@ msda_status run_backward(const msda_problem *p, KernelArgs &a, void *grad_value,
     return MSDA_OK;
 }
 
+// Backward without any allocation ---------------------------------------------
+//
+// Some callers cannot allocate device memory when they run the backward pass:
+// a host framework that hands an extension only its input and output tensors
+// and no workspace, or a serving process whose device memory is fixed at
+// start-up and must not change while requests are in flight.  For them the
+// bf16-grad_value backward can accumulate in this library-owned buffer instead
+// of a caller workspace.  Every GPU that loads the library holds it until the
+// process exits.
+constexpr int64_t kNoAllocScratchFloats = int64_t(4) << 20;  // 16 MiB of float32
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+// Device address of g_noalloc_scratch, looked up once per device (with that
+// device current) on the first call there.  In host code the array's name is
+// only a host-side stand-in, never a device address.
+float *g_noalloc_ptr[kMaxDevices];
+
+msda_status noalloc_scratch(int dev, float **ptr)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return MSDA_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<float *>(p);
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return MSDA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -468,6 +498,54 @@ msda_status msda_zero_grads(const msda_problem *problem, float *grad_value,
     return launch_zero(grad_value, z.value, grad_reference_points,
                        grad_reference_points ? z.queries * 2 : 0,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_backward_noalloc(const msda_problem *problem, const void *value,
+                                  const int64_t *spatial_shapes, const int64_t *level_start_index,
+                                  const float *sampling_locations, const float *attention_weights,
+                                  const void *grad_output, void *grad_value,
+                                  float *grad_sampling_locations, float *grad_attention_weights,
+                                  msda_stream_t stream)
+{
+    msda_status st = check_problem(problem);
+    if (st != MSDA_OK)
+        return st;
+    if (problem->flags & ~(uint32_t)MSDA_GRAD_VALUE_BF16)
+        return MSDA_ERR_INVALID_ARG;
+    const Sizes z = sizes_of(problem);
+    if (z.value > kNoAllocScratchFloats)
+        return MSDA_ERR_UNSUPPORTED;
+    if (!vec_ptr_ok(value, z.value) || !geometry_ptrs_ok(problem, spatial_shapes, level_start_index) ||
+        !ptr_ok(sampling_locations, z.samples * 2) || !ptr_ok(attention_weights, z.samples) ||
+        !ptr_ok(grad_output, z.rows_d) || !ptr_ok(grad_value, z.value) ||
+        !ptr_ok(grad_sampling_locations, z.samples * 2) || !ptr_ok(grad_attention_weights, z.samples))
+        return MSDA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    st = current_device(dev, sms);
+    if (st != MSDA_OK)
+        return st;
+    float *acc = nullptr;
+    st = noalloc_scratch(dev, &acc);
+    if (st != MSDA_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    KernelArgs a = base_args(problem, value, spatial_shapes, level_start_index);
+    a.loc = sampling_locations;
+    a.attn = attention_weights;
+    a.grad_out = grad_output;
+    a.grad_loc = grad_sampling_locations;
+    a.grad_attn = grad_attention_weights;
+    a.grad_value = acc;
+    // the buffer keeps the previous call's sums: clear it first
+    st = launch_zero(acc, z.value, nullptr, 0, s);
+    if (st != MSDA_OK)
+        return st;
+    if (a.rows > 0) {
+        st = launch_backward<false>(problem, a, s);
+        if (st != MSDA_OK)
+            return st;
+    }
+    return launch_to_bf16(acc, grad_value, z.value, s);
 }
 
 msda_status msda_backward_workspace_size(const msda_problem *problem, size_t *bytes)
