@@ -601,6 +601,139 @@ __device__ __forceinline__ void setup_backward_row(const KernelArgs &a, const Ge
     }
 }
 
+// Warp-wide set-up of the backward for L*K = P a power of two <= 32: lane L
+// of round t takes sample (32 t + L) % P of the warp's row (32 t + L) / P, so
+// every input array is read with one contiguous load per round (the loads of
+// up to kWarpSetupRounds rounds are issued together), and the softmax of a row
+// is a reduction over its P lanes (one expf per sample).  Rows of the warp are
+// consecutive processing rows prow0 ..; nrows of them.  (The forward keeps the
+// per-group set-up: its register budget is spent on gathers in flight, and the
+// warp-wide form measured slower there.)
+
+__host__ __device__ __forceinline__ bool warp_setup_ok(int P) { return P <= 32 && (P & (P - 1)) == 0; }
+
+template <bool FUSED>
+__device__ __forceinline__ float seg_max(float v, int P)
+{
+    for (int o = P / 2; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float seg_sum(float v, int P)
+{
+    for (int o = P / 2; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Raw inputs of one sample of the warp-wide set-up, loaded ahead of the math
+// so that the loads of all rounds are in flight together.
+struct WarpIn {
+    float2 p;    // location (non-fused) or offset (fused)
+    float z;     // attention weight (non-fused) or logit (fused)
+    float2 r;    // reference point (fused)
+};
+
+template <bool FUSED>
+__device__ __forceinline__ WarpIn warp_load(const KernelArgs &a, int64_t row, bool active, int s,
+                                            int P, uint64_t pol)
+{
+    WarpIn in;
+    in.p = make_float2(0.f, 0.f);
+    in.r = make_float2(0.f, 0.f);
+    in.z = FUSED ? -INFINITY : 0.f;
+    if (active) {
+        const int64_t idx = row * P + s;
+        if (FUSED) {
+            in.p = ld_stream2(reinterpret_cast<const float2 *>(a.off) + idx, pol);
+            in.z = ld_stream(a.logits + idx, pol);
+            in.r = __ldg(reinterpret_cast<const float2 *>(a.ref) + row / a.M);
+        } else {
+            in.p = ld_stream2(reinterpret_cast<const float2 *>(a.loc) + idx, pol);
+            in.z = ld_stream(a.attn + idx, pol);
+        }
+    }
+    return in;
+}
+
+// Pixel coordinate and weight from the loaded inputs.  Every lane of the warp
+// must call (the softmax shuffles).
+template <bool FUSED>
+__device__ __forceinline__ void warp_sample(const KernelArgs &a, const Geometry &geo, const WarpIn &in,
+                                            bool active, int s, int P, int &l, double &x, double &y,
+                                            float &A)
+{
+    l = s / a.K;
+    const int H = geo.H[l], W = geo.W[l];
+    if (FUSED) {
+        const float mx = seg_max<true>(in.z, P);
+        const float e = active ? expf(in.z - mx) : 0.f;
+        const float sum = seg_sum(e, P);
+        A = active ? e / sum : 0.f;
+        pixel_from_offset(in.r.x, in.r.y, in.p.x, in.p.y, H, W, x, y);
+    } else {
+        A = in.z;
+        pixel_from_location(in.p.x, in.p.y, H, W, x, y);
+    }
+}
+
+constexpr int kWarpSetupRounds = 8;  // rounds whose loads are issued together
+
+// Backward records of the warp's rows (inactive rows and pad slots inert).
+template <bool FUSED>
+__device__ __forceinline__ void setup_backward_warp(const KernelArgs &a, const Geometry &geo,
+                                                    int64_t prow0, int nrows, int lane, uint64_t pol,
+                                                    int Pp, float4 *fa0, int4 *off0, float *As0,
+                                                    int stride)
+{
+    const int P = a.L * a.K;
+    const int per_round = 32 / P;
+    for (int rb = 0; rb < nrows; rb += per_round * kWarpSetupRounds) {
+        WarpIn in[kWarpSetupRounds];
+#pragma unroll
+        for (int t = 0; t < kWarpSetupRounds; ++t) {
+            const int rr = rb + t * per_round + lane / P;
+            const int64_t prow = prow0 + rr;
+            const bool active = rr < nrows && prow < a.rows;
+            in[t] = warp_load<FUSED>(a, active ? memory_row(a, prow) : 0, active, lane % P, P, pol);
+        }
+#pragma unroll
+        for (int t = 0; t < kWarpSetupRounds; ++t) {
+            if (rb + t * per_round >= nrows)
+                break;
+            const int rr = rb + t * per_round + lane / P, s = lane % P;
+            const int64_t prow = prow0 + rr;
+            const bool active = rr < nrows && prow < a.rows;
+            int l;
+            double x, y;
+            float A;
+            warp_sample<FUSED>(a, geo, in[t], active, s, P, l, x, y, A);
+            if (rr >= nrows)
+                continue;
+            const int k = rr * stride + s;
+            if (!active) {
+                fa0[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                off0[k] = make_int4(-1, 0, 0, 0);
+                continue;
+            }
+            const Corners c = corners_of(x, y, geo.H[l], geo.W[l], geo.start[l]);
+            const unsigned bits = (c.in[0] ? 1u : 0u) | (c.in[1] ? 2u : 0u) | (c.in[2] ? 4u : 0u) |
+                                  (c.in[3] ? 8u : 0u);
+            fa0[k] = make_float4(c.fx, c.fy, A, __uint_as_float(bits));
+            off0[k] = c.valid ? make_int4(c.key[0] * a.M, c.key[1] * a.M, c.key[2] * a.M, c.key[3] * a.M)
+                              : make_int4(-1, 0, 0, 0);
+            if (FUSED)
+                As0[k] = A;
+        }
+    }
+    // pad slots P .. Pp-1 (only when P is below the reduce-scatter chunk)
+    for (int k = lane; k < nrows * (Pp - P); k += 32) {
+        const int rr = k / (Pp - P), s = P + k % (Pp - P);
+        fa0[rr * stride + s] = make_float4(0.f, 0.f, 0.f, 0.f);
+        off0[rr * stride + s] = make_int4(-1, 0, 0, 0);
+    }
+}
+
 // ---------------------------------------------------------------- forward --
 
 template <typename T> struct FwdTune;
@@ -777,7 +910,12 @@ backward_kernel(const KernelArgs a)
         const int64_t prow = tile * a.rows_per_tile + slot;
         const bool active = prow < a.rows;
         const int64_t row = active ? memory_row(a, prow) : prow;
-        setup_backward_row<G, FUSED>(a, geo, row, active, gl, pol, Pp, fa, off, As);
+        if (warp_setup_ok(P))
+            setup_backward_warp<FUSED>(a, geo, tile * a.rows_per_tile + warp * Lay::kRowsPerWarp,
+                                       Lay::kRowsPerWarp, lane, pol, Pp, fa - grp * stride,
+                                       off - grp * stride, As - grp * stride, stride);
+        else
+            setup_backward_row<G, FUSED>(a, geo, row, active, gl, pol, Pp, fa, off, As);
         __syncwarp();
         const int64_t bq = active ? row / a.M : 0;
         const int m = active ? (int)(row - bq * a.M) : 0;
