@@ -74,7 +74,9 @@ typedef enum msda_status {
     MSDA_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad size */
     MSDA_ERR_UNSUPPORTED = 2,   /* valid, but outside the supported sizes */
     MSDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
-    MSDA_ERR_DEVICE_CHECK = 4   /* a kernel found inconsistent geometry */
+    MSDA_ERR_DEVICE_CHECK = 4,  /* a kernel found inconsistent geometry */
+    MSDA_ERR_DEVICE_TIMEOUT = 5 /* a kernel gave up waiting for an input copy
+                                   (bounded wait; the call's outputs are invalid) */
 } msda_status;
 
 typedef enum msda_dtype {
@@ -230,8 +232,8 @@ MSDA_API msda_status msda_backward_workspace_size(const msda_problem *problem, s
 
 /*
  * Synchronizes `stream`, then returns in *code the status the kernels recorded
- * on the current device since the last call (MSDA_OK or
- * MSDA_ERR_DEVICE_CHECK), and clears it.  Returns MSDA_ERR_CUDA if the
+ * on the current device since the last call (MSDA_OK, MSDA_ERR_DEVICE_CHECK or
+ * MSDA_ERR_DEVICE_TIMEOUT), and clears it.  Returns MSDA_ERR_CUDA if the
  * synchronization or the read fails.
  */
 MSDA_API msda_status msda_get_device_status(msda_stream_t stream, int32_t *code);

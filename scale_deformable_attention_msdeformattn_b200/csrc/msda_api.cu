@@ -166,16 +166,19 @@ msda_status occupancy(const void *kernel, int dev, int threads, size_t smem, int
 // Launches one compute kernel over all rows as a persistent wave; the row
 // records hold `padded_samples` slots.
 msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, int padded_samples,
-                        KernelArgs &a, cudaStream_t stream)
+                        bool stages, KernelArgs &a, cudaStream_t stream)
 {
     int dev = 0, sms = 0;
     msda_status st = current_device(dev, sms);
     if (st != MSDA_OK)
         return st;
-    const size_t per_warp = (size_t)rpw * msda::record_stride(padded_samples) * record_bytes;
-    int warps = (int)(kCtaSmemBudget / per_warp);
+    // records of the warp's rows, then (power-of-two L*K up to 32) the warp's
+    // double-buffered input stages; the kernel carves the same layout
+    const size_t rec_warp = (size_t)rpw * msda::record_stride(padded_samples) * record_bytes;
+    const size_t stage_warp = msda::stage_bytes_per_warp(stages, rpw, a.L * a.K);
+    int warps = (int)(kCtaSmemBudget / (rec_warp + stage_warp));
     warps = warps < 1 ? 1 : (warps > msda::kMaxWarpsPerCta ? msda::kMaxWarpsPerCta : warps);
-    const size_t smem = per_warp * warps;
+    const size_t smem = msda::align16(rec_warp * warps) + stage_warp * warps;
     const int threads = warps * 32;
     int blocks_per_sm = 0;
     st = occupancy(kernel, dev, threads, smem, blocks_per_sm);
@@ -238,7 +241,7 @@ msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
     case DD:                                                                                       \
         return launch_rows((const void *)msda::forward_kernel<T, DD, FUSED>,                     \
                            msda::forward_rows_per_warp<T, DD>(),                                 \
-                           kForwardRecordBytes, a.L * a.K, a, s);
+                           kForwardRecordBytes, a.L * a.K, msda::forward_stages<T>(), a, s);
     if (p->value_dtype == MSDA_F32) {
         switch (p->head_dim) {
             MSDA_FWD_CASE(float, 8) MSDA_FWD_CASE(float, 16) MSDA_FWD_CASE(float, 32)
@@ -263,7 +266,8 @@ msda_status launch_backward(const msda_problem *p, KernelArgs &a, cudaStream_t s
         return launch_rows((const void *)msda::backward_kernel<T, DD, FUSED>,                    \
                            msda::backward_rows_per_warp<T, DD>(),                                \
                            FUSED ? kFusedBackwardRecordBytes : kBackwardRecordBytes,             \
-                           msda::backward_padded_samples<T, DD>(a.L * a.K), a, s);
+                           msda::backward_padded_samples<T, DD>(a.L * a.K), msda::backward_stages(), \
+                           a, s);
     if (p->value_dtype == MSDA_F32) {
         switch (p->head_dim) {
             MSDA_BWD_CASE(float, 8) MSDA_BWD_CASE(float, 16) MSDA_BWD_CASE(float, 32)
@@ -583,6 +587,7 @@ const char *msda_status_string(msda_status status)
     case MSDA_ERR_UNSUPPORTED: return "sizes outside the supported range";
     case MSDA_ERR_CUDA: return "CUDA runtime error";
     case MSDA_ERR_DEVICE_CHECK: return "kernel found inconsistent spatial_shapes / level_start_index";
+    case MSDA_ERR_DEVICE_TIMEOUT: return "kernel gave up waiting for an input copy";
     }
     return "unknown status";
 }

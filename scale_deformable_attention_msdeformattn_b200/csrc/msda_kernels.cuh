@@ -43,6 +43,8 @@ namespace msda {
 // lane vectors, one sample in flight per lane and 3 CTAs per SM, and bf16
 // rows with 16-byte vectors and four samples in flight; the backward uses
 // 16-byte vectors (whole-sector grad_value reductions, more rows per warp).
+// TMA staging of the set-up inputs pays off in the float32 forward only (the
+// others measured slower with it).
 #ifndef MSDA_FWD_VB_F32
 #define MSDA_FWD_VB_F32 32
 #endif
@@ -60,6 +62,15 @@ namespace msda {
 #endif
 #ifndef MSDA_FWD_MIN_CTAS_BF16
 #define MSDA_FWD_MIN_CTAS_BF16 2
+#endif
+#ifndef MSDA_FWD_STAGE_F32           // TMA-staged set-up inputs (see "input staging")
+#define MSDA_FWD_STAGE_F32 1
+#endif
+#ifndef MSDA_FWD_STAGE_BF16
+#define MSDA_FWD_STAGE_BF16 0
+#endif
+#ifndef MSDA_BWD_STAGE
+#define MSDA_BWD_STAGE 0
 #endif
 #ifndef MSDA_BWD_VB
 #define MSDA_BWD_VB 16
@@ -601,6 +612,130 @@ __device__ __forceinline__ void setup_backward_row(const KernelArgs &a, const Ge
     }
 }
 
+// ----------------------------------------------------------- input staging --
+//
+// For L*K = P a power of two <= 32, each warp copies the set-up inputs of its
+// rows for the *next* tile (locations or offsets, and weights or logits) into
+// a shared-memory double buffer with the TMA bulk-copy engine
+// (cp.async.bulk, completion on an mbarrier) while it gathers the current
+// tile, so set-up loads leave the L1 load path and their latency is hidden.
+// A copy needs 16-byte aligned source and size: a warp slice qualifies when
+// (first row * P) and (rows * P) are multiples of 4; other slices (ragged
+// tails) and other P read global memory directly.  Waits are bounded: after
+// kStageSpinLimit polls the kernel records MSDA_ERR_DEVICE_TIMEOUT (5), gives
+// its other copy in flight a bounded chance to land, and returns.
+
+constexpr int kStageSpinLimit = 1 << 22;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *b)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, unsigned bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t *b, unsigned parity)
+{
+    uint32_t ok;
+    asm volatile("{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+                 " selp.u32 %0, 1, 0, p;\n}\n"
+                 : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait; false after kStageSpinLimit polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, unsigned parity)
+{
+    for (int i = 0; i < kStageSpinLimit; ++i) {
+        if (mbar_test(b, parity))
+            return true;
+        __nanosleep(32);
+    }
+    return false;
+}
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, unsigned bytes, uint64_t *bar,
+                                              uint64_t pol)
+{
+#if MSDA_STREAM_HINTS
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+                 " [%0], [%1], %2, [%3], %4;"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol) : "memory");
+#else
+    (void)pol;
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+#endif
+}
+
+// A warp's double buffer: per stage RPW * P location pairs and RPW * P
+// weights; two mbarriers.
+struct WarpStage {
+    float2 *p;      // [2][rpw * P]
+    float *z;       // [2][rpw * P]
+    uint64_t *bar;  // [2]
+    int cap;        // rpw * P
+};
+
+// Stage capacity (elements per stage) of a warp of rpw rows, 0 when the
+// inputs are never staged; bytes of a warp's stages and barriers.
+__host__ __device__ __forceinline__ int stage_cap(bool enabled, int rpw, int P)
+{
+    return (enabled && MSDA_HEAD_MAJOR == 0 && P <= 32 && (P & (P - 1)) == 0) ? ((rpw * P + 3) & ~3) : 0;
+}
+__host__ __device__ __forceinline__ size_t stage_bytes_per_warp(bool enabled, int rpw, int P)
+{
+    const int c = stage_cap(enabled, rpw, P);
+    return c ? (size_t)c * 2 * 12 + 16 : 0;
+}
+__host__ __device__ __forceinline__ size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+// Carves a warp's stages out of the shared memory after the records.
+__device__ __forceinline__ WarpStage warp_stage(unsigned char *base, int warp, int nwarps, int cap)
+{
+    WarpStage ws;
+    ws.cap = cap;
+    float2 *p_all = reinterpret_cast<float2 *>(base);
+    float *z_all = reinterpret_cast<float *>(p_all + (size_t)nwarps * 2 * cap);
+    uint64_t *b_all = reinterpret_cast<uint64_t *>(z_all + (size_t)nwarps * 2 * cap);
+    ws.p = p_all + (size_t)warp * 2 * cap;
+    ws.z = z_all + (size_t)warp * 2 * cap;
+    ws.bar = b_all + warp * 2;
+    return ws;
+}
+
+// Next tile of this CTA in the banded walk.
+__device__ __forceinline__ int64_t next_tile(int64_t tile)
+{
+    const int64_t band = (int64_t)gridDim.x * MSDA_BAND_TILES;
+    const int64_t i = (tile - (int64_t)blockIdx.x * MSDA_BAND_TILES) % band;
+    return (i + 1 < MSDA_BAND_TILES) ? tile + 1 : tile - i + band;
+}
+
+__device__ __forceinline__ bool stage_ok(int64_t prow0, int nv, int P)
+{
+    return nv > 0 && P <= 32 && (P & (P - 1)) == 0 && ((prow0 * P) & 3) == 0 && ((nv * P) & 3) == 0;
+}
+
+// Lane 0 starts the copies of the inputs of rows prow0 .. prow0 + nv - 1 into
+// stage st (the caller checked stage_ok).
+template <bool FUSED>
+__device__ __forceinline__ void stage_issue(const KernelArgs &a, const WarpStage &ws, int st, int64_t prow0,
+                                            int nv, int lane, uint64_t pol)
+{
+    if (lane != 0)
+        return;
+    const int P = a.L * a.K;
+    const unsigned np = (unsigned)(nv * P);
+    const float2 *src_p = reinterpret_cast<const float2 *>(FUSED ? a.off : a.loc) + prow0 * P;
+    const float *src_z = (FUSED ? a.logits : a.attn) + prow0 * P;
+    mbar_expect_tx(ws.bar + st, np * 12u);
+    bulk_copy_g2s(ws.p + st * ws.cap, src_p, np * 8u, ws.bar + st, pol);
+    bulk_copy_g2s(ws.z + st * ws.cap, src_z, np * 4u, ws.bar + st, pol);
+}
+
 // Warp-wide set-up of the backward for L*K = P a power of two <= 32: lane L
 // of round t takes sample (32 t + L) % P of the warp's row (32 t + L) / P, so
 // every input array is read with one contiguous load per round (the loads of
@@ -656,6 +791,24 @@ __device__ __forceinline__ WarpIn warp_load(const KernelArgs &a, int64_t row, bo
     return in;
 }
 
+// Same inputs from a shared-memory stage (element k of the warp's slice).
+template <bool FUSED>
+__device__ __forceinline__ WarpIn warp_load_staged(const KernelArgs &a, const float2 *sp, const float *sz,
+                                                   int k, int64_t row, bool active)
+{
+    WarpIn in;
+    in.p = make_float2(0.f, 0.f);
+    in.r = make_float2(0.f, 0.f);
+    in.z = FUSED ? -INFINITY : 0.f;
+    if (active) {
+        in.p = sp[k];
+        in.z = sz[k];
+        if (FUSED)
+            in.r = __ldg(reinterpret_cast<const float2 *>(a.ref) + row / a.M);
+    }
+    return in;
+}
+
 // Pixel coordinate and weight from the loaded inputs.  Every lane of the warp
 // must call (the softmax shuffles).
 template <bool FUSED>
@@ -684,7 +837,7 @@ template <bool FUSED>
 __device__ __forceinline__ void setup_backward_warp(const KernelArgs &a, const Geometry &geo,
                                                     int64_t prow0, int nrows, int lane, uint64_t pol,
                                                     int Pp, float4 *fa0, int4 *off0, float *As0,
-                                                    int stride)
+                                                    int stride, const float2 *sp, const float *sz)
 {
     const int P = a.L * a.K;
     const int per_round = 32 / P;
@@ -695,7 +848,9 @@ __device__ __forceinline__ void setup_backward_warp(const KernelArgs &a, const G
             const int rr = rb + t * per_round + lane / P;
             const int64_t prow = prow0 + rr;
             const bool active = rr < nrows && prow < a.rows;
-            in[t] = warp_load<FUSED>(a, active ? memory_row(a, prow) : 0, active, lane % P, P, pol);
+            const int64_t row = active ? memory_row(a, prow) : 0;
+            in[t] = sp ? warp_load_staged<FUSED>(a, sp, sz, rr * P + lane % P, row, active)
+                       : warp_load<FUSED>(a, row, active, lane % P, P, pol);
         }
 #pragma unroll
         for (int t = 0; t < kWarpSetupRounds; ++t) {
@@ -734,16 +889,56 @@ __device__ __forceinline__ void setup_backward_warp(const KernelArgs &a, const G
     }
 }
 
+// Forward records of the warp's rows from a shared-memory stage (staged
+// tiles only; the per-group set-up serves the others).
+template <bool FUSED>
+__device__ __forceinline__ void setup_forward_staged(const KernelArgs &a, const Geometry &geo,
+                                                     int64_t prow0, int nrows, int lane, uint64_t pol,
+                                                     float4 *wa0, int4 *off0, int stride,
+                                                     const float2 *sp, const float *sz)
+{
+    const int P = a.L * a.K;
+    const int per_round = 32 / P;
+    for (int r0 = 0; r0 < nrows; r0 += per_round) {
+        const int rr = r0 + lane / P, s = lane % P;
+        const int64_t prow = prow0 + rr;
+        const bool active = rr < nrows && prow < a.rows;
+        const int64_t row = active ? memory_row(a, prow) : 0;
+        const WarpIn in = warp_load_staged<FUSED>(a, sp, sz, rr * P + s, row, active);
+        int l;
+        double x, y;
+        float A;
+        warp_sample<FUSED>(a, geo, in, active, s, P, l, x, y, A);
+        if (!active)
+            continue;
+        if (FUSED && a.attn_out)
+            st_stream(a.attn_out + row * P + s, A, pol);
+        const Corners c = corners_of(x, y, geo.H[l], geo.W[l], geo.start[l]);
+        const float ay1 = A * c.fy, ay0 = A - ay1;
+        float4 w;
+        w.x = c.in[0] ? ay0 * (1.f - c.fx) : 0.f;
+        w.y = c.in[1] ? ay0 * c.fx : 0.f;
+        w.z = c.in[2] ? ay1 * (1.f - c.fx) : 0.f;
+        w.w = c.in[3] ? ay1 * c.fx : 0.f;
+        wa0[rr * stride + s] = w;
+        off0[rr * stride + s] = c.valid ? make_int4(c.key[0] * a.M, c.key[1] * a.M, c.key[2] * a.M,
+                                                    c.key[3] * a.M)
+                                        : make_int4(-1, 0, 0, 0);
+    }
+}
+
 // ---------------------------------------------------------------- forward --
 
 template <typename T> struct FwdTune;
 template <> struct FwdTune<float> {
     static constexpr int kVB = MSDA_FWD_VB_F32, kInFlight = MSDA_FWD_INFLIGHT_F32,
                          kMinCtas = MSDA_FWD_MIN_CTAS_F32;
+    static constexpr bool kStage = MSDA_FWD_STAGE_F32 != 0;
 };
 template <> struct FwdTune<__nv_bfloat16> {
     static constexpr int kVB = MSDA_FWD_VB_BF16, kInFlight = MSDA_FWD_INFLIGHT_BF16,
                          kMinCtas = MSDA_FWD_MIN_CTAS_BF16;
+    static constexpr bool kStage = MSDA_FWD_STAGE_BF16 != 0;
 };
 
 template <typename T, int D, bool FUSED>
@@ -769,14 +964,60 @@ forward_kernel(const KernelArgs a)
     float4 *wa = reinterpret_cast<float4 *>(smem_raw) + slot * stride;
     int4 *off = reinterpret_cast<int4 *>(smem_raw) + a.rows_per_tile * stride + slot * stride;
     const uint64_t pol = stream_policy();
-
-    const int64_t band = (int64_t)gridDim.x * MSDA_BAND_TILES;
-    for (int64_t tile0 = (int64_t)blockIdx.x * MSDA_BAND_TILES; tile0 < a.ntiles; tile0 += band)
-    for (int64_t tile = tile0; tile < min(tile0 + MSDA_BAND_TILES, a.ntiles); ++tile) {
+    constexpr int RPW = Lay::kRowsPerWarp;
+    const int cap = stage_cap(FwdTune<T>::kStage, RPW, P);
+    const WarpStage ws = warp_stage(smem_raw + align16((size_t)a.rows_per_tile * stride * 32), warp,
+                                    blockDim.x >> 5, cap);
+    if (cap) {
+        if (lane == 0) {
+            mbar_init(ws.bar);
+            mbar_init(ws.bar + 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        __syncwarp();
+    }
+    unsigned phase = 0;  // bit st: parity of the next completion of stage st
+    int k = 0;
+    int64_t tile = (int64_t)blockIdx.x * MSDA_BAND_TILES;
+    if (cap && tile < a.ntiles) {
+        const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
+        const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
+        if (stage_ok(p0, nv, P))
+            stage_issue<FUSED>(a, ws, 0, p0, nv, lane, pol);
+    }
+    for (; tile < a.ntiles; tile = next_tile(tile), ++k) {
+        const int st = k & 1;
+        const int64_t nxt = next_tile(tile);
+        bool next_staged = false;
+        if (cap && nxt < a.ntiles) {
+            const int64_t p0n = nxt * a.rows_per_tile + warp * RPW;
+            const int nvn = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0n));
+            next_staged = stage_ok(p0n, nvn, P);
+            if (next_staged) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                stage_issue<FUSED>(a, ws, st ^ 1, p0n, nvn, lane, pol);
+            }
+        }
         const int64_t prow = tile * a.rows_per_tile + slot;
         const bool active = prow < a.rows;
         const int64_t row = active ? memory_row(a, prow) : prow;
-        setup_forward_row<G, FUSED>(a, geo, row, active, gl, pol, wa, off);
+        const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
+        const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
+        if (cap && stage_ok(p0, nv, P)) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(ws.bar + st, (phase >> st) & 1u));
+            if (!ok) {
+                if (lane == 0)
+                    atomicExch(&g_device_status, 5 /* MSDA_ERR_DEVICE_TIMEOUT */);
+                if (next_staged)
+                    mbar_wait(ws.bar + (st ^ 1), (phase >> (st ^ 1)) & 1u);
+                return;
+            }
+            phase ^= 1u << st;
+            setup_forward_staged<FUSED>(a, geo, p0, RPW, lane, pol, wa - grp * stride, off - grp * stride,
+                                        stride, ws.p + st * cap, ws.z + st * cap);
+        } else {
+            setup_forward_row<G, FUSED>(a, geo, row, active, gl, pol, wa, off);
+        }
         __syncwarp();
         if (active) {
             const int64_t bq = row / a.M;
@@ -903,19 +1144,64 @@ backward_kernel(const KernelArgs a)
     float *gA = reinterpret_cast<float *>(reinterpret_cast<float4 *>(smem_raw) + 2 * arr) + slot * stride;
     float *As = gA + arr;
     const uint64_t pol = stream_policy();
-
-    const int64_t band = (int64_t)gridDim.x * MSDA_BAND_TILES;
-    for (int64_t tile0 = (int64_t)blockIdx.x * MSDA_BAND_TILES; tile0 < a.ntiles; tile0 += band)
-    for (int64_t tile = tile0; tile < min(tile0 + MSDA_BAND_TILES, a.ntiles); ++tile) {
+    constexpr int RPW = Lay::kRowsPerWarp;
+    const int cap = stage_cap(MSDA_BWD_STAGE != 0, RPW, P);
+    const WarpStage ws = warp_stage(smem_raw + align16((size_t)arr * (FUSED ? 40 : 32)), warp,
+                                    blockDim.x >> 5, cap);
+    if (cap) {
+        if (lane == 0) {
+            mbar_init(ws.bar);
+            mbar_init(ws.bar + 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        __syncwarp();
+    }
+    unsigned phase = 0;  // bit st: parity of the next completion of stage st
+    int k = 0;
+    int64_t tile = (int64_t)blockIdx.x * MSDA_BAND_TILES;
+    if (cap && tile < a.ntiles) {
+        const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
+        const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
+        if (stage_ok(p0, nv, P))
+            stage_issue<FUSED>(a, ws, 0, p0, nv, lane, pol);
+    }
+    for (; tile < a.ntiles; tile = next_tile(tile), ++k) {
+        const int st = k & 1;
+        const int64_t nxt = next_tile(tile);
+        bool next_staged = false;
+        if (cap && nxt < a.ntiles) {
+            const int64_t p0n = nxt * a.rows_per_tile + warp * RPW;
+            const int nvn = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0n));
+            next_staged = stage_ok(p0n, nvn, P);
+            if (next_staged) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                stage_issue<FUSED>(a, ws, st ^ 1, p0n, nvn, lane, pol);
+            }
+        }
         const int64_t prow = tile * a.rows_per_tile + slot;
         const bool active = prow < a.rows;
         const int64_t row = active ? memory_row(a, prow) : prow;
-        if (warp_setup_ok(P))
-            setup_backward_warp<FUSED>(a, geo, tile * a.rows_per_tile + warp * Lay::kRowsPerWarp,
-                                       Lay::kRowsPerWarp, lane, pol, Pp, fa - grp * stride,
-                                       off - grp * stride, As - grp * stride, stride);
-        else
+        const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
+        const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
+        if (cap && stage_ok(p0, nv, P)) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(ws.bar + st, (phase >> st) & 1u));
+            if (!ok) {
+                if (lane == 0)
+                    atomicExch(&g_device_status, 5 /* MSDA_ERR_DEVICE_TIMEOUT */);
+                if (next_staged)
+                    mbar_wait(ws.bar + (st ^ 1), (phase >> (st ^ 1)) & 1u);
+                return;
+            }
+            phase ^= 1u << st;
+            setup_backward_warp<FUSED>(a, geo, p0, RPW, lane, pol, Pp, fa - grp * stride,
+                                       off - grp * stride, As - grp * stride, stride, ws.p + st * cap,
+                                       ws.z + st * cap);
+        } else if (warp_setup_ok(P)) {
+            setup_backward_warp<FUSED>(a, geo, p0, RPW, lane, pol, Pp, fa - grp * stride,
+                                       off - grp * stride, As - grp * stride, stride, nullptr, nullptr);
+        } else {
             setup_backward_row<G, FUSED>(a, geo, row, active, gl, pol, Pp, fa, off, As);
+        }
         __syncwarp();
         const int64_t bq = active ? row / a.M : 0;
         const int m = active ? (int)(row - bq * a.M) : 0;
@@ -1067,6 +1353,8 @@ __global__ void f32_to_bf16_kernel(const float4 *src, uint4 *dst, int64_t n8)
 
 // Rows per warp of each kernel (the host sizes CTAs and shared memory by it).
 template <typename T, int D> constexpr int forward_rows_per_warp() { return Layout<T, D, FwdTune<T>::kVB>::kRowsPerWarp; }
+template <typename T> constexpr bool forward_stages() { return FwdTune<T>::kStage; }
+constexpr bool backward_stages() { return MSDA_BWD_STAGE != 0; }
 template <typename T, int D> constexpr int backward_rows_per_warp() { return Layout<T, D, MSDA_BWD_VB>::kRowsPerWarp; }
 // Record slots of a backward row: L*K rounded up to the reduce-scatter chunk.
 template <typename T, int D> inline int backward_padded_samples(int P)
