@@ -90,6 +90,12 @@ typedef enum msda_dtype {
 #define MSDA_ACCUMULATE_GRADS (1u << 1) /* backward adds into grad_value (and
                                           grad_reference_points) instead of
                                           zeroing them first; float32 only */
+#define MSDA_TEST_WITHHOLD_COPY (1u << 31) /* testing only: kernels that stage
+                                          their inputs with bulk copies arm
+                                          the copy but never issue it, so
+                                          their bounded wait runs out and
+                                          they report MSDA_ERR_DEVICE_TIMEOUT
+                                          (outputs are then invalid) */
 
 /* Sizes of one call.  S = sum_l H_l * W_l. */
 typedef struct msda_problem {

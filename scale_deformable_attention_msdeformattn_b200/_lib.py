@@ -22,6 +22,7 @@ MSDA_BF16 = 1
 
 MSDA_GRAD_VALUE_BF16 = 1 << 0
 MSDA_ACCUMULATE_GRADS = 1 << 1
+MSDA_TEST_WITHHOLD_COPY = 1 << 31
 
 
 class Problem(ctypes.Structure):

@@ -53,7 +53,7 @@ msda_status check_problem(const msda_problem *p)
         return MSDA_ERR_INVALID_ARG;
     if (p->value_dtype != MSDA_F32 && p->value_dtype != MSDA_BF16)
         return MSDA_ERR_INVALID_ARG;
-    if (p->flags & ~(uint32_t)(MSDA_GRAD_VALUE_BF16 | MSDA_ACCUMULATE_GRADS))
+    if (p->flags & ~(uint32_t)(MSDA_GRAD_VALUE_BF16 | MSDA_ACCUMULATE_GRADS | MSDA_TEST_WITHHOLD_COPY))
         return MSDA_ERR_INVALID_ARG;
     if ((p->flags & MSDA_GRAD_VALUE_BF16) && (p->flags & MSDA_ACCUMULATE_GRADS))
         return MSDA_ERR_INVALID_ARG;
@@ -297,6 +297,7 @@ KernelArgs base_args(const msda_problem *p, const void *value, const int64_t *sh
     a.M = p->num_heads;
     a.L = p->num_levels;
     a.K = p->num_points;
+    a.withhold_copy = (p->flags & MSDA_TEST_WITHHOLD_COPY) ? 1 : 0;
     return a;
 }
 

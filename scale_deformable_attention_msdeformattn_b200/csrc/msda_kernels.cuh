@@ -117,6 +117,7 @@ struct KernelArgs {
     int64_t ntiles;         // ceil(rows / rows_per_tile)
     int64_t S;
     int Q, M, L, K;
+    int withhold_copy;      // testing: arm the input copies but never issue them
 };
 
 struct Geometry {
@@ -732,6 +733,8 @@ __device__ __forceinline__ void stage_issue(const KernelArgs &a, const WarpStage
     const float2 *src_p = reinterpret_cast<const float2 *>(FUSED ? a.off : a.loc) + prow0 * P;
     const float *src_z = (FUSED ? a.logits : a.attn) + prow0 * P;
     mbar_expect_tx(ws.bar + st, np * 12u);
+    if (a.withhold_copy)
+        return;  // the wait for this stage runs out (failure-path test)
     bulk_copy_g2s(ws.p + st * ws.cap, src_p, np * 8u, ws.bar + st, pol);
     bulk_copy_g2s(ws.z + st * ws.cap, src_z, np * 4u, ws.bar + st, pol);
 }
@@ -1008,7 +1011,7 @@ forward_kernel(const KernelArgs a)
             if (!ok) {
                 if (lane == 0)
                     atomicExch(&g_device_status, 5 /* MSDA_ERR_DEVICE_TIMEOUT */);
-                if (next_staged)
+                if (next_staged && !a.withhold_copy)
                     mbar_wait(ws.bar + (st ^ 1), (phase >> (st ^ 1)) & 1u);
                 return;
             }
@@ -1188,7 +1191,7 @@ backward_kernel(const KernelArgs a)
             if (!ok) {
                 if (lane == 0)
                     atomicExch(&g_device_status, 5 /* MSDA_ERR_DEVICE_TIMEOUT */);
-                if (next_staged)
+                if (next_staged && !a.withhold_copy)
                     mbar_wait(ws.bar + (st ^ 1), (phase >> (st ^ 1)) & 1u);
                 return;
             }
