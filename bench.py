@@ -75,6 +75,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-nonfused", action="store_true")
+    ap.add_argument("--sorted", action="store_true",
+                    help="order the queries by the Morton cell of their reference point "
+                         "(msda_sort_queries, inside the timed step) and process them in that order")
     ap.add_argument("--out", default=None, help="also append the JSON line to this file")
     a = ap.parse_args(argv)
     if a.warmup < 3:
@@ -281,6 +284,7 @@ def run_ours(args):
                "grad_sampling_offsets": goff, "grad_attention_logits": glog}
 
     side = torch.cuda.Stream(device=dev)
+    order = torch.empty(B * Q, dtype=torch.int32, device=dev) if args.sorted else None
 
     def step(ev, tin=None):
         # the zero-fill of the gradient accumulators does not depend on the
@@ -288,14 +292,17 @@ def run_ours(args):
         # backward waits for both
         tin = tin or t
         ev[0].record(stream)
-        side.wait_event(ev[0])
+        if order is not None:
+            msda.sort_queries(tin["reference_points"], query_order=order)
+        ev[6].record(stream)
+        side.wait_event(ev[6])
         with torch.cuda.stream(side):
             ev[4].record(side)
             msda.zero_grads(gv, gref)
             ev[5].record(side)
         msda.fused_forward(tin["value"], tin["spatial_shapes"], tin["level_start_index"],
                            tin["reference_points"], tin["sampling_offsets"],
-                           tin["attention_logits"], out=out)
+                           tin["attention_logits"], out=out, query_order=order)
         ev[1].record(stream)
         stream.wait_event(ev[5])
         ev[2].record(stream)
@@ -303,12 +310,13 @@ def run_ours(args):
                             tin["reference_points"], tin["sampling_offsets"],
                             tin["attention_logits"], tin["grad_output"], accumulate=True,
                             grad_value=gv, grad_reference_points=gref,
-                            grad_sampling_offsets=goff, grad_attention_logits=glog)
+                            grad_sampling_offsets=goff, grad_attention_logits=glog,
+                            query_order=order)
         ev[3].record(stream)
         return outputs
 
     def events(n):
-        return [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n)]
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(n)]
 
     warm = events(args.warmup)
     for i in range(args.warmup):
@@ -332,7 +340,8 @@ def run_ours(args):
     barrier()
     clocks.stop()
 
-    fwd = [e[0].elapsed_time(e[1]) for e in evs]
+    fwd = [e[6].elapsed_time(e[1]) for e in evs]
+    sort = [e[0].elapsed_time(e[6]) for e in evs]
     zero = [e[4].elapsed_time(e[5]) for e in evs]  # on the side stream, under the forward
     bwd = [e[2].elapsed_time(e[3]) for e in evs]
     stepms = [e[0].elapsed_time(e[3]) for e in evs]
@@ -370,12 +379,15 @@ def run_ours(args):
                 "Q": Q, "M": M, "D": D, "L": L, "K": K,
                 "offset_sigma_px": w.offset_sigma, "logit_sigma": w.logit_sigma,
                 "samples_per_step_per_gpu": samples_step,
-                "step": "msda_fused_forward || msda_zero_grads (second stream) -> msda_fused_backward",
+                "step": ("msda_sort_queries -> " if args.sorted else "")
+                + "msda_fused_forward || msda_zero_grads (second stream) -> msda_fused_backward",
+                "query_order": "Morton cell of the reference point" if args.sorted else "natural",
                 "l2": "flushed between steps (256 MiB write outside the timed events)",
                 "parallelism": f"dp{world} (independent batch per GPU)",
             },
             "fwd_ms": round(fwd_ms, 5),
             "zero_ms": round(zero_ms, 5),  # overlapped with the forward
+            "sort_ms": round(statistics.mean(sort), 5) if args.sorted else None,
 
             "bwd_ms": round(bwd_ms, 5),
             "fwd_gsamples_per_s": round(samples_step / (fwd_ms * 1e-3) / 1e9, 4),
@@ -392,7 +404,7 @@ def run_ours(args):
                 "bytes_per_launch": nbytes[dom],
                 "traffic": traffic,
             },
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (4 if args.sorted else 3) * args.steps,
             "host_wall_s": round(wall, 3),
             "clocks": clocks.summary(),
         }
@@ -488,7 +500,7 @@ def _time_e2e(msda, x, t, w, step, flush, n, dev):
         e0.record(stream)
         for k in hin:
             din[k].copy_(hin[k], non_blocking=True)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
         outs = step(ev, din)
         for k in res_names:
             hout[k].copy_(outs[k], non_blocking=True)

@@ -46,6 +46,7 @@
  *     returns an error has enqueued nothing.
  *   - Supported sizes: D (head_dim) in {8, 16, 32, 64, 128, 256};
  *     1 <= L <= 16; 1 <= K <= 32; L*K <= 128; 1 <= M; S < 2^27; S*M < 2^31;
+ *     B*Q < 2^31;
  *     B*Q*M*L*K < 2^40; B or Q may be 0 (nothing to sample).
  *   - No C++ exception crosses this boundary.
  */
@@ -74,7 +75,7 @@ typedef enum msda_status {
     MSDA_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, bad size */
     MSDA_ERR_UNSUPPORTED = 2,   /* valid, but outside the supported sizes */
     MSDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
-    MSDA_ERR_DEVICE_CHECK = 4,  /* a kernel found inconsistent geometry */
+    MSDA_ERR_DEVICE_CHECK = 4,  /* a kernel found inconsistent geometry or a bad query_order entry */
     MSDA_ERR_DEVICE_TIMEOUT = 5 /* a kernel gave up waiting for an input copy
                                    (bounded wait; the call's outputs are invalid) */
 } msda_status;
@@ -108,6 +109,17 @@ typedef struct msda_problem {
     int32_t num_points;   /* K */
     int32_t value_dtype;  /* msda_dtype of value, output, grad_output */
     uint32_t flags;       /* MSDA_* flags above */
+    /* Optional device array [B*Q] int32, 4-byte aligned: the order in which
+     * the kernels process the queries, a permutation of 0 .. B*Q-1 (query
+     * index b*Q + q), e.g. from msda_sort_queries.  NULL: natural order.
+     * Each query's outputs are computed as in the natural order; what can
+     * change is float32 rounding where the order decides the summation
+     * order (grad_value, and the fused softmax sums, whose reduction pattern
+     * can differ between ordered and natural-order set-up).  An entry outside 0 .. B*Q-1 is replaced by 0 and sets the
+     * device status to MSDA_ERR_DEVICE_CHECK; repeated entries are not
+     * detected (the rows of queries missing from the order are not written).
+     * Read by the kernels on the stream: it must stay valid until they end. */
+    const int32_t *query_order;
 } msda_problem;
 
 /*
@@ -231,6 +243,21 @@ MSDA_API msda_status msda_backward_noalloc(const msda_problem *problem, const vo
                                            const void *grad_output, void *grad_value,
                                            float *grad_sampling_locations,
                                            float *grad_attention_weights, msda_stream_t stream);
+
+/*
+ * Processing order that keeps spatially close queries together (the optional
+ * query-sorting step of the operator's data-locality notes,
+ * x-humanoid.csdn.net MSDA explainer §4 "pre-processing and reordering"):
+ * writes into query_order [B*Q] (int32, 4-byte aligned) a permutation of the
+ * B*Q queries sorted by batch, then by the Morton code of the 64 x 64 cell of
+ * [0,1]^2 that holds the query's point (coordinates outside [0,1] are
+ * clamped, NaN counts as 0; the order within a cell is unspecified).
+ * points [B, Q, 2] float32 (x, y), 16-byte aligned, typically the reference
+ * points.  One kernel, one CTA per batch, no workspace.  Only batch, num_queries
+ * and the validity of the rest of `problem` are used.  Asynchronous on `stream`.
+ */
+MSDA_API msda_status msda_sort_queries(const msda_problem *problem, const float *points,
+                                       int32_t *query_order, msda_stream_t stream);
 
 /* Bytes of workspace msda_backward / msda_fused_backward need for `problem`
  * (0 unless MSDA_GRAD_VALUE_BF16 is set).  Host only; enqueues nothing. */

@@ -36,6 +36,7 @@ class Problem(ctypes.Structure):
         ("num_points", ctypes.c_int32),
         ("value_dtype", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
+        ("query_order", ctypes.c_void_p),
     ]
 
 
@@ -49,6 +50,7 @@ _SIGNATURES = {
     "msda_backward_workspace_size": [_PROB, ctypes.POINTER(ctypes.c_size_t)],
     "msda_zero_grads": [_PROB, _P, _P, _P],
     "msda_backward_noalloc": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "msda_sort_queries": [_PROB, _P, _P, _P],
     "msda_get_device_status": [_P, ctypes.POINTER(ctypes.c_int32)],
     "msda_status_string": [ctypes.c_int],
     "msda_version": [],

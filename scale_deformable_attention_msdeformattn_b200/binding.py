@@ -68,13 +68,20 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None, device=None):
 _DTYPES = {torch.float32: _lib.MSDA_F32, torch.bfloat16: _lib.MSDA_BF16}
 
 
-def _problem(value: torch.Tensor, Q: int, L: int, K: int, flags: int = 0) -> _lib.Problem:
+def _problem(value: torch.Tensor, Q: int, L: int, K: int, flags: int = 0,
+             query_order: Optional[torch.Tensor] = None) -> _lib.Problem:
     if value.dim() != 4:
         raise ValueError("value must be [B, S, M, D]")
     if value.dtype not in _DTYPES:
         raise TypeError("value must be float32 or bfloat16")
     B, S, M, D = value.shape
-    return _lib.Problem(B, S, Q, M, D, L, K, _DTYPES[value.dtype], flags)
+    prob = _lib.Problem(B, S, Q, M, D, L, K, _DTYPES[value.dtype], flags)
+    if query_order is not None:
+        if query_order.numel() != B * Q:
+            raise ValueError(f"query_order must hold B*Q = {B * Q} entries")
+        _need(query_order, "query_order", torch.int32, None, value.device)
+        prob.query_order = _ptr(query_order)
+    return prob
 
 
 def _geometry(value, spatial_shapes, level_start_index):
@@ -88,8 +95,10 @@ def _geometry(value, spatial_shapes, level_start_index):
 
 def forward(value: torch.Tensor, spatial_shapes: torch.Tensor, level_start_index: torch.Tensor,
             sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
-            out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """msda_forward: returns out [B, Q, M, D] in value's dtype."""
+            out: Optional[torch.Tensor] = None,
+            query_order: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """msda_forward: returns out [B, Q, M, D] in value's dtype.  query_order:
+    optional int32 [B*Q] processing order (see sort_queries)."""
     _need(value, "value", None)
     L = _geometry(value, spatial_shapes, level_start_index)
     B, S, M, D = value.shape
@@ -101,7 +110,7 @@ def forward(value: torch.Tensor, spatial_shapes: torch.Tensor, level_start_index
     if out is None:
         out = torch.empty((B, Q, M, D), dtype=value.dtype, device=value.device)
     _need(out, "out", value.dtype, (B, Q, M, D), value.device)
-    prob = _problem(value, Q, L, K)
+    prob = _problem(value, Q, L, K, 0, query_order)
     st = _lib.load().msda_forward(ctypes.byref(prob), _ptr(value), _ptr(spatial_shapes),
                                   _ptr(level_start_index), _ptr(sampling_locations),
                                   _ptr(attention_weights), _ptr(out), _stream())
@@ -115,7 +124,8 @@ def backward(value, spatial_shapes, level_start_index, sampling_locations, atten
              grad_sampling_locations: Optional[torch.Tensor] = None,
              grad_attention_weights: Optional[torch.Tensor] = None,
              workspace: Optional[torch.Tensor] = None,
-             accumulate: bool = False) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+             accumulate: bool = False,
+             query_order: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """msda_backward: (grad_value, grad_sampling_locations, grad_attention_weights).
 
     accumulate=True adds into the given float32 grad_value instead of
@@ -142,7 +152,7 @@ def backward(value, spatial_shapes, level_start_index, sampling_locations, atten
     if grad_attention_weights is None:
         grad_attention_weights = torch.empty((B, Q, M, L, K), dtype=torch.float32, device=dev)
     _need(grad_value, "grad_value", grad_value_dtype, (B, S, M, D), dev)
-    prob = _problem(value, Q, L, K, flags)
+    prob = _problem(value, Q, L, K, flags, query_order)
     lib = _lib.load()
     ws_bytes = ctypes.c_size_t(0)
     _check(lib.msda_backward_workspace_size(ctypes.byref(prob), ctypes.byref(ws_bytes)),
@@ -167,7 +177,8 @@ def _logits(attention_logits, B, Q, M, L, K, dev):
 
 def fused_forward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
                   attention_logits, return_attention_weights: bool = False,
-                  out: Optional[torch.Tensor] = None):
+                  out: Optional[torch.Tensor] = None,
+                  query_order: Optional[torch.Tensor] = None):
     """msda_fused_forward: out [B, Q, M, D] (and the softmax weights if asked)."""
     _need(value, "value", None)
     L = _geometry(value, spatial_shapes, level_start_index)
@@ -183,7 +194,7 @@ def fused_forward(value, spatial_shapes, level_start_index, reference_points, sa
         out = torch.empty((B, Q, M, D), dtype=value.dtype, device=dev)
     _need(out, "out", value.dtype, (B, Q, M, D), dev)
     attn = torch.empty((B, Q, M, L, K), dtype=torch.float32, device=dev) if return_attention_weights else None
-    prob = _problem(value, Q, L, K)
+    prob = _problem(value, Q, L, K, 0, query_order)
     st = _lib.load().msda_fused_forward(ctypes.byref(prob), _ptr(value), _ptr(spatial_shapes),
                                         _ptr(level_start_index), _ptr(reference_points),
                                         _ptr(sampling_offsets), _ptr(attention_logits), _ptr(out),
@@ -200,7 +211,8 @@ def fused_backward(value, spatial_shapes, level_start_index, reference_points, s
                    accumulate: bool = False,
                    grad_reference_points: Optional[torch.Tensor] = None,
                    grad_sampling_offsets: Optional[torch.Tensor] = None,
-                   grad_attention_logits: Optional[torch.Tensor] = None):
+                   grad_attention_logits: Optional[torch.Tensor] = None,
+                   query_order: Optional[torch.Tensor] = None):
     """msda_fused_backward: (grad_value, grad_reference_points or None,
     grad_sampling_offsets, grad_attention_logits [B, Q, M, L*K]).
 
@@ -236,7 +248,7 @@ def fused_backward(value, spatial_shapes, level_start_index, reference_points, s
     glog = grad_attention_logits if grad_attention_logits is not None else \
         torch.empty((B, Q, M, L * K), dtype=torch.float32, device=dev)
     _need(glog, "grad_attention_logits", torch.float32, (B, Q, M, L * K), dev)
-    prob = _problem(value, Q, L, K, flags)
+    prob = _problem(value, Q, L, K, flags, query_order)
     lib = _lib.load()
     ws_bytes = ctypes.c_size_t(0)
     _check(lib.msda_backward_workspace_size(ctypes.byref(prob), ctypes.byref(ws_bytes)),
@@ -284,6 +296,25 @@ def backward_noalloc(value, spatial_shapes, level_start_index, sampling_location
                                            _ptr(grad_attention_weights), _stream())
     _check(st, "msda_backward_noalloc")
     return grad_value, grad_sampling_locations, grad_attention_weights
+
+
+def sort_queries(points: torch.Tensor, query_order: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """msda_sort_queries: int32 [B*Q] order of the queries by batch, then by
+    the Morton code of the 64 x 64 cell of [0,1]^2 holding points[b, q]
+    (float32 [B, Q, 2], e.g. the reference points).  Pass the result as
+    query_order to the other calls."""
+    _need(points, "points", torch.float32)
+    if points.dim() != 3 or points.shape[2] != 2:
+        raise ValueError("points must be [B, Q, 2]")
+    B, Q = points.shape[0], points.shape[1]
+    dev = points.device
+    prob = _lib.Problem(B, 1, Q, 1, 8, 1, 1, _lib.MSDA_F32, 0)
+    if query_order is None:
+        query_order = torch.empty(B * Q, dtype=torch.int32, device=dev)
+    _need(query_order, "query_order", torch.int32, (B * Q,), dev)
+    st = _lib.load().msda_sort_queries(ctypes.byref(prob), _ptr(points), _ptr(query_order), _stream())
+    _check(st, "msda_sort_queries")
+    return query_order
 
 
 def zero_grads(grad_value: torch.Tensor, grad_reference_points: Optional[torch.Tensor] = None,

@@ -77,6 +77,10 @@ msda_status check_problem(const msda_problem *p)
     const double values = (double)p->batch * (double)p->num_keys * p->num_heads * p->head_dim;
     if (values >= 9.0e18)
         return MSDA_ERR_UNSUPPORTED;
+    if ((double)p->batch * (double)p->num_queries >= 2147483648.0)
+        return MSDA_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(p->query_order) & 3u)
+        return MSDA_ERR_INVALID_ARG;
     return MSDA_OK;
 }
 
@@ -298,6 +302,7 @@ KernelArgs base_args(const msda_problem *p, const void *value, const int64_t *sh
     a.L = p->num_levels;
     a.K = p->num_points;
     a.withhold_copy = (p->flags & MSDA_TEST_WITHHOLD_COPY) ? 1 : 0;
+    a.order = (p->batch * p->num_queries > 0) ? p->query_order : nullptr;
     return a;
 }
 
@@ -553,6 +558,23 @@ msda_status msda_backward_noalloc(const msda_problem *problem, const void *value
     return launch_to_bf16(acc, grad_value, z.value, s);
 }
 
+msda_status msda_sort_queries(const msda_problem *problem, const float *points, int32_t *query_order,
+                              msda_stream_t stream)
+{
+    msda_status st = check_problem(problem);
+    if (st != MSDA_OK)
+        return st;
+    const int64_t bq = problem->batch * problem->num_queries;
+    if (bq == 0)
+        return MSDA_OK;
+    if (!ptr_ok(points, bq * 2) || !query_order || (reinterpret_cast<uintptr_t>(query_order) & 3u))
+        return MSDA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    msda::sort_queries_kernel<<<(unsigned)problem->batch, msda::kSortThreads, 0, s>>>(
+        reinterpret_cast<const float2 *>(points), problem->num_queries, query_order);
+    return cudaGetLastError() == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
+}
+
 msda_status msda_backward_workspace_size(const msda_problem *problem, size_t *bytes)
 {
     msda_status st = check_problem(problem);
@@ -587,7 +609,7 @@ const char *msda_status_string(msda_status status)
     case MSDA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or bad size)";
     case MSDA_ERR_UNSUPPORTED: return "sizes outside the supported range";
     case MSDA_ERR_CUDA: return "CUDA runtime error";
-    case MSDA_ERR_DEVICE_CHECK: return "kernel found inconsistent spatial_shapes / level_start_index";
+    case MSDA_ERR_DEVICE_CHECK: return "kernel found inconsistent spatial_shapes / level_start_index or a query_order entry out of range";
     case MSDA_ERR_DEVICE_TIMEOUT: return "kernel gave up waiting for an input copy";
     }
     return "unknown status";

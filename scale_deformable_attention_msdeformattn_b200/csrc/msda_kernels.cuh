@@ -118,6 +118,7 @@ struct KernelArgs {
     int64_t S;
     int Q, M, L, K;
     int withhold_copy;      // testing: arm the input copies but never issue them
+    const int32_t *order;   // optional processing order of the B*Q queries
 };
 
 struct Geometry {
@@ -402,10 +403,21 @@ __device__ __forceinline__ float4 ld_grad4<__nv_bfloat16>(const __nv_bfloat16 *r
 // footprint).
 //
 // Processing row p maps to memory row (b * Q + q) * M + m; head-major order
-// takes p = (m * B + b) * Q + q.
+// takes p = (m * B + b) * Q + q; with a query order the p-th query is order[p / M].
 
 __device__ __forceinline__ int64_t memory_row(const KernelArgs &a, int64_t p)
 {
+    if (a.order) {
+        // processing row p is head p % M of the (p / M)-th query of the order;
+        // an entry outside 0 .. B*Q-1 is reported and replaced by query 0
+        const int64_t qi = p / a.M;
+        int64_t q = __ldg(a.order + qi);
+        if (q < 0 || q * a.M >= a.rows) {
+            atomicExch(&g_device_status, 4 /* MSDA_ERR_DEVICE_CHECK */);
+            q = 0;
+        }
+        return q * a.M + (p - qi * a.M);
+    }
 #if MSDA_HEAD_MAJOR
     const int64_t BQ = a.rows / a.M;
     const int64_t m = p / BQ;
@@ -968,7 +980,7 @@ forward_kernel(const KernelArgs a)
     int4 *off = reinterpret_cast<int4 *>(smem_raw) + a.rows_per_tile * stride + slot * stride;
     const uint64_t pol = stream_policy();
     constexpr int RPW = Lay::kRowsPerWarp;
-    const int cap = stage_cap(FwdTune<T>::kStage, RPW, P);
+    const int cap = a.order ? 0 : stage_cap(FwdTune<T>::kStage, RPW, P);  // staged slices are contiguous rows
     const WarpStage ws = warp_stage(smem_raw + align16((size_t)a.rows_per_tile * stride * 32), warp,
                                     blockDim.x >> 5, cap);
     if (cap) {
@@ -1148,7 +1160,7 @@ backward_kernel(const KernelArgs a)
     float *As = gA + arr;
     const uint64_t pol = stream_policy();
     constexpr int RPW = Lay::kRowsPerWarp;
-    const int cap = stage_cap(MSDA_BWD_STAGE != 0, RPW, P);
+    const int cap = a.order ? 0 : stage_cap(MSDA_BWD_STAGE != 0, RPW, P);
     const WarpStage ws = warp_stage(smem_raw + align16((size_t)arr * (FUSED ? 40 : 32)), warp,
                                     blockDim.x >> 5, cap);
     if (cap) {
@@ -1351,6 +1363,115 @@ __global__ void f32_to_bf16_kernel(const float4 *src, uint4 *dst, int64_t n8)
         uint4 r;
         Elem<__nv_bfloat16>::narrow<4>(f, reinterpret_cast<uint32_t *>(&r));
         dst[i] = r;
+    }
+}
+
+// ------------------------------------------------------------ query order --
+//
+// Counting sort of each batch's queries by the Morton code of the 64 x 64 cell
+// of [0,1]^2 holding their point, in one kernel: one CTA of 1024 threads per
+// batch counts the queries per cell in shared memory, scans the counts, then
+// hands each query the next slot of its cell.  Each pass reads the batch's
+// points with kSortInFlight loads in flight per thread.
+
+constexpr int kSortCells = 64;  // cells per axis of [0,1]^2
+constexpr int kSortThreads = 1024, kSortInFlight = 8;
+
+__device__ __forceinline__ uint32_t spread_bits6(uint32_t v)  // 6 bits -> even bit positions
+{
+    v &= 63u;
+    v = (v | (v << 4)) & 0x0f0fu;
+    v = (v | (v << 2)) & 0x3333u;
+    v = (v | (v << 1)) & 0x5555u;
+    return v;
+}
+
+__device__ __forceinline__ uint32_t cell_code(float2 p)
+{
+    // fminf / fmaxf map NaN to the other operand, so every point gets a cell
+    const float fx = fminf(fmaxf(p.x * kSortCells, 0.f), kSortCells - 1.f);
+    const float fy = fminf(fmaxf(p.y * kSortCells, 0.f), kSortCells - 1.f);
+    return spread_bits6((uint32_t)fx) | (spread_bits6((uint32_t)fy) << 1);
+}
+
+// Cell codes of the points i0 + j * kSortThreads + t (j < kSortInFlight);
+// ~0u past the end.
+__device__ __forceinline__ void cell_codes(const float2 *p, int64_t Q, int64_t i0, int t,
+                                           uint32_t (&code)[kSortInFlight])
+{
+    float2 v[kSortInFlight];
+#pragma unroll
+    for (int j = 0; j < kSortInFlight; ++j) {
+        const int64_t i = i0 + (int64_t)j * kSortThreads + t;
+        v[j] = i < Q ? __ldg(p + i) : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < kSortInFlight; ++j)
+        code[j] = i0 + (int64_t)j * kSortThreads + t < Q ? cell_code(v[j]) : ~0u;
+}
+
+__global__ void __launch_bounds__(kSortThreads) sort_queries_kernel(const float2 *pts, int64_t Q,
+                                                                    int32_t *order)
+{
+    constexpr int kCells = kSortCells * kSortCells;
+    static_assert(kCells == 4 * kSortThreads, "the scan takes 4 counters per thread");
+    __shared__ __align__(16) int cnt[kCells];
+    __shared__ int warp_base[kSortThreads / 32];
+    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+    const int64_t base = (int64_t)blockIdx.x * Q;  // first query of this batch
+    const float2 *p = pts + base;
+    reinterpret_cast<int4 *>(cnt)[t] = make_int4(0, 0, 0, 0);
+    __syncthreads();
+    for (int64_t i0 = 0; i0 < Q; i0 += (int64_t)kSortThreads * kSortInFlight) {
+        uint32_t code[kSortInFlight];
+        cell_codes(p, Q, i0, t, code);
+#pragma unroll
+        for (int j = 0; j < kSortInFlight; ++j)
+            if (code[j] != ~0u)
+                atomicAdd(cnt + code[j], 1);
+    }
+    __syncthreads();
+    // exclusive scan of the counters: 4 per thread, warp shuffles, warp totals
+    const int4 c = reinterpret_cast<const int4 *>(cnt)[t];
+    const int own = c.x + c.y + c.z + c.w;
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += y;
+    }
+    if (lane == 31)
+        warp_base[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        const int tot = warp_base[lane];
+        int x = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o)
+                x += y;
+        }
+        warp_base[lane] = x - tot;
+    }
+    __syncthreads();
+    int4 r;
+    r.x = warp_base[wid] + incl - own;
+    r.y = r.x + c.x;
+    r.z = r.y + c.y;
+    r.w = r.z + c.z;
+    reinterpret_cast<int4 *>(cnt)[t] = r;
+    __syncthreads();
+    for (int64_t i0 = 0; i0 < Q; i0 += (int64_t)kSortThreads * kSortInFlight) {
+        uint32_t code[kSortInFlight];
+        cell_codes(p, Q, i0, t, code);
+#pragma unroll
+        for (int j = 0; j < kSortInFlight; ++j)
+            if (code[j] != ~0u) {
+                const int slot = atomicAdd(cnt + code[j], 1);
+                order[base + slot] = (int32_t)(base + i0 + (int64_t)j * kSortThreads + t);
+            }
     }
 }
 

@@ -106,3 +106,21 @@ def test_product_path_has_no_oracle_import():
                 text = open(os.path.join(root, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
                 assert "msda_oracle" not in text, f
+
+
+def test_query_order_checks(lib):
+    """query_order must be 4-byte aligned; B*Q must stay below 2^31; the sort's
+    pointers are checked before anything is enqueued."""
+    prob = _prob()
+    prob.query_order = ctypes.c_void_p(0x100002)
+    assert _fwd(lib, prob) == _lib.MSDA_ERR_INVALID_ARG
+    assert _fwd(lib, _prob(batch=1 << 16, num_queries=1 << 15)) == _lib.MSDA_ERR_UNSUPPORTED
+    p = _prob(batch=3, num_queries=10)
+    assert lib.msda_sort_queries(ctypes.byref(p), FAKE, ctypes.c_void_p(0x100001), None) == \
+        _lib.MSDA_ERR_INVALID_ARG
+    assert lib.msda_sort_queries(ctypes.byref(p), None, FAKE, None) == _lib.MSDA_ERR_INVALID_ARG
+    assert lib.msda_sort_queries(ctypes.byref(p), MISALIGNED, FAKE, None) == _lib.MSDA_ERR_INVALID_ARG
+    assert lib.msda_sort_queries(None, FAKE, FAKE, None) == _lib.MSDA_ERR_INVALID_ARG
+    # nothing to sort: succeeds without touching the device
+    empty = _prob(batch=0)
+    assert lib.msda_sort_queries(ctypes.byref(empty), None, None, None) == _lib.MSDA_OK
