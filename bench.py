@@ -410,10 +410,21 @@ def run_ours(args):
         }
         if want_nonfused:
             result["nonfused"] = _time_nonfused(msda, t, w, nbytes, flush, min(args.steps, 50))
+        if world == 1:
+            result["warm_l2"] = _time_warm(w, step, min(args.steps, 50))
+        stats = _input_stats(w, x)
+        if "value_bytes_touched" in stats:
+            # the value tensor counted by the sectors the gathers touch instead of whole
+            touched = step_bytes - 2 * (stats["value_bytes_whole"] - stats["value_bytes_touched"])
+            stats["hbm_frac_step_touched"] = round(
+                touched / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
+        result["config"]["input_stats"] = stats
         if not args.no_e2e:
             result["e2e"] = _time_e2e(msda, x, t, w, step, flush, min(args.steps, 50), dev)
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
+            result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(
+                w, x, result["cpu_baseline"], args.cpu_seconds)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -470,6 +481,67 @@ def _time_nonfused(msda, t, w, nbytes, flush, n):
             "fwd_hbm_frac": round(nbytes["forward"] / (fwd * 1e-3) / 1e9 / peak, 4),
             "bwd_hbm_frac": round(nbytes["backward"] / (bwd * 1e-3) / 1e9 / peak, 4),
             "fwd_gsamples_per_s": round(w.samples / (fwd * 1e-3) / 1e9, 4), "launches": n}
+
+
+def _time_warm(w, step, n):
+    """The same step back to back with no L2 flush between steps (warm L2)."""
+    import torch
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(n + 3)]
+    for ev in evs:
+        step(ev)
+    torch.cuda.synchronize()
+    ms = [e[0].elapsed_time(e[3]) for e in evs[3:]]
+    med = float(np.median(ms))
+    return {"ms_per_step_median": round(med, 5), "value": round(w.samples / (med * 1e-3) / 1e9, 4),
+            "unit": UNIT, "steps": n}
+
+
+def _input_stats(w: wl.Workload, x: wl.Inputs, max_queries: int = 4096) -> dict:
+    """Share of samples whose bilinear footprint lies wholly / partly outside
+    the level map, from the fused inputs (loc = ref + off / (W, H), pixel =
+    loc * size - 0.5), over every k-th query (at most `max_queries` per batch
+    image); and, for problems of up to 4 M samples, the distinct value bytes
+    the forward touches (whole 32-byte sectors)."""
+    stride = max(1, int(np.ceil(w.num_queries / max_queries)))
+    ref = x.reference_points[:, ::stride].astype(np.float64)        # [B, q, 2]
+    off = x.sampling_offsets[:, ::stride].astype(np.float64)        # [B, q, M, L, K, 2]
+    hw = x.spatial_shapes.astype(np.float64)                        # [L, 2] (H, W)
+    wh = hw[:, ::-1]                                                # (W, H)
+    loc = ref[:, :, None, None, None, :] + off / wh[None, None, None, :, None, :]
+    px = loc * wh[None, None, None, :, None, :] - 0.5
+    lo = np.floor(px)
+    size = wh[None, None, None, :, None, :]
+    inside = (px > -1) & (px < size)
+    full_out = ~(inside[..., 0] & inside[..., 1])
+    any_out = ((lo < 0) | (lo + 1 > size - 1)).any(axis=-1)
+    out = {"samples_counted": int(full_out.size),
+           "fully_outside": round(float(full_out.mean()), 4),
+           "any_corner_outside": round(float(any_out.mean()), 4)}
+    if w.samples <= (4 << 20):
+        loc = (x.reference_points.astype(np.float64)[:, :, None, None, None, :]
+               + x.sampling_offsets.astype(np.float64) / wh[None, None, None, :, None, :])
+        px = loc * wh[None, None, None, :, None, :] - 0.5
+        x0 = np.floor(px[..., 0]).astype(np.int64)
+        y0 = np.floor(px[..., 1]).astype(np.int64)
+        Wl = x.spatial_shapes[:, 1][None, None, None, :, None]
+        Hl = x.spatial_shapes[:, 0][None, None, None, :, None]
+        start = x.level_start_index[None, None, None, :, None]
+        b = np.arange(w.B)[:, None, None, None, None]
+        m = np.arange(w.M)[None, None, :, None, None]
+        elt = 4 if w.dtype == "f32" else 2
+        row_bytes = w.D * elt
+        rows = []
+        for dy in (0, 1):
+            for dx in (0, 1):
+                xi, yi = x0 + dx, y0 + dy
+                ok = (xi >= 0) & (xi < Wl) & (yi >= 0) & (yi < Hl)
+                key = (b * w.S + start + yi * Wl + xi) * w.M + m
+                rows.append(np.broadcast_to(key, ok.shape)[ok])
+        rows = np.unique(np.concatenate(rows))
+        sectors = np.unique((rows[:, None] * row_bytes + np.arange(0, row_bytes, 32)[None, :]) // 32)
+        out["value_bytes_touched"] = int(sectors.size * 32)
+        out["value_bytes_whole"] = int(w.B * w.S * w.M * row_bytes)
+    return out
 
 
 def _time_e2e(msda, x, t, w, step, flush, n, dev):
@@ -559,6 +631,59 @@ def cpu_baseline(w: wl.Workload, x: wl.Inputs, seconds: float) -> dict:
                       f"{smp['samples']} samples) x {passes} passes of fused fwd+bwd, "
                       f"{el:.1f} s", "host_cpus": os.cpu_count(),
             "full_step_ms_extrapolated": round(w.samples / rate * 1e3, 1)}
+
+
+def _cpu_worker(job):
+    """One process of the all-cores oracle leg: fused fwd+bwd over its slice
+    of the sampled queries, `passes` times; returns (seconds, samples)."""
+    folder, q0, q1, passes = job
+    import oracle
+    d = {k: np.load(os.path.join(folder, k + ".npy"), mmap_mode="r")
+         for k in ("value", "grad_output", "spatial_shapes", "level_start_index",
+                   "reference_points", "sampling_offsets", "attention_logits")}
+    smp = {k: (np.ascontiguousarray(v[:, q0:q1]) if k in ("grad_output", "reference_points",
+                                                         "sampling_offsets", "attention_logits")
+               else v) for k, v in d.items()}
+    B, _, M, _ = d["value"].shape
+    L, K = d["sampling_offsets"].shape[3], d["sampling_offsets"].shape[4]
+    t0 = time.perf_counter()
+    for _ in range(passes):
+        _oracle_step(oracle, smp)
+    return time.perf_counter() - t0, passes * B * (q1 - q0) * M * L * K
+
+
+def cpu_baseline_all_cores(w: wl.Workload, x: wl.Inputs, one_thread: dict, seconds: float) -> dict:
+    """The same oracle, unchanged, in one process per host core (spawned), each
+    on its own slice of the sampled queries; value = all samples / the slowest
+    process's time.  The per-process grad_value sums are not combined (a
+    reduction the timing leaves out)."""
+    import multiprocessing as mp
+    import tempfile
+    import oracle
+    oracle.build()
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    stride = max(1, int(round(w.num_queries / (2048 * max(1, cores // 4)))))
+    smp = _oracle_sample(w, x, stride)
+    nq = smp["queries"]
+    nproc = max(1, min(cores, nq))
+    rate1 = one_thread["value"] * 1e9
+    per_proc_samples = smp["samples"] / nproc
+    passes = max(1, int(np.ceil(seconds * rate1 / per_proc_samples)))
+    with tempfile.TemporaryDirectory() as folder:
+        for k in ("value", "grad_output", "spatial_shapes", "level_start_index",
+                  "reference_points", "sampling_offsets", "attention_logits"):
+            np.save(os.path.join(folder, k + ".npy"), smp[k])
+        bounds = np.linspace(0, nq, nproc + 1).astype(int)
+        jobs = [(folder, int(bounds[i]), int(bounds[i + 1]), passes) for i in range(nproc)]
+        with mp.get_context("spawn").Pool(nproc) as pool:
+            res = pool.map(_cpu_worker, jobs)
+    slowest = max(t for t, _ in res)
+    total = sum(n for _, n in res)
+    return {"value": round(total / slowest / 1e9, 6), "unit": UNIT, "cores": nproc,
+            "kind": "oracle",
+            "sample": f"every {stride}th query ({nq} of {w.num_queries}) split over {nproc} "
+                      f"spawned processes x {passes} passes of fused fwd+bwd, slowest "
+                      f"{slowest:.1f} s"}
 
 
 def run_reference(args):
