@@ -190,11 +190,10 @@ msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, int pa
         return st;
     a.rows_per_tile = (int64_t)warps * rpw;
     a.ntiles = (a.rows + a.rows_per_tile - 1) / a.rows_per_tile;
-    // one resident wave, but no more CTAs than there are band slices of work
+    // one resident wave, but no more CTAs than there are tiles
     int64_t ctas = (int64_t)sms * blocks_per_sm;
-    const int64_t slices = (a.ntiles + MSDA_BAND_TILES - 1) / MSDA_BAND_TILES;
-    if (ctas > slices)
-        ctas = slices;
+    if (ctas > a.ntiles)
+        ctas = a.ntiles;
     void *params[] = {&a};
     if (cudaLaunchKernel(kernel, dim3((unsigned)ctas), dim3(threads), params, smem, stream) != cudaSuccess)
         return MSDA_ERR_CUDA;

@@ -78,8 +78,8 @@ namespace msda {
 #ifndef MSDA_BWD_MIN_CTAS
 #define MSDA_BWD_MIN_CTAS 2
 #endif
-#ifndef MSDA_BAND_TILES              // row tiles a CTA walks before the grid moves on
-#define MSDA_BAND_TILES 1
+#ifndef MSDA_CONTIGUOUS_TILES        // 1: each CTA walks one contiguous run of tiles
+#define MSDA_CONTIGUOUS_TILES 0
 #endif
 #ifndef MSDA_HEAD_MAJOR              // 1: process rows head-major
 #define MSDA_HEAD_MAJOR 0
@@ -396,11 +396,8 @@ __device__ __forceinline__ float4 ld_grad4<__nv_bfloat16>(const __nv_bfloat16 *r
 
 // ------------------------------------------------------------- scheduling --
 //
-// Persistent grid, banded: the tiles are cut into bands of gridDim.x *
-// MSDA_BAND_TILES tiles; inside a band CTA c walks its own MSDA_BAND_TILES
-// consecutive tiles (1: a plain grid-stride walk, so that the whole GPU sweeps
-// neighbouring queries together and the L2 working set stays one band's
-// footprint).
+// Persistent grid: one resident wave of CTAs walks the row tiles (see
+// tile_walk for the two walks).
 //
 // Processing row p maps to memory row (b * Q + q) * M + m; head-major order
 // takes p = (m * B + b) * Q + q; with a query order the p-th query is order[p / M].
@@ -720,11 +717,22 @@ __device__ __forceinline__ WarpStage warp_stage(unsigned char *base, int warp, i
 }
 
 // Next tile of this CTA in the banded walk.
-__device__ __forceinline__ int64_t next_tile(int64_t tile)
+// Tiles of this CTA: a grid-stride walk (c, c + G, c + 2G, ...) or, with
+// MSDA_CONTIGUOUS_TILES, the contiguous run [c*T/G, (c+1)*T/G) of the T tiles
+// (consecutive queries then stay on one SM, where the corner rows they share
+// can hit in L1).  The host launches at most T CTAs.
+struct TileWalk {
+    int64_t first, end, step;
+};
+
+__device__ __forceinline__ TileWalk tile_walk(const KernelArgs &a)
 {
-    const int64_t band = (int64_t)gridDim.x * MSDA_BAND_TILES;
-    const int64_t i = (tile - (int64_t)blockIdx.x * MSDA_BAND_TILES) % band;
-    return (i + 1 < MSDA_BAND_TILES) ? tile + 1 : tile - i + band;
+    const int64_t c = blockIdx.x, G = gridDim.x;
+#if MSDA_CONTIGUOUS_TILES
+    return TileWalk{c * a.ntiles / G, (c + 1) * a.ntiles / G, 1};
+#else
+    return TileWalk{c, a.ntiles, G};
+#endif
 }
 
 __device__ __forceinline__ bool stage_ok(int64_t prow0, int nv, int P)
@@ -993,18 +1001,19 @@ forward_kernel(const KernelArgs a)
     }
     unsigned phase = 0;  // bit st: parity of the next completion of stage st
     int k = 0;
-    int64_t tile = (int64_t)blockIdx.x * MSDA_BAND_TILES;
-    if (cap && tile < a.ntiles) {
+    const TileWalk tw = tile_walk(a);
+    int64_t tile = tw.first;
+    if (cap && tile < tw.end) {
         const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
         const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
         if (stage_ok(p0, nv, P))
             stage_issue<FUSED>(a, ws, 0, p0, nv, lane, pol);
     }
-    for (; tile < a.ntiles; tile = next_tile(tile), ++k) {
+    for (; tile < tw.end; tile += tw.step, ++k) {
         const int st = k & 1;
-        const int64_t nxt = next_tile(tile);
+        const int64_t nxt = tile + tw.step;
         bool next_staged = false;
-        if (cap && nxt < a.ntiles) {
+        if (cap && nxt < tw.end) {
             const int64_t p0n = nxt * a.rows_per_tile + warp * RPW;
             const int nvn = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0n));
             next_staged = stage_ok(p0n, nvn, P);
@@ -1173,18 +1182,19 @@ backward_kernel(const KernelArgs a)
     }
     unsigned phase = 0;  // bit st: parity of the next completion of stage st
     int k = 0;
-    int64_t tile = (int64_t)blockIdx.x * MSDA_BAND_TILES;
-    if (cap && tile < a.ntiles) {
+    const TileWalk tw = tile_walk(a);
+    int64_t tile = tw.first;
+    if (cap && tile < tw.end) {
         const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
         const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
         if (stage_ok(p0, nv, P))
             stage_issue<FUSED>(a, ws, 0, p0, nv, lane, pol);
     }
-    for (; tile < a.ntiles; tile = next_tile(tile), ++k) {
+    for (; tile < tw.end; tile += tw.step, ++k) {
         const int st = k & 1;
-        const int64_t nxt = next_tile(tile);
+        const int64_t nxt = tile + tw.step;
         bool next_staged = false;
-        if (cap && nxt < a.ntiles) {
+        if (cap && nxt < tw.end) {
             const int64_t p0n = nxt * a.rows_per_tile + warp * RPW;
             const int nvn = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0n));
             next_staged = stage_ok(p0n, nvn, P);
