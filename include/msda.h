@@ -33,8 +33,8 @@
  *     move in 32-byte vectors).  The library keeps no pointer after the call
  *     returns and allocates no memory.
  *   - value, output and grad_output hold value_dtype elements (float32 or
- *     bfloat16); every other floating-point tensor is float32.  Accumulation
- *     is float32.
+ *     bfloat16; with MSDA_S8 value, output and grad_output are bfloat16);
+ *     every other floating-point tensor is float32.  Accumulation is float32.
  *   - Locations and offsets are (x, y) pairs; spatial_shapes rows are (H, W).
  *   - spatial_shapes [L,2] and level_start_index [L] are int64 device arrays.
  *     Their consistency (H, W >= 1, start[0] = 0, start[l+1] = start[l] +
@@ -82,7 +82,15 @@ typedef enum msda_status {
 
 typedef enum msda_dtype {
     MSDA_F32 = 0,
-    MSDA_BF16 = 1
+    MSDA_BF16 = 1,
+    /* INT8 value storage (the quantisation note of the x-humanoid.csdn.net
+     * MSDA explainer, §4: INT8 cuts the operator's memory traffic): value is
+     * int8 q with one float32 scale per (batch, head) in
+     * msda_problem.value_scale, and the operator samples q * scale; output
+     * and grad_output are bfloat16; grad_value is the gradient with respect
+     * to the dequantized value (float32, or bf16 with MSDA_GRAD_VALUE_BF16).
+     * msda_quantize_value_s8 produces q and the scales. */
+    MSDA_S8 = 2
 } msda_dtype;
 
 /* msda_problem.flags */
@@ -107,7 +115,8 @@ typedef struct msda_problem {
     int32_t head_dim;     /* D */
     int32_t num_levels;   /* L */
     int32_t num_points;   /* K */
-    int32_t value_dtype;  /* msda_dtype of value, output, grad_output */
+    int32_t value_dtype;  /* msda_dtype of value (and of output, grad_output
+                             unless MSDA_S8: then bfloat16) */
     uint32_t flags;       /* MSDA_* flags above */
     /* Optional device array [B*Q] int32, 4-byte aligned: the order in which
      * the kernels process the queries, a permutation of 0 .. B*Q-1 (query
@@ -120,6 +129,10 @@ typedef struct msda_problem {
      * detected (the rows of queries missing from the order are not written).
      * Read by the kernels on the stream: it must stay valid until they end. */
     const int32_t *query_order;
+    /* MSDA_S8 value only (ignored otherwise, required then): device array
+     * [B, M] float32, 4-byte aligned, the dequantization scale of each
+     * (batch, head).  Read by the kernels on the stream. */
+    const float *value_scale;
 } msda_problem;
 
 /*
@@ -243,6 +256,26 @@ MSDA_API msda_status msda_backward_noalloc(const msda_problem *problem, const vo
                                            const void *grad_output, void *grad_value,
                                            float *grad_sampling_locations,
                                            float *grad_attention_weights, msda_stream_t stream);
+
+/*
+ * INT8 value storage for MSDA_S8 (x-humanoid.csdn.net MSDA explainer §4,
+ * "quantization and low-precision inference"; the page gives no scheme, this
+ * is the plain symmetric one): for each (batch b, head m)
+ *   amax  = max over keys s and channels d of |value[b, s, m, d]|
+ *   scale = amax / 127 (float32 division), 1 when amax = 0
+ *   q     = value / scale (float32 division) rounded half to even, clipped to
+ *           [-127, 127]
+ *   value        [B, S, M, D]  problem->value_dtype (MSDA_F32 or MSDA_BF16),
+ *                              finite, 16-byte aligned
+ *   value_s8     [B, S, M, D]  int8, written, 32-byte aligned
+ *   value_scale  [B, M]        float32, written (also used as scratch)
+ * D must be a multiple of 8 (every supported D is).  Four operations on
+ * `stream`: a fill, an absmax reduction, the scales, the quantisation.
+ * Non-finite inputs give unspecified q and scales.
+ */
+MSDA_API msda_status msda_quantize_value_s8(const msda_problem *problem, const void *value,
+                                            void *value_s8, float *value_scale,
+                                            msda_stream_t stream);
 
 /*
  * Processing order that keeps spatially close queries together (the optional

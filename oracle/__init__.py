@@ -51,8 +51,10 @@ def _load():
             lib.msda_oracle_sampling_locations.argtypes = [D, P, P, P, P]
             lib.msda_oracle_softmax.argtypes = [D, P, P]
             lib.msda_oracle_fused_chain.argtypes = [D, P, P, P, P, P, P, P]
+            lib.msda_oracle_quantize_value_s8.argtypes = [D, P, P, P]
             for f in ("msda_oracle_forward", "msda_oracle_backward", "msda_oracle_sampling_locations",
-                      "msda_oracle_softmax", "msda_oracle_fused_chain"):
+                      "msda_oracle_softmax", "msda_oracle_fused_chain",
+                      "msda_oracle_quantize_value_s8"):
                 getattr(lib, f).restype = None
             _lib = lib
     return _lib
@@ -166,3 +168,24 @@ def pixel_coordinates(spatial_shapes, sampling_locations):
     W = sh[:, 1].astype(np.float64)[None, None, None, :, None]
     H = sh[:, 0].astype(np.float64)[None, None, None, :, None]
     return loc[..., 0] * W - 0.5, loc[..., 1] * H - 0.5
+
+
+def quantize_value_s8(value):
+    """INT8 value storage: (q int8 [B,S,M,D], scale float32 [B,M]) with one
+    symmetric absmax scale per (batch, head).  `value` is float32, or bfloat16
+    bit patterns (uint16), widened exactly to float32."""
+    v = np.asarray(value)
+    if v.dtype == np.uint16:
+        v = (v.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    B, S, M, D = v.shape
+    d = _Dims(B, S, 0, M, D, 0, 0)
+    q = np.empty(v.shape, np.int8)
+    scale = np.empty((B, M), np.float32)
+    _load().msda_oracle_quantize_value_s8(ctypes.byref(d), _p(v), _p(q), _p(scale))
+    return q, scale
+
+
+def dequantize_value_s8(q, scale):
+    """q * scale in float64 (exact), [B,S,M,D]: the value the operator samples."""
+    return np.asarray(q, np.float64) * np.asarray(scale, np.float64)[:, None, :, None]

@@ -285,3 +285,42 @@ void msda_oracle_fused_chain(const oracle_dims *d, const int64_t *shapes, const 
         }
     }
 }
+
+/*
+ * INT8 value storage ([csdn] §4, "quantization and low-precision inference":
+ * store the operator's data as INT8 to cut memory traffic; the page gives no
+ * scheme).  Reading taken (listed with the others): symmetric quantisation
+ * with one scale per (batch, head), in float32 as a quantising kernel would
+ * compute it:
+ *   amax  = max over s, d of |value[b, s, m, d]|
+ *   scale = amax / 127, or 1 when amax == 0
+ *   q     = value / scale rounded half to even, clipped to [-127, 127]
+ * The operator then samples the dequantized tensor q * scale (exact in
+ * double), so the core sums above are unchanged.  value: [B, S, M, D] float32
+ * (finite); q: [B, S, M, D]; scale: [B, M].
+ */
+void msda_oracle_quantize_value_s8(const oracle_dims *d, const float *value, int8_t *q, float *scale)
+{
+    for (int64_t b = 0; b < d->B; ++b)
+        for (int64_t m = 0; m < d->M; ++m) {
+            float amax = 0.0f;
+            for (int64_t s = 0; s < d->S; ++s)
+                for (int64_t c = 0; c < d->D; ++c) {
+                    const float a = fabsf(value[((b * d->S + s) * d->M + m) * d->D + c]);
+                    if (a > amax)
+                        amax = a;
+                }
+            const float sc = amax > 0.0f ? amax / 127.0f : 1.0f;
+            scale[b * d->M + m] = sc;
+            for (int64_t s = 0; s < d->S; ++s)
+                for (int64_t c = 0; c < d->D; ++c) {
+                    const int64_t i = ((b * d->S + s) * d->M + m) * d->D + c;
+                    float r = nearbyintf(value[i] / sc); /* default mode: half to even */
+                    if (r > 127.0f)
+                        r = 127.0f;
+                    if (r < -127.0f)
+                        r = -127.0f;
+                    q[i] = (int8_t)r;
+                }
+        }
+}

@@ -15,6 +15,7 @@ from .binding import (  # noqa: F401
     fused_backward,
     fused_forward,
     ms_deform_attn,
+    quantize_value_s8,
     sort_queries,
     version,
     zero_grads,

@@ -19,6 +19,7 @@ MSDA_ERR_DEVICE_TIMEOUT = 5
 
 MSDA_F32 = 0
 MSDA_BF16 = 1
+MSDA_S8 = 2
 
 MSDA_GRAD_VALUE_BF16 = 1 << 0
 MSDA_ACCUMULATE_GRADS = 1 << 1
@@ -37,6 +38,7 @@ class Problem(ctypes.Structure):
         ("value_dtype", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
         ("query_order", ctypes.c_void_p),
+        ("value_scale", ctypes.c_void_p),
     ]
 
 
@@ -51,6 +53,7 @@ _SIGNATURES = {
     "msda_zero_grads": [_PROB, _P, _P, _P],
     "msda_backward_noalloc": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "msda_sort_queries": [_PROB, _P, _P, _P],
+    "msda_quantize_value_s8": [_PROB, _P, _P, _P, _P],
     "msda_get_device_status": [_P, ctypes.POINTER(ctypes.c_int32)],
     "msda_status_string": [ctypes.c_int],
     "msda_version": [],

@@ -65,17 +65,28 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None, device=None):
     return t
 
 
-_DTYPES = {torch.float32: _lib.MSDA_F32, torch.bfloat16: _lib.MSDA_BF16}
+_DTYPES = {torch.float32: _lib.MSDA_F32, torch.bfloat16: _lib.MSDA_BF16, torch.int8: _lib.MSDA_S8}
+
+
+def _row_dtype(value: torch.Tensor):
+    """dtype of output / grad_output: value's, bfloat16 for INT8 value."""
+    return torch.bfloat16 if value.dtype == torch.int8 else value.dtype
 
 
 def _problem(value: torch.Tensor, Q: int, L: int, K: int, flags: int = 0,
-             query_order: Optional[torch.Tensor] = None) -> _lib.Problem:
+             query_order: Optional[torch.Tensor] = None,
+             value_scale: Optional[torch.Tensor] = None) -> _lib.Problem:
     if value.dim() != 4:
         raise ValueError("value must be [B, S, M, D]")
     if value.dtype not in _DTYPES:
-        raise TypeError("value must be float32 or bfloat16")
+        raise TypeError("value must be float32, bfloat16 or int8 (with value_scale)")
     B, S, M, D = value.shape
     prob = _lib.Problem(B, S, Q, M, D, L, K, _DTYPES[value.dtype], flags)
+    if value.dtype == torch.int8:
+        if value_scale is None:
+            raise ValueError("int8 value needs value_scale [B, M] (see quantize_value_s8)")
+        _need(value_scale, "value_scale", torch.float32, (B, M), value.device)
+        prob.value_scale = _ptr(value_scale)
     if query_order is not None:
         if query_order.numel() != B * Q:
             raise ValueError(f"query_order must hold B*Q = {B * Q} entries")
@@ -96,9 +107,11 @@ def _geometry(value, spatial_shapes, level_start_index):
 def forward(value: torch.Tensor, spatial_shapes: torch.Tensor, level_start_index: torch.Tensor,
             sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
             out: Optional[torch.Tensor] = None,
-            query_order: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """msda_forward: returns out [B, Q, M, D] in value's dtype.  query_order:
-    optional int32 [B*Q] processing order (see sort_queries)."""
+            query_order: Optional[torch.Tensor] = None,
+            value_scale: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """msda_forward: returns out [B, Q, M, D] in value's dtype (bfloat16 for
+    int8 value, which needs value_scale [B, M]).  query_order: optional int32
+    [B*Q] processing order (see sort_queries)."""
     _need(value, "value", None)
     L = _geometry(value, spatial_shapes, level_start_index)
     B, S, M, D = value.shape
@@ -108,9 +121,9 @@ def forward(value: torch.Tensor, spatial_shapes: torch.Tensor, level_start_index
     _need(sampling_locations, "sampling_locations", torch.float32, (B, Q, M, L, K, 2), value.device)
     _need(attention_weights, "attention_weights", torch.float32, (B, Q, M, L, K), value.device)
     if out is None:
-        out = torch.empty((B, Q, M, D), dtype=value.dtype, device=value.device)
-    _need(out, "out", value.dtype, (B, Q, M, D), value.device)
-    prob = _problem(value, Q, L, K, 0, query_order)
+        out = torch.empty((B, Q, M, D), dtype=_row_dtype(value), device=value.device)
+    _need(out, "out", _row_dtype(value), (B, Q, M, D), value.device)
+    prob = _problem(value, Q, L, K, 0, query_order, value_scale)
     st = _lib.load().msda_forward(ctypes.byref(prob), _ptr(value), _ptr(spatial_shapes),
                                   _ptr(level_start_index), _ptr(sampling_locations),
                                   _ptr(attention_weights), _ptr(out), _stream())
@@ -125,7 +138,8 @@ def backward(value, spatial_shapes, level_start_index, sampling_locations, atten
              grad_attention_weights: Optional[torch.Tensor] = None,
              workspace: Optional[torch.Tensor] = None,
              accumulate: bool = False,
-             query_order: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+             query_order: Optional[torch.Tensor] = None,
+             value_scale: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """msda_backward: (grad_value, grad_sampling_locations, grad_attention_weights).
 
     accumulate=True adds into the given float32 grad_value instead of
@@ -137,7 +151,7 @@ def backward(value, spatial_shapes, level_start_index, sampling_locations, atten
     dev = value.device
     _need(sampling_locations, "sampling_locations", torch.float32, (B, Q, M, L, K, 2), dev)
     _need(attention_weights, "attention_weights", torch.float32, (B, Q, M, L, K), dev)
-    _need(grad_output, "grad_output", value.dtype, (B, Q, M, D), dev)
+    _need(grad_output, "grad_output", _row_dtype(value), (B, Q, M, D), dev)
     flags = _lib.MSDA_GRAD_VALUE_BF16 if grad_value_dtype == torch.bfloat16 else 0
     if grad_value_dtype not in (torch.float32, torch.bfloat16):
         raise TypeError("grad_value_dtype must be float32 or bfloat16")
@@ -152,7 +166,7 @@ def backward(value, spatial_shapes, level_start_index, sampling_locations, atten
     if grad_attention_weights is None:
         grad_attention_weights = torch.empty((B, Q, M, L, K), dtype=torch.float32, device=dev)
     _need(grad_value, "grad_value", grad_value_dtype, (B, S, M, D), dev)
-    prob = _problem(value, Q, L, K, flags, query_order)
+    prob = _problem(value, Q, L, K, flags, query_order, value_scale)
     lib = _lib.load()
     ws_bytes = ctypes.c_size_t(0)
     _check(lib.msda_backward_workspace_size(ctypes.byref(prob), ctypes.byref(ws_bytes)),
@@ -178,7 +192,8 @@ def _logits(attention_logits, B, Q, M, L, K, dev):
 def fused_forward(value, spatial_shapes, level_start_index, reference_points, sampling_offsets,
                   attention_logits, return_attention_weights: bool = False,
                   out: Optional[torch.Tensor] = None,
-                  query_order: Optional[torch.Tensor] = None):
+                  query_order: Optional[torch.Tensor] = None,
+                  value_scale: Optional[torch.Tensor] = None):
     """msda_fused_forward: out [B, Q, M, D] (and the softmax weights if asked)."""
     _need(value, "value", None)
     L = _geometry(value, spatial_shapes, level_start_index)
@@ -191,10 +206,10 @@ def fused_forward(value, spatial_shapes, level_start_index, reference_points, sa
     _need(sampling_offsets, "sampling_offsets", torch.float32, (B, Q, M, L, K, 2), dev)
     attention_logits = _logits(attention_logits, B, Q, M, L, K, dev)
     if out is None:
-        out = torch.empty((B, Q, M, D), dtype=value.dtype, device=dev)
-    _need(out, "out", value.dtype, (B, Q, M, D), dev)
+        out = torch.empty((B, Q, M, D), dtype=_row_dtype(value), device=dev)
+    _need(out, "out", _row_dtype(value), (B, Q, M, D), dev)
     attn = torch.empty((B, Q, M, L, K), dtype=torch.float32, device=dev) if return_attention_weights else None
-    prob = _problem(value, Q, L, K, 0, query_order)
+    prob = _problem(value, Q, L, K, 0, query_order, value_scale)
     st = _lib.load().msda_fused_forward(ctypes.byref(prob), _ptr(value), _ptr(spatial_shapes),
                                         _ptr(level_start_index), _ptr(reference_points),
                                         _ptr(sampling_offsets), _ptr(attention_logits), _ptr(out),
@@ -212,7 +227,8 @@ def fused_backward(value, spatial_shapes, level_start_index, reference_points, s
                    grad_reference_points: Optional[torch.Tensor] = None,
                    grad_sampling_offsets: Optional[torch.Tensor] = None,
                    grad_attention_logits: Optional[torch.Tensor] = None,
-                   query_order: Optional[torch.Tensor] = None):
+                   query_order: Optional[torch.Tensor] = None,
+                   value_scale: Optional[torch.Tensor] = None):
     """msda_fused_backward: (grad_value, grad_reference_points or None,
     grad_sampling_offsets, grad_attention_logits [B, Q, M, L*K]).
 
@@ -226,7 +242,7 @@ def fused_backward(value, spatial_shapes, level_start_index, reference_points, s
     _need(reference_points, "reference_points", torch.float32, (B, Q, 2), dev)
     _need(sampling_offsets, "sampling_offsets", torch.float32, (B, Q, M, L, K, 2), dev)
     attention_logits = _logits(attention_logits, B, Q, M, L, K, dev)
-    _need(grad_output, "grad_output", value.dtype, (B, Q, M, D), dev)
+    _need(grad_output, "grad_output", _row_dtype(value), (B, Q, M, D), dev)
     if grad_value_dtype not in (torch.float32, torch.bfloat16):
         raise TypeError("grad_value_dtype must be float32 or bfloat16")
     flags = _lib.MSDA_GRAD_VALUE_BF16 if grad_value_dtype == torch.bfloat16 else 0
@@ -248,7 +264,7 @@ def fused_backward(value, spatial_shapes, level_start_index, reference_points, s
     glog = grad_attention_logits if grad_attention_logits is not None else \
         torch.empty((B, Q, M, L * K), dtype=torch.float32, device=dev)
     _need(glog, "grad_attention_logits", torch.float32, (B, Q, M, L * K), dev)
-    prob = _problem(value, Q, L, K, flags, query_order)
+    prob = _problem(value, Q, L, K, flags, query_order, value_scale)
     lib = _lib.load()
     ws_bytes = ctypes.c_size_t(0)
     _check(lib.msda_backward_workspace_size(ctypes.byref(prob), ctypes.byref(ws_bytes)),
@@ -296,6 +312,28 @@ def backward_noalloc(value, spatial_shapes, level_start_index, sampling_location
                                            _ptr(grad_attention_weights), _stream())
     _check(st, "msda_backward_noalloc")
     return grad_value, grad_sampling_locations, grad_attention_weights
+
+
+def quantize_value_s8(value: torch.Tensor, value_s8: Optional[torch.Tensor] = None,
+                      value_scale: Optional[torch.Tensor] = None):
+    """msda_quantize_value_s8: (int8 value [B, S, M, D], float32 scale [B, M])
+    from a float32 or bfloat16 value, one symmetric absmax scale per
+    (batch, head); pass both to the other calls (value_scale=...)."""
+    _need(value, "value", None)
+    if value.dim() != 4 or value.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("value must be a float32 or bfloat16 [B, S, M, D] tensor")
+    B, S, M, D = value.shape
+    if value_s8 is None:
+        value_s8 = torch.empty((B, S, M, D), dtype=torch.int8, device=value.device)
+    if value_scale is None:
+        value_scale = torch.empty((B, M), dtype=torch.float32, device=value.device)
+    _need(value_s8, "value_s8", torch.int8, (B, S, M, D), value.device)
+    _need(value_scale, "value_scale", torch.float32, (B, M), value.device)
+    prob = _lib.Problem(B, S, 1, M, D, 1, 1, _DTYPES[value.dtype], 0)
+    st = _lib.load().msda_quantize_value_s8(ctypes.byref(prob), _ptr(value), _ptr(value_s8),
+                                            _ptr(value_scale), _stream())
+    _check(st, "msda_quantize_value_s8")
+    return value_s8, value_scale
 
 
 def sort_queries(points: torch.Tensor, query_order: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -28,7 +28,7 @@ bool is_supported_head_dim(int d)
     return d == 8 || d == 16 || d == 32 || d == 64 || d == 128 || d == 256;
 }
 
-size_t elem_bytes(int32_t dtype) { return dtype == MSDA_BF16 ? 2 : 4; }
+size_t elem_bytes(int32_t dtype) { return dtype == MSDA_BF16 ? 2 : (dtype == MSDA_S8 ? 1 : 4); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
@@ -51,7 +51,10 @@ msda_status check_problem(const msda_problem *p)
     if (p->batch < 0 || p->num_queries < 0 || p->num_keys < 1 || p->num_heads < 1 ||
         p->num_levels < 1 || p->num_points < 1 || p->head_dim < 1)
         return MSDA_ERR_INVALID_ARG;
-    if (p->value_dtype != MSDA_F32 && p->value_dtype != MSDA_BF16)
+    if (p->value_dtype != MSDA_F32 && p->value_dtype != MSDA_BF16 && p->value_dtype != MSDA_S8)
+        return MSDA_ERR_INVALID_ARG;
+    if (p->value_dtype == MSDA_S8 &&
+        (!p->value_scale || (reinterpret_cast<uintptr_t>(p->value_scale) & 3u)))
         return MSDA_ERR_INVALID_ARG;
     if (p->flags & ~(uint32_t)(MSDA_GRAD_VALUE_BF16 | MSDA_ACCUMULATE_GRADS | MSDA_TEST_WITHHOLD_COPY))
         return MSDA_ERR_INVALID_ARG;
@@ -250,11 +253,16 @@ msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
             MSDA_FWD_CASE(float, 8) MSDA_FWD_CASE(float, 16) MSDA_FWD_CASE(float, 32)
             MSDA_FWD_CASE(float, 64) MSDA_FWD_CASE(float, 128) MSDA_FWD_CASE(float, 256)
         }
-    } else {
+    } else if (p->value_dtype == MSDA_BF16) {
         switch (p->head_dim) {
             MSDA_FWD_CASE(__nv_bfloat16, 8) MSDA_FWD_CASE(__nv_bfloat16, 16)
             MSDA_FWD_CASE(__nv_bfloat16, 32) MSDA_FWD_CASE(__nv_bfloat16, 64)
             MSDA_FWD_CASE(__nv_bfloat16, 128) MSDA_FWD_CASE(__nv_bfloat16, 256)
+        }
+    } else {
+        switch (p->head_dim) {
+            MSDA_FWD_CASE(msda::S8, 8) MSDA_FWD_CASE(msda::S8, 16) MSDA_FWD_CASE(msda::S8, 32)
+            MSDA_FWD_CASE(msda::S8, 64) MSDA_FWD_CASE(msda::S8, 128) MSDA_FWD_CASE(msda::S8, 256)
         }
     }
 #undef MSDA_FWD_CASE
@@ -276,11 +284,16 @@ msda_status launch_backward(const msda_problem *p, KernelArgs &a, cudaStream_t s
             MSDA_BWD_CASE(float, 8) MSDA_BWD_CASE(float, 16) MSDA_BWD_CASE(float, 32)
             MSDA_BWD_CASE(float, 64) MSDA_BWD_CASE(float, 128) MSDA_BWD_CASE(float, 256)
         }
-    } else {
+    } else if (p->value_dtype == MSDA_BF16) {
         switch (p->head_dim) {
             MSDA_BWD_CASE(__nv_bfloat16, 8) MSDA_BWD_CASE(__nv_bfloat16, 16)
             MSDA_BWD_CASE(__nv_bfloat16, 32) MSDA_BWD_CASE(__nv_bfloat16, 64)
             MSDA_BWD_CASE(__nv_bfloat16, 128) MSDA_BWD_CASE(__nv_bfloat16, 256)
+        }
+    } else {
+        switch (p->head_dim) {
+            MSDA_BWD_CASE(msda::S8, 8) MSDA_BWD_CASE(msda::S8, 16) MSDA_BWD_CASE(msda::S8, 32)
+            MSDA_BWD_CASE(msda::S8, 64) MSDA_BWD_CASE(msda::S8, 128) MSDA_BWD_CASE(msda::S8, 256)
         }
     }
 #undef MSDA_BWD_CASE
@@ -302,6 +315,7 @@ KernelArgs base_args(const msda_problem *p, const void *value, const int64_t *sh
     a.K = p->num_points;
     a.withhold_copy = (p->flags & MSDA_TEST_WITHHOLD_COPY) ? 1 : 0;
     a.order = (p->batch * p->num_queries > 0) ? p->query_order : nullptr;
+    a.scale = p->value_dtype == MSDA_S8 ? p->value_scale : nullptr;
     return a;
 }
 
@@ -555,6 +569,59 @@ msda_status msda_backward_noalloc(const msda_problem *problem, const void *value
             return st;
     }
     return launch_to_bf16(acc, grad_value, z.value, s);
+}
+
+msda_status msda_quantize_value_s8(const msda_problem *problem, const void *value, void *value_s8,
+                                   float *value_scale, msda_stream_t stream)
+{
+    msda_status st = check_problem(problem);
+    if (st != MSDA_OK)
+        return st;
+    if (problem->value_dtype != MSDA_F32 && problem->value_dtype != MSDA_BF16)
+        return MSDA_ERR_INVALID_ARG;
+    const int64_t B = problem->batch, S = problem->num_keys;
+    const int M = problem->num_heads, D = problem->head_dim;
+    const int64_t n = B * S * M * (int64_t)D;
+    if (B == 0)
+        return MSDA_OK;
+    if (!ptr_ok(value, n) || !vec_ptr_ok(value_s8, n) || !value_scale ||
+        (reinterpret_cast<uintptr_t>(value_scale) & 3u) || D % 8 != 0)
+        return MSDA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    st = current_device(dev, sms);
+    if (st != MSDA_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t bm = B * M;
+    if (cudaMemsetAsync(value_scale, 0, (size_t)bm * sizeof(float), s) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    // about four CTAs per SM in the reduction, each over >= 1 key of one (b, m)
+    int64_t chunks = ((int64_t)sms * 4 + bm - 1) / bm;
+    if (chunks > S)
+        chunks = S;
+    if (chunks * bm > 0x7fffffffLL)
+        chunks = 0x7fffffffLL / bm;
+    if (chunks < 1)
+        return MSDA_ERR_UNSUPPORTED;
+    unsigned *amax = reinterpret_cast<unsigned *>(value_scale);
+    int64_t qblocks = (n / 8 + 255) / 256;
+    if (qblocks > (int64_t)sms * 8)
+        qblocks = (int64_t)sms * 8;
+    if (problem->value_dtype == MSDA_F32) {
+        const float *v = static_cast<const float *>(value);
+        msda::absmax_kernel<float><<<(unsigned)(chunks * bm), 256, 0, s>>>(v, S, M, D, (int)chunks, amax);
+        msda::s8_scale_kernel<<<(unsigned)((bm + 255) / 256), 256, 0, s>>>(value_scale, bm);
+        msda::quantize_s8_kernel<float><<<(unsigned)qblocks, 256, 0, s>>>(
+            v, value_scale, n / 8, S, M, D, static_cast<uint2 *>(value_s8));
+    } else {
+        const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(value);
+        msda::absmax_kernel<__nv_bfloat16><<<(unsigned)(chunks * bm), 256, 0, s>>>(v, S, M, D, (int)chunks,
+                                                                                  amax);
+        msda::s8_scale_kernel<<<(unsigned)((bm + 255) / 256), 256, 0, s>>>(value_scale, bm);
+        msda::quantize_s8_kernel<__nv_bfloat16><<<(unsigned)qblocks, 256, 0, s>>>(
+            v, value_scale, n / 8, S, M, D, static_cast<uint2 *>(value_s8));
+    }
+    return cudaGetLastError() == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
 }
 
 msda_status msda_sort_queries(const msda_problem *problem, const float *points, int32_t *query_order,

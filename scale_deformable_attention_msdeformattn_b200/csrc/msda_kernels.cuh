@@ -37,6 +37,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace msda {
 
 // Tuning knobs (compile-time).  The forward gathers float32 rows with 32-byte
@@ -71,6 +73,15 @@ namespace msda {
 #endif
 #ifndef MSDA_BWD_STAGE
 #define MSDA_BWD_STAGE 0
+#endif
+#ifndef MSDA_FWD_VB_S8               // INT8 value: bytes per lane vector
+#define MSDA_FWD_VB_S8 8
+#endif
+#ifndef MSDA_FWD_INFLIGHT_S8
+#define MSDA_FWD_INFLIGHT_S8 4
+#endif
+#ifndef MSDA_FWD_MIN_CTAS_S8
+#define MSDA_FWD_MIN_CTAS_S8 2
 #endif
 #ifndef MSDA_BWD_VB
 #define MSDA_BWD_VB 16
@@ -119,6 +130,7 @@ struct KernelArgs {
     int Q, M, L, K;
     int withhold_copy;      // testing: arm the input copies but never issue them
     const int32_t *order;   // optional processing order of the B*Q queries
+    const float *scale;     // INT8 value: dequantization scale per (batch, head)
 };
 
 struct Geometry {
@@ -164,10 +176,12 @@ struct alignas(32) U8 {
 };
 
 template <int VB> struct RawOf;
+template <> struct RawOf<8> { using type = uint2; };
 template <> struct RawOf<16> { using type = uint4; };
 template <> struct RawOf<32> { using type = U8; };
 
 // Read-only vector load of `value` (L1-cached).
+__device__ __forceinline__ uint2 ld_vec(const uint2 *p) { return __ldg(p); }
 __device__ __forceinline__ uint4 ld_vec(const uint4 *p) { return __ldg(p); }
 __device__ __forceinline__ U8 ld_vec(const U8 *p)
 {
@@ -225,6 +239,33 @@ template <> struct Elem<__nv_bfloat16> {
     }
 };
 
+// INT8 value storage: a signed byte per channel, dequantized by the
+// (batch, head) scale of KernelArgs::scale.  Never written by the kernels.
+struct S8 {
+    int8_t bits;
+};
+template <> struct Elem<S8> {
+    static constexpr int kBytes = 1;
+    // Exact: byte b (offset to b + 128 by the xor) is placed in the low
+    // mantissa bits of the float 2^23, which is then subtracted with the
+    // offset.
+    template <int NW> __device__ __forceinline__ static void widen(const uint32_t *u, float *f)
+    {
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+            const uint32_t x = u[i] ^ 0x80808080u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                f[4 * i + k] = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7540u + k)) - 8388736.0f;
+        }
+    }
+};
+
+// Element type of output and grad_output rows: the value type, except bf16
+// rows for INT8 value.
+template <typename T> struct RowOf { using type = T; };
+template <> struct RowOf<S8> { using type = __nv_bfloat16; };
+
 // Lane layout of one row of D channels with VB-byte lane vectors.
 template <typename T, int D, int VB> struct Layout {
     static constexpr int kVB = (D * Elem<T>::kBytes < VB) ? D * Elem<T>::kBytes : VB;
@@ -236,7 +277,7 @@ template <typename T, int D, int VB> struct Layout {
     static constexpr int kCh = kNvec / kG;                   // vectors per lane
     static constexpr int kRowsPerWarp = 32 / kG;
     static constexpr int kLaneElems = kCh * kEpv;            // channels per lane
-    static_assert(kVB == 16 || kVB == 32, "vector size");
+    static_assert(kVB == 8 || kVB == 16 || kVB == 32, "vector size");
     static_assert(kNvec >= 1 && kNvec % kG == 0, "unsupported head_dim");
     __device__ __forceinline__ static void widen(const Raw &r, float *f)
     {
@@ -249,6 +290,10 @@ template <typename T, int D, int VB> struct Layout {
         return r;
     }
 };
+
+// Lane vector width of the backward for each value type.
+template <typename T> struct BwdVB { static constexpr int kVB = MSDA_BWD_VB; };
+template <> struct BwdVB<S8> { static constexpr int kVB = 8; };
 
 template <int G>
 __device__ __forceinline__ float group_sum(float v)
@@ -963,6 +1008,11 @@ template <> struct FwdTune<__nv_bfloat16> {
                          kMinCtas = MSDA_FWD_MIN_CTAS_BF16;
     static constexpr bool kStage = MSDA_FWD_STAGE_BF16 != 0;
 };
+template <> struct FwdTune<S8> {
+    static constexpr int kVB = MSDA_FWD_VB_S8, kInFlight = MSDA_FWD_INFLIGHT_S8,
+                         kMinCtas = MSDA_FWD_MIN_CTAS_S8;
+    static constexpr bool kStage = false;
+};
 
 template <typename T, int D, bool FUSED>
 __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, FwdTune<T>::kMinCtas)
@@ -1091,10 +1141,26 @@ forward_kernel(const KernelArgs a)
                         }
                 }
             }
-            Raw *obase = reinterpret_cast<Raw *>(static_cast<T *>(a.out) + row * D) + gl;
+            if constexpr (std::is_same<T, S8>::value) {
+                // dequantize once per row, store bf16 (EPV = 8 channels, 16 bytes)
+                static_assert(EPV == 8, "INT8 lanes hold 8 channels");
+                const float sc = __ldg(a.scale + b * a.M + m);
 #pragma unroll
-            for (int j = 0; j < CH; ++j)
-                st_vec(obase + j * G, Lay::narrow(acc + j * EPV));
+                for (int e = 0; e < E; ++e)
+                    acc[e] *= sc;
+                uint4 *obase = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + row * D) + gl;
+#pragma unroll
+                for (int j = 0; j < CH; ++j) {
+                    uint4 r;
+                    Elem<__nv_bfloat16>::narrow<4>(acc + j * EPV, reinterpret_cast<uint32_t *>(&r));
+                    obase[j * G] = r;
+                }
+            } else {
+                Raw *obase = reinterpret_cast<Raw *>(static_cast<T *>(a.out) + row * D) + gl;
+#pragma unroll
+                for (int j = 0; j < CH; ++j)
+                    st_vec(obase + j * G, Lay::narrow(acc + j * EPV));
+            }
         }
         __syncwarp();
     }
@@ -1136,7 +1202,8 @@ template <typename T, int D, bool FUSED>
 __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, MSDA_BWD_MIN_CTAS)
 backward_kernel(const KernelArgs a)
 {
-    using Lay = Layout<T, D, MSDA_BWD_VB>;
+    using Lay = Layout<T, D, BwdVB<T>::kVB>;
+    using R = typename RowOf<T>::type;  // grad_output element
     using Raw = typename Lay::Raw;
     constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Lay::kEpv;
     constexpr int C = BwdChunk<G>::kC;
@@ -1239,18 +1306,18 @@ backward_kernel(const KernelArgs a)
         float2 g2[E / 2];
         float4 gr[NR];
         if (active) {
-            const T *grow = static_cast<const T *>(a.grad_out) + row * D;
+            const R *grow = static_cast<const R *>(a.grad_out) + row * D;
 #pragma unroll
             for (int j = 0; j < CH; ++j)
 #pragma unroll
                 for (int q4 = 0; q4 < EPV / 4; ++q4) {
-                    const float4 t4 = ld_grad4<T>(grow, (j * G + gl) * EPV + 4 * q4, pol);
+                    const float4 t4 = ld_grad4<R>(grow, (j * G + gl) * EPV + 4 * q4, pol);
                     g2[(j * EPV + 4 * q4) / 2] = make_float2(t4.x, t4.y);
                     g2[(j * EPV + 4 * q4) / 2 + 1] = make_float2(t4.z, t4.w);
                 }
 #pragma unroll
             for (int h = 0; h < NR; ++h)
-                gr[h] = ld_grad4<T>(grow, (h * G + gl) * 4, pol);
+                gr[h] = ld_grad4<R>(grow, (h * G + gl) * 4, pol);
         } else {
 #pragma unroll
             for (int e = 0; e < E / 2; ++e)
@@ -1261,6 +1328,9 @@ backward_kernel(const KernelArgs a)
         }
         const int64_t base = row * P;
         float dot = 0.f, ref_gx = 0.f, ref_gy = 0.f;  // fused: per-owner partial sums
+        float vsc = 1.f;  // INT8 value: the dot products are in quantized units
+        if constexpr (std::is_same<T, S8>::value)
+            vsc = active ? __ldg(a.scale + b * a.M + m) : 0.f;
         for (int c0 = 0; c0 < Pp; c0 += C) {
             float part[C][3];
 #pragma unroll
@@ -1288,7 +1358,8 @@ backward_kernel(const KernelArgs a)
                 const unsigned inm = __float_as_uint(r.w);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    d[c] = (inm & (1u << c)) ? d[c] : 0.f;  // corners outside the map read 0
+                    d[c] = (inm & (1u << c)) ? (std::is_same<T, S8>::value ? d[c] * vsc : d[c])
+                                             : 0.f;  // corners outside the map read 0
                 const float fx = r.x, fy = r.y, A = r.z, ex = 1.f - fx, ey = 1.f - fy;
                 const float w[4] = {ex * ey, fx * ey, ex * fy, fx * fy};
                 part[i][0] = w[0] * d[0] + w[1] * d[1] + w[2] * d[2] + w[3] * d[3];
@@ -1373,6 +1444,96 @@ __global__ void f32_to_bf16_kernel(const float4 *src, uint4 *dst, int64_t n8)
         uint4 r;
         Elem<__nv_bfloat16>::narrow<4>(f, reinterpret_cast<uint32_t *>(&r));
         dst[i] = r;
+    }
+}
+
+// ------------------------------------------------------ INT8 quantisation --
+//
+// value [B, S, M, D] (float32 or bf16) -> int8 with one symmetric scale per
+// (batch, head): amax = max |value[b, :, m, :]|, scale = amax / 127 (1 when
+// amax = 0), q = value / scale rounded half to even, clipped to +-127.  Three
+// kernels: per-(b, m) absmax (into the scale array as float bits, zeroed by
+// the host), scale = amax / 127 in place, quantise.
+
+// Eight consecutive channels starting at p, widened to float32.
+__device__ __forceinline__ void load8(const float *p, float (&f)[8])
+{
+    const float4 x = __ldg(reinterpret_cast<const float4 *>(p));
+    const float4 y = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+    f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+    f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&f)[8])
+{
+    const uint4 r = __ldg(reinterpret_cast<const uint4 *>(p));
+    Elem<__nv_bfloat16>::widen<4>(reinterpret_cast<const uint32_t *>(&r), f);
+}
+
+// CTA blockIdx.x covers (b, m) = blockIdx.x / chunks and the chunk
+// blockIdx.x % chunks of the S keys; one atomicMax per CTA.  |x| >= 0, so the
+// float bit patterns order like the values.
+template <typename T>
+__global__ void __launch_bounds__(256) absmax_kernel(const T *v, int64_t S, int M, int D, int chunks,
+                                                     unsigned *amax)
+{
+    __shared__ float part[8];
+    const int64_t bm = blockIdx.x / chunks;
+    const int64_t chunk = blockIdx.x % chunks;
+    const int64_t b = bm / M, m = bm % M;
+    const int nv = D / 8;
+    const int64_t s0 = S * chunk / chunks, s1 = S * (chunk + 1) / chunks;
+    float mx = 0.f;
+    for (int64_t i = threadIdx.x; i < (s1 - s0) * nv; i += blockDim.x) {
+        const int64_t s = s0 + i / nv;
+        const int j = (int)(i % nv);
+        float f[8];
+        load8(v + ((b * S + s) * M + m) * D + j * 8, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            mx = fmaxf(mx, fabsf(f[e]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0)
+        part[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+            mx = fmaxf(mx, part[w]);
+        atomicMax(amax + bm, __float_as_uint(mx));
+    }
+}
+
+__global__ void s8_scale_kernel(float *scale, int64_t n)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) {
+        const float amax = scale[i];
+        scale[i] = amax > 0.f ? __fdiv_rn(amax, 127.f) : 1.f;
+    }
+}
+
+// Eight channels per thread step (D is a multiple of 8).
+template <typename T>
+__global__ void quantize_s8_kernel(const T *v, const float *scale, int64_t n8, int64_t S, int M, int D,
+                                   uint2 *q)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
+        const int64_t row = i * 8 / D;  // (b * S + s) * M + m
+        const int64_t m = row % M, b = row / ((int64_t)S * M);
+        const float sc = __ldg(scale + b * M + m);
+        float f[8];
+        load8(v + i * 8, f);
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            int r = __float2int_rn(__fdiv_rn(f[e], sc));  // half to even
+            r = r > 127 ? 127 : (r < -127 ? -127 : r);
+            w[e >> 2] |= ((uint32_t)r & 0xffu) << (8 * (e & 3));
+        }
+        q[i] = make_uint2(w[0], w[1]);
     }
 }
 
@@ -1489,11 +1650,11 @@ __global__ void __launch_bounds__(kSortThreads) sort_queries_kernel(const float2
 template <typename T, int D> constexpr int forward_rows_per_warp() { return Layout<T, D, FwdTune<T>::kVB>::kRowsPerWarp; }
 template <typename T> constexpr bool forward_stages() { return FwdTune<T>::kStage; }
 constexpr bool backward_stages() { return MSDA_BWD_STAGE != 0; }
-template <typename T, int D> constexpr int backward_rows_per_warp() { return Layout<T, D, MSDA_BWD_VB>::kRowsPerWarp; }
+template <typename T, int D> constexpr int backward_rows_per_warp() { return Layout<T, D, BwdVB<T>::kVB>::kRowsPerWarp; }
 // Record slots of a backward row: L*K rounded up to the reduce-scatter chunk.
 template <typename T, int D> inline int backward_padded_samples(int P)
 {
-    constexpr int C = BwdChunk<Layout<T, D, MSDA_BWD_VB>::kG>::kC;
+    constexpr int C = BwdChunk<Layout<T, D, BwdVB<T>::kVB>::kG>::kC;
     return (P + C - 1) / C * C;
 }
 

@@ -13,7 +13,7 @@ TOL = {"f32": 1e-5, "bf16": 2e-2}
 
 
 def value_tensor(arr: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
-    if dtype == "bf16":
+    if dtype in ("bf16", "s8"):  # s8 workloads carry the bf16 source
         return torch.from_numpy(arr.view(np.int16)).to(device).view(torch.bfloat16)
     return torch.from_numpy(arr).to(device)
 

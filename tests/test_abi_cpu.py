@@ -124,3 +124,21 @@ def test_query_order_checks(lib):
     # nothing to sort: succeeds without touching the device
     empty = _prob(batch=0)
     assert lib.msda_sort_queries(ctypes.byref(empty), None, None, None) == _lib.MSDA_OK
+
+
+def test_int8_checks(lib):
+    """MSDA_S8 needs a 4-byte aligned value_scale; the quantiser takes a
+    float32 / bf16 source with D a multiple of 8 and 32-byte aligned codes."""
+    p = _prob(value_dtype=_lib.MSDA_S8)
+    assert _fwd(lib, p) == _lib.MSDA_ERR_INVALID_ARG
+    p.value_scale = ctypes.c_void_p(0x100002)
+    assert _fwd(lib, p) == _lib.MSDA_ERR_INVALID_ARG
+    src = _prob(value_dtype=_lib.MSDA_S8)
+    src.value_scale = FAKE
+    assert lib.msda_quantize_value_s8(ctypes.byref(src), FAKE, FAKE, FAKE, None) == \
+        _lib.MSDA_ERR_INVALID_ARG
+    f32 = _prob()
+    assert lib.msda_quantize_value_s8(ctypes.byref(f32), FAKE, MISALIGNED, FAKE, None) == \
+        _lib.MSDA_ERR_INVALID_ARG
+    assert lib.msda_quantize_value_s8(ctypes.byref(f32), FAKE, FAKE, None, None) == \
+        _lib.MSDA_ERR_INVALID_ARG

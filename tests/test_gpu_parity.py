@@ -66,7 +66,8 @@ def _run_fused(w: wl.Workload, x=None, want_ref=True):
     return errs
 
 
-ALL = sorted(wl.WORKLOADS, key=lambda n: wl.WORKLOADS[n].index)
+ALL = sorted((n for n in wl.WORKLOADS if wl.WORKLOADS[n].dtype != "s8"),
+             key=lambda n: wl.WORKLOADS[n].index)  # INT8 value: tests/test_gpu_int8.py
 
 
 @pytest.mark.parametrize("name", ALL)
