@@ -92,9 +92,10 @@ def parse_args(argv=None):
 def algorithmic_bytes(w: wl.Workload) -> dict:
     """Each tensor of a launch touched once (inputs read, outputs written)."""
     B, S, Q, M, D, L, K = w.B, w.S, w.num_queries, w.M, w.D, w.L, w.K
-    e = 2 if w.dtype == "bf16" else 4
+    e = {"f32": 4, "bf16": 2, "s8": 1}[w.dtype]       # value element
+    er = {"f32": 4, "bf16": 2, "s8": 2}[w.dtype]      # output / grad_output element
     value = B * S * M * D * e
-    rowd = B * Q * M * D * e
+    rowd = B * Q * M * D * er
     samples = B * Q * M * L * K
     loc = samples * 2 * 4
     attn = samples * 4
@@ -104,8 +105,10 @@ def algorithmic_bytes(w: wl.Workload) -> dict:
     bwd = rowd + value + loc + attn + gvalue + loc + attn
     fused_fwd = value + loc + attn + ref + rowd             # offsets, logits, ref -> out
     fused_bwd = rowd + value + loc + attn + ref + gvalue + loc + attn + ref
+    # INT8 storage: the bf16 source read once, the codes written once
+    quantize = B * S * M * D * 3 if w.dtype == "s8" else 0
     return {"forward": fwd, "backward": bwd, "fused_forward": fused_fwd,
-            "fused_backward": fused_bwd, "zero_grads": gvalue + ref}
+            "fused_backward": fused_bwd, "zero_grads": gvalue + ref, "quantize": quantize}
 
 
 # --------------------------------------------------------------- clocks ----
@@ -285,6 +288,9 @@ def run_ours(args):
 
     side = torch.cuda.Stream(device=dev)
     order = torch.empty(B * Q, dtype=torch.int32, device=dev) if args.sorted else None
+    int8 = w.dtype == "s8"
+    qv = torch.empty((B, S, M, D), dtype=torch.int8, device=dev) if int8 else None
+    qs = torch.empty((B, M), dtype=torch.float32, device=dev) if int8 else None
 
     def step(ev, tin=None):
         # the zero-fill of the gradient accumulators does not depend on the
@@ -294,24 +300,27 @@ def run_ours(args):
         ev[0].record(stream)
         if order is not None:
             msda.sort_queries(tin["reference_points"], query_order=order)
+        if int8:  # the step's value arrives as bf16 and is stored as INT8
+            msda.quantize_value_s8(tin["value"], value_s8=qv, value_scale=qs)
+        value = qv if int8 else tin["value"]
         ev[6].record(stream)
         side.wait_event(ev[6])
         with torch.cuda.stream(side):
             ev[4].record(side)
             msda.zero_grads(gv, gref)
             ev[5].record(side)
-        msda.fused_forward(tin["value"], tin["spatial_shapes"], tin["level_start_index"],
+        msda.fused_forward(value, tin["spatial_shapes"], tin["level_start_index"],
                            tin["reference_points"], tin["sampling_offsets"],
-                           tin["attention_logits"], out=out, query_order=order)
+                           tin["attention_logits"], out=out, query_order=order, value_scale=qs)
         ev[1].record(stream)
         stream.wait_event(ev[5])
         ev[2].record(stream)
-        msda.fused_backward(tin["value"], tin["spatial_shapes"], tin["level_start_index"],
+        msda.fused_backward(value, tin["spatial_shapes"], tin["level_start_index"],
                             tin["reference_points"], tin["sampling_offsets"],
                             tin["attention_logits"], tin["grad_output"], accumulate=True,
                             grad_value=gv, grad_reference_points=gref,
                             grad_sampling_offsets=goff, grad_attention_logits=glog,
-                            query_order=order)
+                            query_order=order, value_scale=qs)
         ev[3].record(stream)
         return outputs
 
@@ -341,7 +350,7 @@ def run_ours(args):
     clocks.stop()
 
     fwd = [e[6].elapsed_time(e[1]) for e in evs]
-    sort = [e[0].elapsed_time(e[6]) for e in evs]
+    pre = [e[0].elapsed_time(e[6]) for e in evs]
     zero = [e[4].elapsed_time(e[5]) for e in evs]  # on the side stream, under the forward
     bwd = [e[2].elapsed_time(e[3]) for e in evs]
     stepms = [e[0].elapsed_time(e[3]) for e in evs]
@@ -359,7 +368,7 @@ def run_ours(args):
         achieved = nbytes[dom] / (dom_ms * 1e-3) / 1e9
         tr = NCU_TRAFFIC.get((dom, w.name))
         traffic = tr["bytes"] if tr and tr.get("csrc") == csrc_hash() else None
-        step_bytes = nbytes["fused_forward"] + nbytes["fused_backward"]
+        step_bytes = nbytes["fused_forward"] + nbytes["fused_backward"] + nbytes["quantize"]
         result = {
             "metric": METRIC,
             "value": round(value, 4),
@@ -371,7 +380,8 @@ def run_ours(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "f32" if w.dtype == "f32" else "bf16 value / f32 accumulate",
+            "dtype": {"f32": "f32", "bf16": "bf16 value / f32 accumulate",
+                      "s8": "int8 value (per batch-head scale) / bf16 rows / f32 accumulate"}[w.dtype],
             "data": "synthetic: seeded SplitMix64 + Box-Muller draws of the workload's shapes "
                     "and distributions (no dataset)",
             "config": {
@@ -380,6 +390,7 @@ def run_ours(args):
                 "offset_sigma_px": w.offset_sigma, "logit_sigma": w.logit_sigma,
                 "samples_per_step_per_gpu": samples_step,
                 "step": ("msda_sort_queries -> " if args.sorted else "")
+                + ("msda_quantize_value_s8 -> " if int8 else "")
                 + "msda_fused_forward || msda_zero_grads (second stream) -> msda_fused_backward",
                 "query_order": "Morton cell of the reference point" if args.sorted else "natural",
                 "l2": "flushed between steps (256 MiB write outside the timed events)",
@@ -387,7 +398,8 @@ def run_ours(args):
             },
             "fwd_ms": round(fwd_ms, 5),
             "zero_ms": round(zero_ms, 5),  # overlapped with the forward
-            "sort_ms": round(statistics.mean(sort), 5) if args.sorted else None,
+            # before the forward: the query sort (--sorted) and the INT8 quantisation
+            "pre_ms": round(statistics.mean(pre), 5) if (args.sorted or int8) else None,
 
             "bwd_ms": round(bwd_ms, 5),
             "fwd_gsamples_per_s": round(samples_step / (fwd_ms * 1e-3) / 1e9, 4),
@@ -404,12 +416,15 @@ def run_ours(args):
                 "bytes_per_launch": nbytes[dom],
                 "traffic": traffic,
             },
-            "gpu_launches": (4 if args.sorted else 3) * args.steps,
+            "gpu_launches": (3 + (1 if args.sorted else 0) + (3 if int8 else 0)) * args.steps,
             "host_wall_s": round(wall, 3),
             "clocks": clocks.summary(),
         }
         if want_nonfused:
-            result["nonfused"] = _time_nonfused(msda, t, w, nbytes, flush, min(args.steps, 50))
+            if int8:
+                msda.quantize_value_s8(t["value"], value_s8=qv, value_scale=qs)
+            result["nonfused"] = _time_nonfused(msda, t, w, nbytes, flush, min(args.steps, 50),
+                                                qv if int8 else t["value"], qs)
         if world == 1:
             result["warm_l2"] = _time_warm(w, step, min(args.steps, 50))
         stats = _input_stats(w, x)
@@ -447,15 +462,15 @@ def _peaks():
         return {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def _time_nonfused(msda, t, w, nbytes, flush, n):
+def _time_nonfused(msda, t, w, nbytes, flush, n, value, value_scale=None):
     """msda_forward / msda_backward (pre-computed locations and weights) on the
     same workload: per-launch device times (L2 flushed before each)."""
     import torch
     stream = torch.cuda.current_stream()
-    args = (t["value"], t["spatial_shapes"], t["level_start_index"], t["sampling_locations"],
+    args = (value, t["spatial_shapes"], t["level_start_index"], t["sampling_locations"],
             t["attention_weights"])
     out = torch.empty_like(t["grad_output"])
-    gv = torch.empty(t["value"].shape, dtype=torch.float32, device=t["value"].device)
+    gv = torch.empty(value.shape, dtype=torch.float32, device=value.device)
     gl = torch.empty_like(t["sampling_locations"])
     ga = torch.empty_like(t["attention_weights"])
     f, b = [], []
@@ -463,13 +478,13 @@ def _time_nonfused(msda, t, w, nbytes, flush, n):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         flush.fill_(float(i))
         e[0].record(stream)
-        msda.forward(*args, out=out)
+        msda.forward(*args, out=out, value_scale=value_scale)
         e[1].record(stream)
         msda.zero_grads(gv)
         flush.fill_(float(i + 1))
         e[2].record(stream)
         msda.backward(*args, t["grad_output"], grad_value=gv, grad_sampling_locations=gl,
-                      grad_attention_weights=ga, accumulate=True)
+                      grad_attention_weights=ga, accumulate=True, value_scale=value_scale)
         e[3].record(stream)
         if i >= 3:
             f.append(e)
@@ -528,7 +543,7 @@ def _input_stats(w: wl.Workload, x: wl.Inputs, max_queries: int = 4096) -> dict:
         start = x.level_start_index[None, None, None, :, None]
         b = np.arange(w.B)[:, None, None, None, None]
         m = np.arange(w.M)[None, None, :, None, None]
-        elt = 4 if w.dtype == "f32" else 2
+        elt = {"f32": 4, "bf16": 2, "s8": 1}[w.dtype]
         row_bytes = w.D * elt
         rows = []
         for dy in (0, 1):
