@@ -29,6 +29,12 @@ class _Dims(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in ("B", "S", "Q", "M", "D", "L", "K")]
 
 
+class _DcnDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("N", "H", "W", "G", "C", "Ho", "Wo", "kh", "kw",
+                                              "stride_h", "stride_w", "pad_h", "pad_w",
+                                              "dil_h", "dil_w")]
+
+
 def build(force: bool = False) -> str:
     """Compiles the oracle with gcc into oracle/_build (no GPU involved)."""
     os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
@@ -52,9 +58,13 @@ def _load():
             lib.msda_oracle_softmax.argtypes = [D, P, P]
             lib.msda_oracle_fused_chain.argtypes = [D, P, P, P, P, P, P, P]
             lib.msda_oracle_quantize_value_s8.argtypes = [D, P, P, P]
+            DD = ctypes.POINTER(_DcnDims)
+            lib.msda_oracle_dcn_forward.argtypes = [DD, P, P, P, P]
+            lib.msda_oracle_dcn_backward.argtypes = [DD, P, P, P, P, P, P, P]
             for f in ("msda_oracle_forward", "msda_oracle_backward", "msda_oracle_sampling_locations",
                       "msda_oracle_softmax", "msda_oracle_fused_chain",
-                      "msda_oracle_quantize_value_s8"):
+                      "msda_oracle_quantize_value_s8", "msda_oracle_dcn_forward",
+                      "msda_oracle_dcn_backward"):
                 getattr(lib, f).restype = None
             _lib = lib
     return _lib
@@ -189,3 +199,41 @@ def quantize_value_s8(value):
 def dequantize_value_s8(q, scale):
     """q * scale in float64 (exact), [B,S,M,D]: the value the operator samples."""
     return np.asarray(q, np.float64) * np.asarray(scale, np.float64)[:, None, :, None]
+
+
+def dcn_output_size(H: int, W: int, kernel, stride=(1, 1), pad=(0, 0), dil=(1, 1)):
+    """(Ho, Wo) of the convolution grid."""
+    kh, kw = kernel
+    return ((H + 2 * pad[0] - dil[0] * (kh - 1) - 1) // stride[0] + 1,
+            (W + 2 * pad[1] - dil[1] * (kw - 1) - 1) // stride[1] + 1)
+
+
+def _dcn_dims(x, kernel, stride, pad, dil):
+    N, H, W, G, C = x.shape
+    Ho, Wo = dcn_output_size(H, W, kernel, stride, pad, dil)
+    return _DcnDims(N, H, W, G, C, Ho, Wo, kernel[0], kernel[1], stride[0], stride[1],
+                    pad[0], pad[1], dil[0], dil[1])
+
+
+def dcn_forward(x, offset, mask, kernel, stride=(1, 1), pad=(0, 0), dil=(1, 1)):
+    """DCNv3 core forward, float64: x [N,H,W,G,C], offset [N,Ho,Wo,G,K,2]
+    (x, y) pixels, mask [N,Ho,Wo,G,K] -> y [N,Ho,Wo,G,C]."""
+    xv, off, m = _f64(x), _f64(offset), _f64(mask)
+    d = _dcn_dims(xv, kernel, stride, pad, dil)
+    assert off.shape == (d.N, d.Ho, d.Wo, d.G, d.kh * d.kw, 2) and m.shape == off.shape[:-1]
+    y = np.empty((d.N, d.Ho, d.Wo, d.G, d.C), np.float64)
+    _load().msda_oracle_dcn_forward(ctypes.byref(d), _p(xv), _p(off), _p(m), _p(y))
+    return y
+
+
+def dcn_backward(x, offset, mask, grad_y, kernel, stride=(1, 1), pad=(0, 0), dil=(1, 1)):
+    """(grad_x, grad_offset, grad_mask), float64."""
+    xv, off, m, gy = _f64(x), _f64(offset), _f64(mask), _f64(grad_y)
+    d = _dcn_dims(xv, kernel, stride, pad, dil)
+    assert gy.shape == (d.N, d.Ho, d.Wo, d.G, d.C)
+    gx = np.empty_like(xv)
+    goff = np.empty_like(off)
+    gm = np.empty_like(m)
+    _load().msda_oracle_dcn_backward(ctypes.byref(d), _p(xv), _p(off), _p(m), _p(gy), _p(gx),
+                                     _p(goff), _p(gm))
+    return gx, goff, gm

@@ -67,12 +67,19 @@ typedef struct {
     double w[4];
 } bilinear;
 
+static bilinear bilinear_at_pixel(double x, double y, int64_t H, int64_t W);
+
+/* A normalized location: pixel coordinate x = lx * W - 0.5, y = ly * H - 0.5. */
 static bilinear bilinear_setup(double lx, double ly, int64_t H, int64_t W)
+{
+    return bilinear_at_pixel(lx * (double)W - 0.5, ly * (double)H - 0.5, H, W);
+}
+
+/* A pixel coordinate (pixel centres at integers). */
+static bilinear bilinear_at_pixel(double x, double y, int64_t H, int64_t W)
 {
     bilinear s;
     memset(&s, 0, sizeof s);
-    double x = lx * (double)W - 0.5;
-    double y = ly * (double)H - 0.5;
     s.valid = (x > -1.0) && (x < (double)W) && (y > -1.0) && (y < (double)H);
     if (!s.valid)
         return s;
@@ -323,4 +330,126 @@ void msda_oracle_quantize_value_s8(const oracle_dims *d, const float *value, int
                     q[i] = (int8_t)r;
                 }
         }
+}
+
+/*
+ * DCNv3 core ([discosf] §4.2): for output pixel p0 = (i, j) of image n and
+ * group g,
+ *   y[n,i,j,g,:] = sum_k m[n,i,j,g,k] * x_g(p0 + p_k + dp[n,i,j,g,k])
+ * where x_g bilinearly samples group g of the channels-last input
+ * x[N, H, W, G, C] at a pixel coordinate (pixel centres at integers, corners
+ * outside the map contribute zero, a sample is taken only when -1 < px < W
+ * and -1 < py < H).  The grid p0 + p_k is the convolution's: point k = r*kw + c
+ * of a kh x kw kernel sits at
+ *   px = j*stride_w - pad_w + c*dil_w,  py = i*stride_h - pad_h + r*dil_h,
+ * and the offset dp = (dx, dy) is added in pixels.  The shared projection w_g
+ * of the formula is a linear layer outside the core, like the attention's
+ * projections.  Readings (listed with the others): the page gives the
+ * formula only; the conv grid, the pixel-centre convention, (x, y) offset
+ * order and taking m as given (no normalisation inside the core) are the
+ * plainest completions.
+ * Layouts: x [N,H,W,G,C]; offset [N,Ho,Wo,G,K,2]; mask [N,Ho,Wo,G,K];
+ * y [N,Ho,Wo,G,C]; K = kh*kw.
+ */
+typedef struct {
+    int64_t N, H, W, G, C, Ho, Wo, kh, kw, stride_h, stride_w, pad_h, pad_w, dil_h, dil_w;
+} dcn_dims;
+
+static bilinear dcn_sample(const dcn_dims *d, int64_t i, int64_t j, int64_t k, const double *dp)
+{
+    const int64_t r = k / d->kw, c = k % d->kw;
+    const double px = (double)(j * d->stride_w - d->pad_w + c * d->dil_w) + dp[0];
+    const double py = (double)(i * d->stride_h - d->pad_h + r * d->dil_h) + dp[1];
+    return bilinear_at_pixel(px, py, d->H, d->W);
+}
+
+static int64_t dcn_row(const dcn_dims *d, int64_t n, int64_t cy, int64_t cx, int64_t g)
+{
+    return (((n * d->H + cy) * d->W + cx) * d->G + g) * d->C;
+}
+
+void msda_oracle_dcn_forward(const dcn_dims *d, const double *x, const double *offset,
+                             const double *mask, double *y)
+{
+    const int64_t K = d->kh * d->kw;
+    for (int64_t n = 0; n < d->N; ++n)
+    for (int64_t i = 0; i < d->Ho; ++i)
+    for (int64_t j = 0; j < d->Wo; ++j)
+    for (int64_t g = 0; g < d->G; ++g) {
+        const int64_t row = ((n * d->Ho + i) * d->Wo + j) * d->G + g;
+        double *o = y + row * d->C;
+        for (int64_t ch = 0; ch < d->C; ++ch)
+            o[ch] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const int64_t p = row * K + k;
+            bilinear s = dcn_sample(d, i, j, k, offset + 2 * p);
+            if (!s.valid)
+                continue;
+            for (int c = 0; c < 4; ++c) {
+                if (!s.inb[c])
+                    continue;
+                const double *v = x + dcn_row(d, n, s.cy[c], s.cx[c], g);
+                for (int64_t ch = 0; ch < d->C; ++ch)
+                    o[ch] += mask[p] * s.w[c] * v[ch];
+            }
+        }
+    }
+}
+
+/*
+ * DCNv3 core backward: exact derivative of the forward sum.  With s the
+ * bilinear sample and g = grad_y[n,i,j,g,:]:
+ *   grad_mask      = <g, s>
+ *   grad_offset_x  = m * <g, ds/dpx>,  grad_offset_y = m * <g, ds/dpy>
+ *                    (the offsets are in pixels: no scale factor)
+ *   grad_x[corner c] += m * w_c * g   (in-map corners; grad_x zeroed first)
+ */
+void msda_oracle_dcn_backward(const dcn_dims *d, const double *x, const double *offset,
+                              const double *mask, const double *grad_y, double *grad_x,
+                              double *grad_offset, double *grad_mask)
+{
+    const int64_t K = d->kh * d->kw;
+    const int64_t nx = d->N * d->H * d->W * d->G * d->C;
+    for (int64_t t = 0; t < nx; ++t)
+        grad_x[t] = 0.0;
+    for (int64_t n = 0; n < d->N; ++n)
+    for (int64_t i = 0; i < d->Ho; ++i)
+    for (int64_t j = 0; j < d->Wo; ++j)
+    for (int64_t g = 0; g < d->G; ++g) {
+        const int64_t row = ((n * d->Ho + i) * d->Wo + j) * d->G + g;
+        const double *gy = grad_y + row * d->C;
+        for (int64_t k = 0; k < K; ++k) {
+            const int64_t p = row * K + k;
+            bilinear s = dcn_sample(d, i, j, k, offset + 2 * p);
+            grad_mask[p] = 0.0;
+            grad_offset[2 * p] = 0.0;
+            grad_offset[2 * p + 1] = 0.0;
+            if (!s.valid)
+                continue;
+            const double *v[4];
+            for (int c = 0; c < 4; ++c)
+                v[c] = s.inb[c] ? x + dcn_row(d, n, s.cy[c], s.cx[c], g) : 0;
+            double gm = 0.0, gx = 0.0, gyy = 0.0;
+            for (int64_t ch = 0; ch < d->C; ++ch) {
+                const double v00 = v[0] ? v[0][ch] : 0.0, v01 = v[1] ? v[1][ch] : 0.0;
+                const double v10 = v[2] ? v[2][ch] : 0.0, v11 = v[3] ? v[3][ch] : 0.0;
+                const double samp = s.w[0] * v00 + s.w[1] * v01 + s.w[2] * v10 + s.w[3] * v11;
+                const double dx = (1.0 - s.fy) * (v01 - v00) + s.fy * (v11 - v10);
+                const double dy = (1.0 - s.fx) * (v10 - v00) + s.fx * (v11 - v01);
+                gm += gy[ch] * samp;
+                gx += gy[ch] * dx;
+                gyy += gy[ch] * dy;
+            }
+            grad_mask[p] = gm;
+            grad_offset[2 * p] = mask[p] * gx;
+            grad_offset[2 * p + 1] = mask[p] * gyy;
+            for (int c = 0; c < 4; ++c) {
+                if (!s.inb[c])
+                    continue;
+                double *gxr = grad_x + dcn_row(d, n, s.cy[c], s.cx[c], g);
+                for (int64_t ch = 0; ch < d->C; ++ch)
+                    gxr[ch] += mask[p] * s.w[c] * gy[ch];
+            }
+        }
+    }
 }

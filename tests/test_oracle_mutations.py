@@ -14,14 +14,16 @@ import subprocess
 import pytest
 
 import oracle
+from tests import test_oracle_dcn as dcn_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "msda_oracle.c")
+_PIX = "return bilinear_at_pixel(lx * (double)W - 0.5, ly * (double)H - 0.5, H, W);"
 
 MUTATIONS = {
-    "no_half_pixel_shift": ("double x = lx * (double)W - 0.5;", "double x = lx * (double)W;"),
-    "align_corners_true": ("double x = lx * (double)W - 0.5;", "double x = lx * (double)(W - 1);"),
-    "x_y_swapped_scale": ("double y = ly * (double)H - 0.5;", "double y = ly * (double)W - 0.5;"),
+    "no_half_pixel_shift": (_PIX, "return bilinear_at_pixel(lx * (double)W, ly * (double)H - 0.5, H, W);"),
+    "align_corners_true": (_PIX, "return bilinear_at_pixel(lx * (double)(W - 1), ly * (double)H - 0.5, H, W);"),
+    "x_y_swapped_scale": (_PIX, "return bilinear_at_pixel(lx * (double)W - 0.5, ly * (double)W - 0.5, H, W);"),
     "corner_weight_transposed": ("s.w[1] = (1.0 - s.fy) * s.fx;", "s.w[1] = s.fy * (1.0 - s.fx);"),
     "column_mirrored": ("int64_t key = start_l + cy * W + cx;",
                         "int64_t key = start_l + cy * W + (W - 1 - cx);"),
@@ -33,13 +35,13 @@ MUTATIONS = {
                               "s.cy[c] = s.cy[c] < 0 ? 0 : (s.cy[c] >= H ? H - 1 : s.cy[c]); "
                               "s.inb[c] = 1;"),
     "grad_x_scale_H": ("grad_loc[2 * p] = (double)W * a * gx;", "grad_loc[2 * p] = (double)H * a * gx;"),
-    "dsdx_sign": ("double dx = (1.0 - s.fy) * (v01 - v00) + s.fy * (v11 - v10);",
-                  "double dx = (1.0 - s.fy) * (v00 - v01) + s.fy * (v11 - v10);"),
-    "dsdy_dropped_term": ("double dy = (1.0 - s.fx) * (v10 - v00) + s.fx * (v11 - v01);",
-                          "double dy = (1.0 - s.fx) * (v10 - v00);"),
+    "dsdx_sign": ("  double dx = (1.0 - s.fy) * (v01 - v00) + s.fy * (v11 - v10);",
+                  "  double dx = (1.0 - s.fy) * (v00 - v01) + s.fy * (v11 - v10);"),
+    "dsdy_dropped_term": ("  double dy = (1.0 - s.fx) * (v10 - v00) + s.fx * (v11 - v01);",
+                          "  double dy = (1.0 - s.fx) * (v10 - v00);"),
     "grad_value_no_weight": ("gv[ch] += a * s.w[c] * g[ch];", "gv[ch] += a * g[ch];"),
-    "grad_attn_unweighted": ("double samp = s.w[0] * v00 + s.w[1] * v01 + s.w[2] * v10 + s.w[3] * v11;",
-                             "double samp = v00 + v01 + v10 + v11;"),
+    "grad_attn_unweighted": ("  double samp = s.w[0] * v00 + s.w[1] * v01 + s.w[2] * v10 + s.w[3] * v11;",
+                             "  double samp = v00 + v01 + v10 + v11;"),
     "offset_normalizer_swapped": ("loc[2 * p] = r[0] + off[2 * p] / (double)shapes[2 * l + 1];",
                                   "loc[2 * p] = r[0] + off[2 * p] / (double)shapes[2 * l];"),
     "softmax_no_normalize": ("a[j] /= sum;", "a[j] /= 1.0;"),
@@ -49,6 +51,20 @@ MUTATIONS = {
                             "grad_off[2 * p] = grad_loc[2 * p];"),
     "grad_ref_y_from_x": ("grad_ref[2 * (b * d->Q + q) + 1] += grad_loc[2 * p + 1];",
                           "grad_ref[2 * (b * d->Q + q) + 1] += grad_loc[2 * p];"),
+}
+
+# mistakes in the DCNv3 core, caught by its own pins
+DCN_MUTATIONS = {
+    "dcn_no_dilation": ("const double px = (double)(j * d->stride_w - d->pad_w + c * d->dil_w) + dp[0];",
+                        "const double px = (double)(j * d->stride_w - d->pad_w + c) + dp[0];"),
+    "dcn_offset_xy_swapped": ("const double py = (double)(i * d->stride_h - d->pad_h + r * d->dil_h) + dp[1];",
+                              "const double py = (double)(i * d->stride_h - d->pad_h + r * d->dil_h) + dp[0];"),
+    "dcn_grid_transposed": ("const int64_t r = k / d->kw, c = k % d->kw;",
+                            "const int64_t c = k / d->kh, r = k % d->kh;"),
+    "dcn_grad_offset_unweighted": ("grad_offset[2 * p] = mask[p] * gx;", "grad_offset[2 * p] = gx;"),
+    "dcn_grad_x_no_mask": ("gxr[ch] += mask[p] * s.w[c] * gy[ch];", "gxr[ch] += s.w[c] * gy[ch];"),
+    "dcn_stride_ignored": ("const double py = (double)(i * d->stride_h - d->pad_h + r * d->dil_h) + dp[1];",
+                           "const double py = (double)(i - d->pad_h + r * d->dil_h) + dp[1];"),
 }
 
 PIN_CHECKS = [
@@ -63,6 +79,15 @@ PIN_CHECKS = [
     lambda o: pins.test_matches_torch_grid_sample(o, "ragged"),
 ]
 
+DCN_PIN_CHECKS = [
+    lambda o: dcn_pins.test_zero_offsets_are_a_depthwise_convolution((3, 3), (2, 2), (1, 1), (1, 1)),
+    lambda o: dcn_pins.test_zero_offsets_are_a_depthwise_convolution((3, 3), (1, 1), (2, 2), (2, 2)),
+    lambda o: dcn_pins.test_zero_offsets_are_a_depthwise_convolution((5, 3), (1, 2), (2, 1), (1, 1)),
+    lambda o: dcn_pins.test_integer_and_half_pixel_offsets(),
+    lambda o: dcn_pins.test_backward_finite_differences(),
+    lambda o: dcn_pins.test_adjoint_identities(),
+]
+
 
 @contextlib.contextmanager
 def _swapped(lib_path):
@@ -70,7 +95,8 @@ def _swapped(lib_path):
     saved = oracle._lib
     lib = ctypes.CDLL(lib_path)
     for name in ("msda_oracle_forward", "msda_oracle_backward", "msda_oracle_sampling_locations",
-                 "msda_oracle_softmax", "msda_oracle_fused_chain"):
+                 "msda_oracle_softmax", "msda_oracle_fused_chain", "msda_oracle_dcn_forward",
+                 "msda_oracle_dcn_backward"):
         f, ref = getattr(lib, name), getattr(saved, name)
         f.argtypes, f.restype = ref.argtypes, ref.restype
     oracle._lib = lib
@@ -80,9 +106,10 @@ def _swapped(lib_path):
         oracle._lib = saved
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS))
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(DCN_MUTATIONS))
 def test_planted_mistake_is_caught(name, tmp_path):
-    old, new = MUTATIONS[name]
+    old, new = MUTATIONS[name] if name in MUTATIONS else DCN_MUTATIONS[name]
+    checks = PIN_CHECKS if name in MUTATIONS else DCN_PIN_CHECKS
     src = open(SRC).read()
     assert src.count(old) == 1, name
     mutated = tmp_path / "mut.c"
@@ -92,7 +119,7 @@ def test_planted_mistake_is_caught(name, tmp_path):
                            str(mutated), "-lm"])
     failures = 0
     with _swapped(lib_path):
-        for check in PIN_CHECKS:
+        for check in checks:
             try:
                 check(oracle)
             except AssertionError:
