@@ -297,6 +297,69 @@ MSDA_API msda_status msda_sort_queries(const msda_problem *problem, const float 
 MSDA_API msda_status msda_backward_workspace_size(const msda_problem *problem, size_t *bytes);
 
 /*
+ * DCNv3 core (discosf.com/news/5175395 §4.2, the operator of InternImage):
+ *
+ *   y[n,i,j,g,:] = sum_k mask[n,i,j,g,k] * x_g( p0(i,j) + p_k + offset[n,i,j,g,k] )
+ *
+ * the same gather-reduce on one map, with a convolution's sampling grid.
+ * Point k = r*kernel_w + c of output pixel (i, j) sits at pixel coordinate
+ *   px = j*stride_w - pad_w + c*dilation_w + dx,
+ *   py = i*stride_h - pad_h + r*dilation_h + dy
+ * (pixel centres at integers; bilinear; corners outside the H x W map read
+ * zero; a sample is taken only when -1 < px < W and -1 < py < H).  The group
+ * projection w_g of the formula is a linear layer outside the core.  The page
+ * gives only the formula: the grid convention, (dx, dy) order and taking the
+ * mask as given (no normalisation inside the core) are this library's
+ * reading.  Output size: Ho = (H + 2*pad_h - dilation_h*(kernel_h-1) - 1) /
+ * stride_h + 1, likewise Wo.
+ *   input        [N, H, W, G, C]          value_dtype (channels last, group-major)
+ *   offset       [N, Ho, Wo, G, K, 2]     float32 (dx, dy) pixels, K = kh*kw
+ *   mask         [N, Ho, Wo, G, K]        float32
+ *   output       [N, Ho, Wo, G, C]        value_dtype (bf16 for MSDA_S8)
+ * Supported: C (group_channels) in {8, 16, 32, 64, 128, 256}; kernel_w <= 32,
+ * kernel_h <= 16, kernel_h*kernel_w <= 128; H, W <= 65535; stride and
+ * dilation >= 1; pad >= 0; N*Ho*Wo < 2^31.  Flags and dtypes as for the
+ * attention calls (MSDA_S8 needs value_scale [N, G]).
+ */
+typedef struct msda_dcn_problem {
+    int64_t batch;          /* N */
+    int32_t height, width;  /* H, W of the input map */
+    int32_t groups;         /* G */
+    int32_t group_channels; /* C */
+    int32_t kernel_h, kernel_w;
+    int32_t stride_h, stride_w;
+    int32_t pad_h, pad_w;
+    int32_t dilation_h, dilation_w;
+    int32_t value_dtype;    /* msda_dtype of input (and output, grad_output) */
+    uint32_t flags;         /* MSDA_GRAD_VALUE_BF16, MSDA_ACCUMULATE_GRADS */
+    const float *value_scale; /* MSDA_S8 only: [N, G] float32 */
+} msda_dcn_problem;
+
+/* Ho and Wo of `problem` (host only). */
+MSDA_API msda_status msda_dcn_output_size(const msda_dcn_problem *problem, int64_t *out_h,
+                                          int64_t *out_w);
+
+MSDA_API msda_status msda_dcn_forward(const msda_dcn_problem *problem, const void *input,
+                                      const float *offset, const float *mask, void *output,
+                                      msda_stream_t stream);
+
+/*
+ * Gradients of the DCNv3 core: grad_input (zeroed first unless
+ * MSDA_ACCUMULATE_GRADS; float32, or bf16 through a float32 workspace of
+ * msda_dcn_backward_workspace_size() bytes with MSDA_GRAD_VALUE_BF16),
+ * grad_offset [N,Ho,Wo,G,K,2] = mask * <g, dsample/dp> (pixels) and grad_mask
+ * [N,Ho,Wo,G,K] = <g, sample>, both overwritten.
+ */
+MSDA_API msda_status msda_dcn_backward(const msda_dcn_problem *problem, const void *input,
+                                       const float *offset, const float *mask,
+                                       const void *grad_output, void *grad_input,
+                                       float *grad_offset, float *grad_mask, void *workspace,
+                                       size_t workspace_bytes, msda_stream_t stream);
+
+MSDA_API msda_status msda_dcn_backward_workspace_size(const msda_dcn_problem *problem,
+                                                      size_t *bytes);
+
+/*
  * Synchronizes `stream`, then returns in *code the status the kernels recorded
  * on the current device since the last call (MSDA_OK, MSDA_ERR_DEVICE_CHECK or
  * MSDA_ERR_DEVICE_TIMEOUT), and clears it.  Returns MSDA_ERR_CUDA if the

@@ -10,6 +10,8 @@ from .binding import (  # noqa: F401
     MSDeformAttnFusedFunction,
     backward,
     backward_noalloc,
+    dcn_backward,
+    dcn_forward,
     device_status,
     forward,
     fused_backward,

@@ -44,6 +44,30 @@ class Problem(ctypes.Structure):
 
 _P = ctypes.c_void_p
 _PROB = ctypes.POINTER(Problem)
+class DcnProblem(ctypes.Structure):
+    """msda_dcn_problem of include/msda.h."""
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("height", ctypes.c_int32),
+        ("width", ctypes.c_int32),
+        ("groups", ctypes.c_int32),
+        ("group_channels", ctypes.c_int32),
+        ("kernel_h", ctypes.c_int32),
+        ("kernel_w", ctypes.c_int32),
+        ("stride_h", ctypes.c_int32),
+        ("stride_w", ctypes.c_int32),
+        ("pad_h", ctypes.c_int32),
+        ("pad_w", ctypes.c_int32),
+        ("dilation_h", ctypes.c_int32),
+        ("dilation_w", ctypes.c_int32),
+        ("value_dtype", ctypes.c_int32),
+        ("flags", ctypes.c_uint32),
+        ("value_scale", ctypes.c_void_p),
+    ]
+
+
+_DCN = ctypes.POINTER(DcnProblem)
+
 _SIGNATURES = {
     "msda_forward": [_PROB, _P, _P, _P, _P, _P, _P, _P],
     "msda_backward": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
@@ -54,6 +78,10 @@ _SIGNATURES = {
     "msda_backward_noalloc": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "msda_sort_queries": [_PROB, _P, _P, _P],
     "msda_quantize_value_s8": [_PROB, _P, _P, _P, _P],
+    "msda_dcn_output_size": [_DCN, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)],
+    "msda_dcn_forward": [_DCN, _P, _P, _P, _P, _P],
+    "msda_dcn_backward": [_DCN, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "msda_dcn_backward_workspace_size": [_DCN, ctypes.POINTER(ctypes.c_size_t)],
     "msda_get_device_status": [_P, ctypes.POINTER(ctypes.c_int32)],
     "msda_status_string": [ctypes.c_int],
     "msda_version": [],

@@ -336,6 +336,86 @@ def quantize_value_s8(value: torch.Tensor, value_s8: Optional[torch.Tensor] = No
     return value_s8, value_scale
 
 
+def _pair(v):
+    return (int(v), int(v)) if isinstance(v, int) else (int(v[0]), int(v[1]))
+
+
+def _dcn_problem(input: torch.Tensor, kernel, stride, pad, dilation, flags=0, value_scale=None):
+    if input.dim() != 5:
+        raise ValueError("input must be [N, H, W, G, C]")
+    if input.dtype not in _DTYPES:
+        raise TypeError("input must be float32, bfloat16 or int8 (with value_scale)")
+    N, H, W, G, C = input.shape
+    (kh, kw), (sh, sw), (ph, pw), (dh, dw) = _pair(kernel), _pair(stride), _pair(pad), _pair(dilation)
+    prob = _lib.DcnProblem(N, H, W, G, C, kh, kw, sh, sw, ph, pw, dh, dw, _DTYPES[input.dtype], flags)
+    if input.dtype == torch.int8:
+        if value_scale is None:
+            raise ValueError("int8 input needs value_scale [N, G] (see quantize_value_s8)")
+        _need(value_scale, "value_scale", torch.float32, (N, G), input.device)
+        prob.value_scale = _ptr(value_scale)
+    ho, wo = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(_lib.load().msda_dcn_output_size(ctypes.byref(prob), ctypes.byref(ho), ctypes.byref(wo)),
+           "msda_dcn_output_size")
+    return prob, ho.value, wo.value
+
+
+def dcn_forward(input: torch.Tensor, offset: torch.Tensor, mask: torch.Tensor, kernel=3, stride=1,
+                pad=1, dilation=1, out: Optional[torch.Tensor] = None,
+                value_scale: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """msda_dcn_forward (DCNv3 core): input [N,H,W,G,C], offset [N,Ho,Wo,G,K,2]
+    (dx, dy) pixels, mask [N,Ho,Wo,G,K] (used as given) -> [N,Ho,Wo,G,C]."""
+    _need(input, "input", None)
+    prob, Ho, Wo = _dcn_problem(input, kernel, stride, pad, dilation, 0, value_scale)
+    N, H, W, G, C = input.shape
+    K = prob.kernel_h * prob.kernel_w
+    dev = input.device
+    _need(offset, "offset", torch.float32, (N, Ho, Wo, G, K, 2), dev)
+    _need(mask, "mask", torch.float32, (N, Ho, Wo, G, K), dev)
+    if out is None:
+        out = torch.empty((N, Ho, Wo, G, C), dtype=_row_dtype(input), device=dev)
+    _need(out, "out", _row_dtype(input), (N, Ho, Wo, G, C), dev)
+    st = _lib.load().msda_dcn_forward(ctypes.byref(prob), _ptr(input), _ptr(offset), _ptr(mask),
+                                      _ptr(out), _stream())
+    _check(st, "msda_dcn_forward")
+    return out
+
+
+def dcn_backward(input, offset, mask, grad_output, kernel=3, stride=1, pad=1, dilation=1,
+                 grad_input_dtype=torch.float32, grad_input: Optional[torch.Tensor] = None,
+                 accumulate: bool = False, value_scale: Optional[torch.Tensor] = None):
+    """msda_dcn_backward: (grad_input, grad_offset, grad_mask)."""
+    _need(input, "input", None)
+    if grad_input_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("grad_input_dtype must be float32 or bfloat16")
+    flags = _lib.MSDA_GRAD_VALUE_BF16 if grad_input_dtype == torch.bfloat16 else 0
+    if accumulate:
+        if grad_input is None:
+            raise ValueError("accumulate=True needs the grad_input buffer to add into")
+        flags |= _lib.MSDA_ACCUMULATE_GRADS
+    prob, Ho, Wo = _dcn_problem(input, kernel, stride, pad, dilation, flags, value_scale)
+    N, H, W, G, C = input.shape
+    K = prob.kernel_h * prob.kernel_w
+    dev = input.device
+    _need(offset, "offset", torch.float32, (N, Ho, Wo, G, K, 2), dev)
+    _need(mask, "mask", torch.float32, (N, Ho, Wo, G, K), dev)
+    _need(grad_output, "grad_output", _row_dtype(input), (N, Ho, Wo, G, C), dev)
+    if grad_input is None:
+        grad_input = torch.empty((N, H, W, G, C), dtype=grad_input_dtype, device=dev)
+    _need(grad_input, "grad_input", grad_input_dtype, (N, H, W, G, C), dev)
+    goff = torch.empty_like(offset)
+    gmask = torch.empty_like(mask)
+    lib = _lib.load()
+    ws_bytes = ctypes.c_size_t(0)
+    _check(lib.msda_dcn_backward_workspace_size(ctypes.byref(prob), ctypes.byref(ws_bytes)),
+           "msda_dcn_backward_workspace_size")
+    workspace = torch.empty(ws_bytes.value, dtype=torch.uint8, device=dev) if ws_bytes.value else None
+    st = lib.msda_dcn_backward(ctypes.byref(prob), _ptr(input), _ptr(offset), _ptr(mask),
+                               _ptr(grad_output), _ptr(grad_input), _ptr(goff), _ptr(gmask),
+                               _ptr(workspace), ws_bytes.value, _stream())
+    _check(st, "msda_dcn_backward")
+    return grad_input, goff, gmask
+
+
 def sort_queries(points: torch.Tensor, query_order: Optional[torch.Tensor] = None) -> torch.Tensor:
     """msda_sort_queries: int32 [B*Q] order of the queries by batch, then by
     the Morton code of the 64 x 64 cell of [0,1]^2 holding points[b, q]

@@ -400,9 +400,129 @@ msda_status noalloc_scratch(int dev, float **ptr)
     return MSDA_OK;
 }
 
+// DCNv3 core as the attention kernels' non-fused path: keys = the H*W input
+// pixels, queries = the Ho*Wo output pixels, heads = groups, head_dim =
+// group channels, levels = kernel rows, points = kernel columns.
+msda_status dcn_to_problem(const msda_dcn_problem *d, msda_problem &p, int64_t &ho, int64_t &wo)
+{
+    if (!d)
+        return MSDA_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->height < 1 || d->width < 1 || d->groups < 1 || d->group_channels < 1 ||
+        d->kernel_h < 1 || d->kernel_w < 1 || d->stride_h < 1 || d->stride_w < 1 || d->pad_h < 0 ||
+        d->pad_w < 0 || d->dilation_h < 1 || d->dilation_w < 1)
+        return MSDA_ERR_INVALID_ARG;
+    if (d->height > 65535 || d->width > 65535 || d->pad_h > 65535 || d->pad_w > 65535 ||
+        d->stride_h > 65535 || d->stride_w > 65535 || d->dilation_h > 65535 || d->dilation_w > 65535)
+        return MSDA_ERR_UNSUPPORTED;
+    ho = ((int64_t)d->height + 2 * (int64_t)d->pad_h - (int64_t)d->dilation_h * (d->kernel_h - 1) - 1);
+    wo = ((int64_t)d->width + 2 * (int64_t)d->pad_w - (int64_t)d->dilation_w * (d->kernel_w - 1) - 1);
+    ho = ho < 0 ? 0 : ho / d->stride_h + 1;
+    wo = wo < 0 ? 0 : wo / d->stride_w + 1;
+    p = msda_problem{};
+    p.batch = d->batch;
+    p.num_keys = (int64_t)d->height * d->width;
+    p.num_queries = ho * wo;
+    p.num_heads = d->groups;
+    p.head_dim = d->group_channels;
+    p.num_levels = d->kernel_h;
+    p.num_points = d->kernel_w;
+    p.value_dtype = d->value_dtype;
+    p.flags = d->flags;
+    p.value_scale = d->value_scale;
+    if (p.flags & MSDA_TEST_WITHHOLD_COPY)
+        return MSDA_ERR_INVALID_ARG;
+    return check_problem(&p);
+}
+
+void dcn_args(const msda_dcn_problem *d, int64_t wo, KernelArgs &a)
+{
+    a.dcn = 1;
+    a.dcn_h = d->height;
+    a.dcn_w = d->width;
+    a.dcn_wo = (int)wo;
+    a.stride_h = d->stride_h;
+    a.stride_w = d->stride_w;
+    a.pad_h = d->pad_h;
+    a.pad_w = d->pad_w;
+    a.dil_h = d->dilation_h;
+    a.dil_w = d->dilation_w;
+}
+
 }  // namespace
 
 extern "C" {
+
+msda_status msda_dcn_output_size(const msda_dcn_problem *problem, int64_t *out_h, int64_t *out_w)
+{
+    msda_problem p;
+    int64_t ho = 0, wo = 0;
+    msda_status st = dcn_to_problem(problem, p, ho, wo);
+    if (st != MSDA_OK)
+        return st;
+    if (!out_h || !out_w)
+        return MSDA_ERR_INVALID_ARG;
+    *out_h = ho;
+    *out_w = wo;
+    return MSDA_OK;
+}
+
+msda_status msda_dcn_forward(const msda_dcn_problem *problem, const void *input, const float *offset,
+                             const float *mask, void *output, msda_stream_t stream)
+{
+    msda_problem p;
+    int64_t ho = 0, wo = 0;
+    msda_status st = dcn_to_problem(problem, p, ho, wo);
+    if (st != MSDA_OK)
+        return st;
+    const Sizes z = sizes_of(&p);
+    if (!vec_ptr_ok(input, z.value) || !ptr_ok(offset, z.samples * 2) || !ptr_ok(mask, z.samples) ||
+        !vec_ptr_ok(output, z.rows_d))
+        return MSDA_ERR_INVALID_ARG;
+    KernelArgs a = base_args(&p, input, nullptr, nullptr);
+    if (a.rows == 0)
+        return MSDA_OK;
+    dcn_args(problem, wo, a);
+    a.loc = offset;
+    a.attn = mask;
+    a.out = output;
+    return launch_forward<false>(&p, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_dcn_backward(const msda_dcn_problem *problem, const void *input, const float *offset,
+                              const float *mask, const void *grad_output, void *grad_input,
+                              float *grad_offset, float *grad_mask, void *workspace,
+                              size_t workspace_bytes, msda_stream_t stream)
+{
+    msda_problem p;
+    int64_t ho = 0, wo = 0;
+    msda_status st = dcn_to_problem(problem, p, ho, wo);
+    if (st != MSDA_OK)
+        return st;
+    const Sizes z = sizes_of(&p);
+    if (!vec_ptr_ok(input, z.value) || !ptr_ok(offset, z.samples * 2) || !ptr_ok(mask, z.samples) ||
+        !ptr_ok(grad_output, z.rows_d) || !ptr_ok(grad_input, z.value) ||
+        !ptr_ok(grad_offset, z.samples * 2) || !ptr_ok(grad_mask, z.samples))
+        return MSDA_ERR_INVALID_ARG;
+    KernelArgs a = base_args(&p, input, nullptr, nullptr);
+    dcn_args(problem, wo, a);
+    a.loc = offset;
+    a.attn = mask;
+    a.grad_out = grad_output;
+    a.grad_loc = grad_offset;
+    a.grad_attn = grad_mask;
+    return run_backward<false>(&p, a, grad_input, workspace, workspace_bytes,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_dcn_backward_workspace_size(const msda_dcn_problem *problem, size_t *bytes)
+{
+    msda_problem p;
+    int64_t ho = 0, wo = 0;
+    msda_status st = dcn_to_problem(problem, p, ho, wo);
+    if (st != MSDA_OK)
+        return st;
+    return msda_backward_workspace_size(&p, bytes);
+}
 
 msda_status msda_forward(const msda_problem *problem, const void *value,
                          const int64_t *spatial_shapes, const int64_t *level_start_index,

@@ -131,6 +131,13 @@ struct KernelArgs {
     int withhold_copy;      // testing: arm the input copies but never issue them
     const int32_t *order;   // optional processing order of the B*Q queries
     const float *scale;     // INT8 value: dequantization scale per (batch, head)
+    // DCNv3 core (non-fused kernels): levels are the kh kernel rows, points
+    // the kw kernel columns, all on the one H x W map; the pixel coordinate
+    // of sample (l, k) of output pixel q = (i, j) is the convolution grid
+    // point plus the offset, and the offset gradient is not rescaled
+    int dcn;
+    int dcn_h, dcn_w, dcn_wo;
+    int stride_h, stride_w, pad_h, pad_w, dil_h, dil_w;
 };
 
 struct Geometry {
@@ -145,6 +152,15 @@ struct Geometry {
 // it in the device status word.
 __device__ __forceinline__ bool load_geometry(const KernelArgs &a, Geometry &geo, int &ok)
 {
+    if (a.dcn) {  // every kernel row samples the one input map (host-checked sizes)
+        if (threadIdx.x < a.L) {
+            geo.H[threadIdx.x] = a.dcn_h;
+            geo.W[threadIdx.x] = a.dcn_w;
+            geo.start[threadIdx.x] = 0;
+        }
+        __syncthreads();
+        return true;
+    }
     if (threadIdx.x == 0) {
         int good = 1;
         int64_t run = 0;
@@ -509,6 +525,20 @@ __device__ __forceinline__ void pixel_from_offset(float rx, float ry, float ox, 
     y = __dsub_rn(__dmul_rn(ly, (double)H), 0.5);
 }
 
+// DCNv3: sample s = r * kw + c of memory row `row` (= (b * Q + q) * G + g,
+// q = i * Wo + j) sits at the convolution grid point plus its offset,
+//   x = (j * stride_w - pad_w + c * dil_w) + dx,  y = (i * stride_h - pad_h + r * dil_h) + dy,
+// the integer part exact and one float64 addition.
+__device__ __forceinline__ void pixel_from_dcn(const KernelArgs &a, int64_t row, int s, float dx, float dy,
+                                               double &x, double &y)
+{
+    const int64_t q = (row / a.M) % a.Q;
+    const int64_t i = q / a.dcn_wo, j = q - i * a.dcn_wo;
+    const int r = s / a.K, c = s - r * a.K;
+    x = __dadd_rn((double)(j * a.stride_w - a.pad_w + (int64_t)c * a.dil_w), (double)dx);
+    y = __dadd_rn((double)(i * a.stride_h - a.pad_h + (int64_t)r * a.dil_h), (double)dy);
+}
+
 // Corner geometry of one sample at pixel coordinate (x, y) of a level.
 struct Corners {
     bool valid;          // -1 < x < W and -1 < y < H
@@ -590,7 +620,10 @@ __device__ __forceinline__ void sample_input(const KernelArgs &a, int64_t base, 
         A = expf(ld_stream(a.logits + base + s, pol) - mx) * inv_sum;
     } else {
         const float2 p = ld_stream2(reinterpret_cast<const float2 *>(a.loc) + base + s, pol);
-        pixel_from_location(p.x, p.y, H, W, x, y);
+        if (a.dcn)
+            pixel_from_dcn(a, base / (a.L * a.K), s, p.x, p.y, x, y);
+        else
+            pixel_from_location(p.x, p.y, H, W, x, y);
         A = ld_stream(a.attn + base + s, pol);
     }
 }
@@ -881,8 +914,8 @@ __device__ __forceinline__ WarpIn warp_load_staged(const KernelArgs &a, const fl
 // must call (the softmax shuffles).
 template <bool FUSED>
 __device__ __forceinline__ void warp_sample(const KernelArgs &a, const Geometry &geo, const WarpIn &in,
-                                            bool active, int s, int P, int &l, double &x, double &y,
-                                            float &A)
+                                            bool active, int64_t row, int s, int P, int &l, double &x,
+                                            double &y, float &A)
 {
     l = s / a.K;
     const int H = geo.H[l], W = geo.W[l];
@@ -894,7 +927,10 @@ __device__ __forceinline__ void warp_sample(const KernelArgs &a, const Geometry 
         pixel_from_offset(in.r.x, in.r.y, in.p.x, in.p.y, H, W, x, y);
     } else {
         A = in.z;
-        pixel_from_location(in.p.x, in.p.y, H, W, x, y);
+        if (a.dcn)
+            pixel_from_dcn(a, row, s, in.p.x, in.p.y, x, y);
+        else
+            pixel_from_location(in.p.x, in.p.y, H, W, x, y);
     }
 }
 
@@ -930,7 +966,8 @@ __device__ __forceinline__ void setup_backward_warp(const KernelArgs &a, const G
             int l;
             double x, y;
             float A;
-            warp_sample<FUSED>(a, geo, in[t], active, s, P, l, x, y, A);
+            const int64_t row = (a.dcn && active) ? memory_row(a, prow) : 0;  // DCN grid point
+            warp_sample<FUSED>(a, geo, in[t], active, row, s, P, l, x, y, A);
             if (rr >= nrows)
                 continue;
             const int k = rr * stride + s;
@@ -976,7 +1013,7 @@ __device__ __forceinline__ void setup_forward_staged(const KernelArgs &a, const 
         int l;
         double x, y;
         float A;
-        warp_sample<FUSED>(a, geo, in, active, s, P, l, x, y, A);
+        warp_sample<FUSED>(a, geo, in, active, row, s, P, l, x, y, A);
         if (!active)
             continue;
         if (FUSED && a.attn_out)
@@ -1395,8 +1432,10 @@ backward_kernel(const KernelArgs a)
                     ref_gx += W * part[0][1];
                     ref_gy += H * part[0][2];
                 } else {
+                    // DCN offsets are in pixels: no normalized-unit factor
+                    const float sx = a.dcn ? 1.f : W, sy = a.dcn ? 1.f : H;
                     st_stream2(reinterpret_cast<float2 *>(a.grad_loc) + base + s,
-                               make_float2(W * part[0][1], H * part[0][2]), pol);
+                               make_float2(sx * part[0][1], sy * part[0][2]), pol);
                     st_stream(a.grad_attn + base + s, part[0][0], pol);
                 }
             }

@@ -270,3 +270,100 @@ def generate(w: Workload, with_nonfused: bool = True) -> Inputs:
         sampling_locations=np.ascontiguousarray(loc, dtype=np.float32),
         attention_weights=np.ascontiguousarray(wts, dtype=np.float32),
     )
+
+
+# ----------------------------------------------------------- DCNv3 core ----
+#
+# Stand-ins for InternImage's DCNv3 layers (discosf.com/news/5175395 §4.2 gives
+# the operator and mentions 7x7 and larger kernels, but no layer sizes): a
+# classification stage-1 layer at 224^2 input (56 x 56, 64 channels in 4
+# groups), a detection stage-2 layer at 800 x 1333 (100 x 167, 128 channels in
+# 8 groups) and a 7 x 7 large-kernel layer.  Offsets are N(0, sigma) pixels,
+# masks a flat Dirichlet draw over the K points of each (n, i, j, g).
+
+@dataclasses.dataclass(frozen=True)
+class DcnWorkload:
+    name: str
+    index: int               # seed = 0x5EED0000 + index
+    N: int
+    H: int
+    W: int
+    G: int
+    C: int
+    kernel: Tuple[int, int]
+    stride: Tuple[int, int]
+    pad: Tuple[int, int]
+    dil: Tuple[int, int]
+    dtype: str               # "f32", "bf16" or "s8" (as Workload.dtype)
+    offset_sigma: float
+
+    @property
+    def seed(self) -> int:
+        return 0x5EED0000 + self.index
+
+    @property
+    def K(self) -> int:
+        return self.kernel[0] * self.kernel[1]
+
+    @property
+    def out_hw(self) -> Tuple[int, int]:
+        kh, kw = self.kernel
+        return ((self.H + 2 * self.pad[0] - self.dil[0] * (kh - 1) - 1) // self.stride[0] + 1,
+                (self.W + 2 * self.pad[1] - self.dil[1] * (kw - 1) - 1) // self.stride[1] + 1)
+
+    @property
+    def samples(self) -> int:
+        Ho, Wo = self.out_hw
+        return self.N * Ho * Wo * self.G * self.K
+
+
+DCN_WORKLOADS: Dict[str, DcnWorkload] = {
+    w.name: w
+    for w in [
+        DcnWorkload("dcnv3_stage1_f32", 10, 32, 56, 56, 4, 16, (3, 3), (1, 1), (1, 1), (1, 1),
+                    "f32", 1.0),
+        DcnWorkload("dcnv3_det_stage2_bf16", 11, 2, 100, 167, 8, 16, (3, 3), (1, 1), (1, 1), (1, 1),
+                    "bf16", 1.0),
+        DcnWorkload("dcnv3_k7_bf16", 12, 2, 50, 84, 16, 16, (7, 7), (1, 1), (3, 3), (1, 1),
+                    "bf16", 2.0),
+    ]
+}
+
+TAG_DCN_MASK = 8
+
+
+@dataclasses.dataclass
+class DcnInputs:
+    workload: DcnWorkload
+    input: np.ndarray        # [N, H, W, G, C] float32, or bf16 bits (uint16) for bf16 / s8
+    offset: np.ndarray       # [N, Ho, Wo, G, K, 2] float32 (dx, dy) pixels
+    mask: np.ndarray         # [N, Ho, Wo, G, K] float32
+    grad_output: np.ndarray  # [N, Ho, Wo, G, C] float32 or bf16 bits
+
+    def input_f64(self) -> np.ndarray:
+        return _widen(self.input)
+
+    def grad_output_f64(self) -> np.ndarray:
+        return _widen(self.grad_output)
+
+
+def generate_dcn(w: DcnWorkload) -> DcnInputs:
+    N, H, W, G, C, K = w.N, w.H, w.W, w.G, w.C, w.K
+    Ho, Wo = w.out_hw
+    x = normal(w.seed, TAG_VALUE, N * H * W * G * C).reshape(N, H, W, G, C)
+    off = (w.offset_sigma * normal(w.seed, TAG_OFFSETS, N * Ho * Wo * G * K * 2)
+           ).reshape(N, Ho, Wo, G, K, 2)
+    e = -np.log(1.0 - uniform(w.seed, TAG_DCN_MASK, N * Ho * Wo * G * K)).reshape(N, Ho, Wo, G, K)
+    e = np.maximum(e, 1e-30)
+    mask = e / e.sum(-1, keepdims=True)
+    gy = normal(w.seed, TAG_GRAD_OUT, N * Ho * Wo * G * C).reshape(N, Ho, Wo, G, C)
+    return DcnInputs(w, _store(x, w.dtype), off.astype(np.float32), mask.astype(np.float32),
+                     _store(gy, w.dtype))
+
+
+def custom_dcn(name: str, N: int, H: int, W: int, G: int, C: int, kernel, stride=(1, 1),
+               pad=(1, 1), dil=(1, 1), dtype: str = "f32", offset_sigma: float = 1.0,
+               index: int = 700) -> DcnWorkload:
+    """A small ad-hoc DCNv3 workload (tests)."""
+    return DcnWorkload(name, index, N, H, W, G, C, tuple(kernel), tuple(stride), tuple(pad),
+                       tuple(dil), dtype, offset_sigma)

@@ -142,3 +142,42 @@ def test_int8_checks(lib):
         _lib.MSDA_ERR_INVALID_ARG
     assert lib.msda_quantize_value_s8(ctypes.byref(f32), FAKE, FAKE, None, None) == \
         _lib.MSDA_ERR_INVALID_ARG
+
+
+def test_dcn_checks(lib):
+    """msda_dcn_*: output size of the convolution grid, parameter checks and
+    pointer checks before anything is enqueued."""
+    def prob(**kw):
+        d = dict(batch=2, height=56, width=56, groups=4, group_channels=16, kernel_h=3, kernel_w=3,
+                 stride_h=1, stride_w=1, pad_h=1, pad_w=1, dilation_h=1, dilation_w=1,
+                 value_dtype=_lib.MSDA_F32, flags=0)
+        d.update(kw)
+        return _lib.DcnProblem(**d)
+
+    ho, wo = ctypes.c_int64(0), ctypes.c_int64(0)
+
+    def size(p):
+        st = lib.msda_dcn_output_size(ctypes.byref(p), ctypes.byref(ho), ctypes.byref(wo))
+        return st, ho.value, wo.value
+
+    assert size(prob()) == (0, 56, 56)
+    assert size(prob(kernel_h=7, kernel_w=7, stride_h=2, stride_w=2, pad_h=3, pad_w=3)) == (0, 28, 28)
+    assert size(prob(kernel_h=5, dilation_h=2, pad_h=0, height=9))[:2] == (0, 1)
+    assert size(prob(kernel_h=5, dilation_h=3, pad_h=0, height=9))[:2] == (0, 0)  # nothing to sample
+    assert size(prob(stride_w=0))[0] == _lib.MSDA_ERR_INVALID_ARG
+    assert size(prob(pad_h=-1))[0] == _lib.MSDA_ERR_INVALID_ARG
+    assert size(prob(kernel_w=33, pad_w=16))[0] == _lib.MSDA_ERR_UNSUPPORTED
+    assert size(prob(kernel_h=17, pad_h=8))[0] == _lib.MSDA_ERR_UNSUPPORTED
+    assert size(prob(group_channels=24))[0] == _lib.MSDA_ERR_UNSUPPORTED
+    assert size(prob(value_dtype=_lib.MSDA_S8))[0] == _lib.MSDA_ERR_INVALID_ARG  # no value_scale
+    p = prob()
+    assert lib.msda_dcn_forward(ctypes.byref(p), MISALIGNED, FAKE, FAKE, FAKE, None) == \
+        _lib.MSDA_ERR_INVALID_ARG
+    assert lib.msda_dcn_forward(ctypes.byref(p), FAKE, FAKE, None, FAKE, None) == \
+        _lib.MSDA_ERR_INVALID_ARG
+    n = ctypes.c_size_t(0)
+    pb = prob(flags=_lib.MSDA_GRAD_VALUE_BF16)
+    assert lib.msda_dcn_backward_workspace_size(ctypes.byref(pb), ctypes.byref(n)) == 0
+    assert n.value == 2 * 56 * 56 * 4 * 16 * 4
+    assert lib.msda_dcn_backward(ctypes.byref(pb), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 16, None) == _lib.MSDA_ERR_INVALID_ARG
