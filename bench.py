@@ -20,6 +20,7 @@ no data-path collective).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import glob
 import hashlib
@@ -69,7 +70,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="detr_encoder_f32", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default="detr_encoder_f32",
+                    choices=sorted(wl.WORKLOADS) + sorted(wl.DCN_WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="host-core seconds spent timing the oracle for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -753,11 +755,278 @@ def run_reference(args):
     return result
 
 
+# ------------------------------------------------------------ DCNv3 core --
+
+def dcn_algorithmic_bytes(w: wl.DcnWorkload) -> dict:
+    Ho, Wo = w.out_hw
+    e = {"f32": 4, "bf16": 2, "s8": 1}[w.dtype]
+    er = {"f32": 4, "bf16": 2, "s8": 2}[w.dtype]
+    x = w.N * w.H * w.W * w.G * w.C
+    rows = w.N * Ho * Wo * w.G * w.C
+    off, mask = w.samples * 8, w.samples * 4
+    fwd = x * e + off + mask + rows * er
+    bwd = rows * er + x * e + off + mask + x * 4 + off + mask
+    return {"dcn_forward": fwd, "dcn_backward": bwd, "quantize": x * 3 if w.dtype == "s8" else 0}
+
+
+def _dcn_to_device(x: wl.DcnInputs, dev):
+    import torch
+
+    def val(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    return {"input": val(x.input), "offset": torch.from_numpy(x.offset).to(dev),
+            "mask": torch.from_numpy(x.mask).to(dev), "grad_output": val(x.grad_output)}
+
+
+def _dcn_band(w: wl.DcnWorkload, x: wl.DcnInputs, max_samples: int):
+    """A bounded sample of the workload: the top band of input rows of image 0,
+    with the offsets, masks and output gradients of the output rows it
+    yields (the same layer on a shorter map)."""
+    import oracle
+    Ho, Wo = w.out_hw
+    per_row = Wo * w.G * w.K
+    rows_out = max(1, min(Ho, max_samples // per_row))
+    hb = min(w.H, rows_out * w.stride[0])
+    hob, _ = oracle.dcn_output_size(hb, w.W, w.kernel, w.stride, w.pad, w.dil)
+    hob = max(0, min(hob, Ho))
+    return dict(x=x.input_f64()[0:1, :hb], off=x.offset[0:1, :hob], mask=x.mask[0:1, :hob],
+                gy=x.grad_output_f64()[0:1, :hob], samples=hob * per_row, rows=hb)
+
+
+def _dcn_oracle_pass(w: wl.DcnWorkload, band) -> None:
+    import oracle
+    og = dict(kernel=w.kernel, stride=w.stride, pad=w.pad, dil=w.dil)
+    oracle.dcn_forward(band["x"], band["off"], band["mask"], **og)
+    oracle.dcn_backward(band["x"], band["off"], band["mask"], band["gy"], **og)
+
+
+def _dcn_oracle_cpu(w: wl.DcnWorkload, x: wl.DcnInputs, seconds: float):
+    """The oracle's DCNv3 core (fp64 C loops, one thread), forward + backward
+    on a band of image 0 of about 2^18 samples, repeated for `seconds`.
+    Returns (G samples/s, sample text)."""
+    import oracle
+    oracle.build()
+    band = _dcn_band(w, x, 1 << 18)
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        _dcn_oracle_pass(w, band)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    text = (f"input rows 0..{band['rows'] - 1} of image 0 of {w.N} ({band['samples']} samples) "
+            f"x {passes} passes, {el:.1f} s")
+    return band["samples"] * passes / el / 1e9, text
+
+
+def run_dcn(args):
+    """The DCNv3 core step: msda_dcn_forward || zero-fill -> msda_dcn_backward
+    (INT8 input: msda_quantize_value_s8 first), same timing rules as the
+    attention step."""
+    import torch
+    import torch.distributed as dist
+    import scale_deformable_attention_msdeformattn_b200 as msda
+
+    world, rank, local = _dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    base = wl.DCN_WORKLOADS[args.workload]
+    w = dataclasses.replace(base, index=base.index + 1000 * rank) if rank else base
+    x = wl.generate_dcn(w)
+    t = _dcn_to_device(x, dev)
+    N, H, W, G, C = w.N, w.H, w.W, w.G, w.C
+    Ho, Wo = w.out_hw
+    geo = dict(kernel=w.kernel, stride=w.stride, pad=w.pad, dilation=w.dil)
+    int8 = w.dtype == "s8"
+    q = torch.empty((N, H, W, G, C), dtype=torch.int8, device=dev) if int8 else None
+    qs = torch.empty((N, G), dtype=torch.float32, device=dev) if int8 else None
+    out = torch.empty((N, Ho, Wo, G, C), dtype=t["grad_output"].dtype, device=dev)
+    gx = torch.empty((N, H, W, G, C), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream(device=dev)
+
+    def step(ev, tin=None):
+        tin = tin or t
+        ev[0].record(stream)
+        inp = tin["input"]
+        if int8:
+            msda.quantize_value_s8(inp.flatten(1, 2), value_s8=q.flatten(1, 2), value_scale=qs)
+            inp = q
+        ev[4].record(stream)
+        side.wait_event(ev[4])
+        with torch.cuda.stream(side):
+            msda.zero_grads(gx.flatten(1, 2))
+            ev[5].record(side)
+        msda.dcn_forward(inp, tin["offset"], tin["mask"], out=out, value_scale=qs, **geo)
+        ev[1].record(stream)
+        stream.wait_event(ev[5])
+        ev[2].record(stream)
+        res = msda.dcn_backward(inp, tin["offset"], tin["mask"], tin["grad_output"], grad_input=gx,
+                                accumulate=True, value_scale=qs, **geo)
+        ev[3].record(stream)
+        return {"out": out, "grad_input": res[0], "grad_offset": res[1], "grad_mask": res[2]}
+
+    def events(n):
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n)]
+
+    warm = events(args.warmup)
+    for i in range(args.warmup):
+        flush.fill_(float(i))
+        step(warm[i])
+    torch.cuda.synchronize()
+    if msda.device_status() != 0:
+        raise SystemExit("kernels reported a device check")
+    evs = events(args.steps)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    stepms = [e[0].elapsed_time(e[3]) for e in evs]
+    total_ms, value = aggregate_over_ranks(float(sum(stepms)), w.samples, args.steps, world, dev)
+    result = None
+    if rank == 0:
+        peaks = _peaks()
+        nb = dcn_algorithmic_bytes(w)
+        fwd_ms = statistics.mean(e[4].elapsed_time(e[1]) for e in evs)
+        bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+        dom, dom_ms = ("dcn_backward", bwd_ms) if bwd_ms >= fwd_ms else ("dcn_forward", fwd_ms)
+        achieved = nb[dom] / (dom_ms * 1e-3) / 1e9
+        ms_per_step = total_ms / args.steps
+        result = {
+            "metric": METRIC + " (DCNv3 core workload)", "value": round(value, 4), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": {"f32": "f32", "bf16": "bf16 input / f32 accumulate",
+                      "s8": "int8 input (per image-group scale) / bf16 rows / f32 accumulate"}[w.dtype],
+            "data": "synthetic: seeded SplitMix64 + Box-Muller draws (no dataset)",
+            "config": {"workload": w.name, "N": N, "H": H, "W": W, "G": G, "C": C,
+                       "kernel": list(w.kernel), "stride": list(w.stride), "pad": list(w.pad),
+                       "dilation": list(w.dil), "offset_sigma_px": w.offset_sigma,
+                       "samples_per_step_per_gpu": w.samples,
+                       "step": ("msda_quantize_value_s8 -> " if int8 else "")
+                       + "msda_dcn_forward || msda_zero_grads (second stream) -> msda_dcn_backward",
+                       "l2": "flushed between steps (256 MiB write outside the timed events)",
+                       "parallelism": f"dp{world} (independent batch per GPU)"},
+            "fwd_ms": round(fwd_ms, 5), "bwd_ms": round(bwd_ms, 5),
+            "step_ms_p10_p50_p90": [round(float(np.percentile(stepms, p)), 5) for p in (10, 50, 90)],
+            "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                         "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4),
+                         "bytes_per_launch": nb[dom], "traffic": None},
+            "gpu_launches": (3 + (3 if int8 else 0)) * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if not args.no_e2e and world == 1:
+            hin = {k: v.cpu().pin_memory() for k, v in t.items()}
+            din = {k: torch.empty_like(v) for k, v in t.items()}
+            hout = {"out": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                    "grad_input": torch.empty(gx.shape, dtype=torch.float32).pin_memory(),
+                    "grad_offset": torch.empty(t["offset"].shape).pin_memory(),
+                    "grad_mask": torch.empty(t["mask"].shape).pin_memory()}
+            times = []
+            for i in range(min(args.steps, 50) + 2):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                flush.fill_(float(i))
+                e0.record(stream)
+                for k in hin:
+                    din[k].copy_(hin[k], non_blocking=True)
+                outs = step(events(1)[0], din)
+                for k in hout:
+                    hout[k].copy_(outs[k], non_blocking=True)
+                e1.record(stream)
+                if i >= 2:
+                    times.append((e0, e1))
+            torch.cuda.synchronize()
+            ms = statistics.mean(a.elapsed_time(b) for a, b in times)
+            result["e2e"] = {"value": round(w.samples / (ms * 1e-3) / 1e9, 4), "unit": UNIT,
+                             "ms_per_step": round(ms, 4),
+                             "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for v in hin.values())),
+                             "d2h_bytes_per_step": int(sum(v.numel() * v.element_size() for v in hout.values())),
+                             "steps": len(times)}
+        if world == 1 and not args.no_cpu_baseline:
+            rate, sample = _dcn_oracle_cpu(w, x, args.cpu_seconds)
+            result["cpu_baseline"] = {"value": round(rate, 6), "unit": UNIT, "cores": 1,
+                                      "kind": "oracle", "sample": sample}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        line = json.dumps(result)
+        print(line, flush=True)
+        if args.out:
+            with open(args.out, "a") as f:
+                f.write(line + "\n")
+    return result
+
+
+def run_dcn_reference(args):
+    """Reference arm for a DCNv3 workload: the oracle's DCNv3 core on a band of
+    image 0 per step, sized so that warm-up + steps end in about two minutes
+    (rank 0 only)."""
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    w = wl.DCN_WORKLOADS[args.workload]
+    x = wl.generate_dcn(w)
+    probe = _dcn_band(w, x, 1 << 14)
+    t0 = time.perf_counter()
+    _dcn_oracle_pass(w, probe)
+    per_sample = (time.perf_counter() - t0) / max(1, probe["samples"])
+    budget = 120.0 / (args.steps + args.warmup)
+    band = _dcn_band(w, x, int(max(1, budget / per_sample)))
+    for _ in range(args.warmup):
+        _dcn_oracle_pass(w, band)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _dcn_oracle_pass(w, band)
+    el = time.perf_counter() - t0
+    value = band["samples"] * args.steps / el / 1e9
+    sample = f"input rows 0..{band['rows'] - 1} of image 0 ({band['samples']} samples) per step"
+    result = {"impl": "reference", "metric": METRIC + " (DCNv3 core workload)", "value": round(value, 6),
+              "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+              "ms_per_step": round(w.samples / (value * 1e9) * 1e3, 3), "higher_is_better": True,
+              "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+              "data": "synthetic: seeded SplitMix64 + Box-Muller draws (no dataset)",
+              "config": {"workload": w.name, "step": "oracle dcn_forward + dcn_backward (fp64 C loops)",
+                         "parallelism": "one host thread"},
+              "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+                               "sample": sample},
+              "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                      "d2h_bytes_per_step": 0}}
+    line = json.dumps(result)
+    print(line, flush=True)
+    if args.out:
+        with open(args.out, "a") as f:
+            f.write(line + "\n")
+    return result
+
+
 def main(argv=None):
     args = parse_args(argv)
+    dcn = args.workload in wl.DCN_WORKLOADS
     if args.impl == "reference":
-        return run_reference(args)
-    return run_ours(args)
+        return run_dcn_reference(args) if dcn else run_reference(args)
+    return run_dcn(args) if dcn else run_ours(args)
 
 
 if __name__ == "__main__":
