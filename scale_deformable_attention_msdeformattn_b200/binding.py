@@ -382,7 +382,9 @@ def dcn_forward(input: torch.Tensor, offset: torch.Tensor, mask: torch.Tensor, k
 
 def dcn_backward(input, offset, mask, grad_output, kernel=3, stride=1, pad=1, dilation=1,
                  grad_input_dtype=torch.float32, grad_input: Optional[torch.Tensor] = None,
-                 accumulate: bool = False, value_scale: Optional[torch.Tensor] = None):
+                 accumulate: bool = False, value_scale: Optional[torch.Tensor] = None,
+                 grad_offset: Optional[torch.Tensor] = None,
+                 grad_mask: Optional[torch.Tensor] = None):
     """msda_dcn_backward: (grad_input, grad_offset, grad_mask)."""
     _need(input, "input", None)
     if grad_input_dtype not in (torch.float32, torch.bfloat16):
@@ -402,8 +404,10 @@ def dcn_backward(input, offset, mask, grad_output, kernel=3, stride=1, pad=1, di
     if grad_input is None:
         grad_input = torch.empty((N, H, W, G, C), dtype=grad_input_dtype, device=dev)
     _need(grad_input, "grad_input", grad_input_dtype, (N, H, W, G, C), dev)
-    goff = torch.empty_like(offset)
-    gmask = torch.empty_like(mask)
+    goff = grad_offset if grad_offset is not None else torch.empty_like(offset)
+    gmask = grad_mask if grad_mask is not None else torch.empty_like(mask)
+    _need(goff, "grad_offset", torch.float32, tuple(offset.shape), dev)
+    _need(gmask, "grad_mask", torch.float32, tuple(mask.shape), dev)
     lib = _lib.load()
     ws_bytes = ctypes.c_size_t(0)
     _check(lib.msda_dcn_backward_workspace_size(ctypes.byref(prob), ctypes.byref(ws_bytes)),
