@@ -240,12 +240,16 @@ msda_status launch_to_bf16(const float *src, void *dst, int64_t n, cudaStream_t 
 
 // Kernel selection -----------------------------------------------------------
 
+// The general kernels (query order, DCN grid) are separate instantiations, so
+// that the plain attention kernels carry none of their branches.
 template <bool FUSED>
 msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 {
+    const bool gen = a.order != nullptr || a.dcn != 0;
 #define MSDA_FWD_CASE(T, DD)                                                                      \
     case DD:                                                                                       \
-        return launch_rows((const void *)msda::forward_kernel<T, DD, FUSED>,                     \
+        return launch_rows(gen ? (const void *)msda::forward_kernel<T, DD, FUSED, true>          \
+                               : (const void *)msda::forward_kernel<T, DD, FUSED, false>,        \
                            msda::forward_rows_per_warp<T, DD>(),                                 \
                            kForwardRecordBytes, a.L * a.K, msda::forward_stages<T>(), a, s);
     if (p->value_dtype == MSDA_F32) {
@@ -272,9 +276,11 @@ msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 template <bool FUSED>
 msda_status launch_backward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 {
+    const bool gen = a.order != nullptr || a.dcn != 0;
 #define MSDA_BWD_CASE(T, DD)                                                                       \
     case DD:                                                                                        \
-        return launch_rows((const void *)msda::backward_kernel<T, DD, FUSED>,                    \
+        return launch_rows(gen ? (const void *)msda::backward_kernel<T, DD, FUSED, true>         \
+                               : (const void *)msda::backward_kernel<T, DD, FUSED, false>,       \
                            msda::backward_rows_per_warp<T, DD>(),                                \
                            FUSED ? kFusedBackwardRecordBytes : kBackwardRecordBytes,             \
                            msda::backward_padded_samples<T, DD>(a.L * a.K), msda::backward_stages(), \

@@ -1051,10 +1051,18 @@ template <> struct FwdTune<S8> {
     static constexpr bool kStage = false;
 };
 
-template <typename T, int D, bool FUSED>
+// GEN = false: the plain attention kernel (natural query order, no DCN grid),
+// with those branches removed at compile time; GEN = true honours
+// KernelArgs::order and KernelArgs::dcn.
+template <typename T, int D, bool FUSED, bool GEN>
 __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, FwdTune<T>::kMinCtas)
-forward_kernel(const KernelArgs a)
+forward_kernel(const KernelArgs a_in)
 {
+    KernelArgs a = a_in;
+    if constexpr (!GEN) {
+        a.order = nullptr;
+        a.dcn = 0;
+    }
     using Lay = Layout<T, D, FwdTune<T>::kVB>;
     using Raw = typename Lay::Raw;
     constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Lay::kEpv;
@@ -1235,10 +1243,15 @@ __device__ __forceinline__ void reduce_scatter3(float (&v)[C][3], int gl)
 // Samples per backward reduce-scatter chunk for G lanes per row.
 template <int G> struct BwdChunk { static constexpr int kC = G < 4 ? G : 4; };
 
-template <typename T, int D, bool FUSED>
+template <typename T, int D, bool FUSED, bool GEN>
 __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, MSDA_BWD_MIN_CTAS)
-backward_kernel(const KernelArgs a)
+backward_kernel(const KernelArgs a_in)
 {
+    KernelArgs a = a_in;
+    if constexpr (!GEN) {
+        a.order = nullptr;
+        a.dcn = 0;
+    }
     using Lay = Layout<T, D, BwdVB<T>::kVB>;
     using R = typename RowOf<T>::type;  // grad_output element
     using Raw = typename Lay::Raw;
