@@ -300,6 +300,7 @@ def run_ours(args):
         # backward waits for both
         tin = tin or t
         o = o or outputs
+        stream = torch.cuda.current_stream()  # the capture stream under graph capture
         ev[0].record(stream)
         if order is not None:
             msda.sort_queries(tin["reference_points"], query_order=order)
@@ -431,6 +432,7 @@ def run_ours(args):
                                                 qv if int8 else t["value"], qs)
         if world == 1:
             result["warm_l2"] = _time_warm(w, step, min(args.steps, 50))
+            result["graph"] = _time_graph(w.samples, step, flush, min(args.steps, 100), 7)
         stats = _input_stats(w, x)
         if "value_bytes_touched" in stats:
             # the value tensor counted by the sectors the gathers touch instead of whole
@@ -501,6 +503,39 @@ def _time_nonfused(msda, t, w, nbytes, flush, n, value, value_scale=None):
             "fwd_hbm_frac": round(nbytes["forward"] / (fwd * 1e-3) / 1e9 / peak, 4),
             "bwd_hbm_frac": round(nbytes["backward"] / (bwd * 1e-3) / 1e9 / peak, 4),
             "fwd_gsamples_per_s": round(w.samples / (fwd * 1e-3) / 1e9, 4), "launches": n}
+
+
+def _time_graph(samples, step, flush, n, nev):
+    """The step captured once into a CUDA graph (its two streams included) and
+    replayed n times, L2 flushed before each replay outside the graph; events
+    around each replay.  Removes the host's launch cost from the step."""
+    import torch
+    stream = torch.cuda.current_stream()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        step([torch.cuda.Event() for _ in range(nev)])  # once more on the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=cap):
+            step([torch.cuda.Event() for _ in range(nev)])
+    stream.wait_stream(cap)
+    for i in range(3):
+        flush.fill_(float(i))
+        g.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i, (a, b) in enumerate(evs):
+        flush.fill_(float(i))
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    med = float(np.median(ms))
+    del g
+    return {"ms_per_step_median": round(med, 5), "ms_per_step_mean": round(float(np.mean(ms)), 5),
+            "value": round(samples / (float(np.mean(ms)) * 1e-3) / 1e9, 4), "unit": UNIT, "steps": n,
+            "l2": "flushed before each replay"}
 
 
 def _time_warm(w, step, n):
@@ -886,6 +921,7 @@ def run_dcn(args):
     def step(ev, tin=None, o=None):
         tin = tin or t
         o = o or outputs
+        stream = torch.cuda.current_stream()
         ev[0].record(stream)
         inp = tin["input"]
         if int8:
@@ -965,6 +1001,8 @@ def run_dcn(args):
             "gpu_launches": (3 + (3 if int8 else 0)) * args.steps,
             "clocks": clocks.summary(),
         }
+        if world == 1:
+            result["graph"] = _time_graph(w.samples, step, flush, min(args.steps, 100), 6)
         if not args.no_e2e and world == 1:
             hin = {k: v.cpu().pin_memory() for k, v in t.items()}
             result["e2e"] = _time_e2e(hin, step, make_outputs, flush, min(args.steps, 50), w.samples,
