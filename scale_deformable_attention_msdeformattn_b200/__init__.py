@@ -10,8 +10,10 @@ from .binding import (  # noqa: F401
     MSDeformAttnFusedFunction,
     backward,
     backward_noalloc,
+    DCNv3CoreFunction,
     dcn_backward,
     dcn_forward,
+    dcnv3_core,
     device_status,
     forward,
     fused_backward,

@@ -510,3 +510,27 @@ def ms_deform_attn(value, spatial_shapes, level_start_index, sampling_locations,
     out = MSDeformAttnFunction.apply(value, spatial_shapes, level_start_index, sampling_locations,
                                      attention_weights)
     return out.flatten(2)
+
+
+class DCNv3CoreFunction(torch.autograd.Function):
+    """Autograd wrapper over msda_dcn_forward / msda_dcn_backward (float32 or
+    bfloat16 input; grad_input in the input's dtype)."""
+
+    @staticmethod
+    def forward(ctx, input, offset, mask, kernel=3, stride=1, pad=1, dilation=1):
+        ctx.save_for_backward(input, offset, mask)
+        ctx.geo = dict(kernel=kernel, stride=stride, pad=pad, dilation=dilation)
+        return dcn_forward(input, offset, mask, **ctx.geo)
+
+    @staticmethod
+    def backward(ctx, grad_output):
+        input, offset, mask = ctx.saved_tensors
+        gx, goff, gm = dcn_backward(input, offset, mask, grad_output.contiguous(),
+                                    grad_input_dtype=input.dtype, **ctx.geo)
+        return gx, goff, gm, None, None, None, None
+
+
+def dcnv3_core(input, offset, mask, kernel=3, stride=1, pad=1, dilation=1):
+    """Differentiable DCNv3 core: [N, H, W, G, C] -> [N, Ho, Wo, G*C] (the
+    layout the group projection w_g consumes)."""
+    return DCNv3CoreFunction.apply(input, offset, mask, kernel, stride, pad, dilation).flatten(3)

@@ -110,3 +110,22 @@ def test_dcn_host_checks():
         msda.dcn_forward(x, off[:, :4], m, kernel=3, pad=1)
     y = msda.dcn_forward(x, off, m, kernel=3, pad=1)
     assert y.shape == (1, 5, 5, 2, 16) and not y.any()
+
+
+def test_dcn_autograd_wrapper():
+    w = wl.custom_dcn("dcn_autograd", 2, 9, 11, 2, 16, (3, 3), (1, 1), (1, 1), (1, 1), "f32", 1.0,
+                      index=790)
+    x = wl.generate_dcn(w)
+    t = _upload(x)
+    inp = t["input"].clone().requires_grad_(True)
+    off = t["offset"].clone().requires_grad_(True)
+    m = t["mask"].clone().requires_grad_(True)
+    y = msda.dcnv3_core(inp, off, m, kernel=3, stride=1, pad=1, dilation=1)
+    Ho, Wo = w.out_hw
+    assert y.shape == (2, Ho, Wo, 32)
+    (y * t["grad_output"].flatten(3)).sum().backward()
+    og = dict(kernel=w.kernel, stride=w.stride, pad=w.pad, dil=w.dil)
+    rgx, rgoff, rgm = oracle.dcn_backward(x.input_f64(), x.offset, x.mask, x.grad_output_f64(), **og)
+    assert_close(inp.grad, rgx, 1e-5, "autograd grad_input")
+    assert_close(off.grad, rgoff, 1e-5, "autograd grad_offset")
+    assert_close(m.grad, rgm, 1e-5, "autograd grad_mask")
