@@ -99,6 +99,15 @@ typedef enum msda_dtype {
 #define MSDA_ACCUMULATE_GRADS (1u << 1) /* backward adds into grad_value (and
                                           grad_reference_points) instead of
                                           zeroing them first; float32 only */
+#define MSDA_STAGE_INPUTS (1u << 2) /* forward: each warp copies its next rows'
+                                          set-up inputs into shared memory with
+                                          bulk copies (completion on an
+                                          mbarrier, bounded wait) while it
+                                          gathers the current rows, instead of
+                                          loading them directly; power-of-two
+                                          L*K <= 32, natural query order.  A
+                                          performance option (off by default:
+                                          slower with the default lane layout) */
 #define MSDA_TEST_WITHHOLD_COPY (1u << 31) /* testing only: kernels that stage
                                           their inputs with bulk copies arm
                                           the copy but never issue it, so

@@ -56,7 +56,8 @@ msda_status check_problem(const msda_problem *p)
     if (p->value_dtype == MSDA_S8 &&
         (!p->value_scale || (reinterpret_cast<uintptr_t>(p->value_scale) & 3u)))
         return MSDA_ERR_INVALID_ARG;
-    if (p->flags & ~(uint32_t)(MSDA_GRAD_VALUE_BF16 | MSDA_ACCUMULATE_GRADS | MSDA_TEST_WITHHOLD_COPY))
+    if (p->flags & ~(uint32_t)(MSDA_GRAD_VALUE_BF16 | MSDA_ACCUMULATE_GRADS | MSDA_STAGE_INPUTS |
+                               MSDA_TEST_WITHHOLD_COPY))
         return MSDA_ERR_INVALID_ARG;
     if ((p->flags & MSDA_GRAD_VALUE_BF16) && (p->flags & MSDA_ACCUMULATE_GRADS))
         return MSDA_ERR_INVALID_ARG;
@@ -245,13 +246,14 @@ msda_status launch_to_bf16(const float *src, void *dst, int64_t n, cudaStream_t 
 template <bool FUSED>
 msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 {
-    const bool gen = a.order != nullptr || a.dcn != 0;
+    const bool gen = a.order != nullptr || a.dcn != 0 || a.stage != 0;
 #define MSDA_FWD_CASE(T, DD)                                                                      \
     case DD:                                                                                       \
         return launch_rows(gen ? (const void *)msda::forward_kernel<T, DD, FUSED, true>          \
                                : (const void *)msda::forward_kernel<T, DD, FUSED, false>,        \
                            msda::forward_rows_per_warp<T, DD>(),                                 \
-                           kForwardRecordBytes, a.L * a.K, msda::forward_stages<T>(), a, s);
+                           kForwardRecordBytes, a.L * a.K,                                       \
+                           msda::forward_stages<T>() || (a.stage && !a.order), a, s);
     if (p->value_dtype == MSDA_F32) {
         switch (p->head_dim) {
             MSDA_FWD_CASE(float, 8) MSDA_FWD_CASE(float, 16) MSDA_FWD_CASE(float, 32)
@@ -276,7 +278,7 @@ msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 template <bool FUSED>
 msda_status launch_backward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 {
-    const bool gen = a.order != nullptr || a.dcn != 0;
+    const bool gen = a.order != nullptr || a.dcn != 0 || a.stage != 0;
 #define MSDA_BWD_CASE(T, DD)                                                                       \
     case DD:                                                                                        \
         return launch_rows(gen ? (const void *)msda::backward_kernel<T, DD, FUSED, true>         \
@@ -320,6 +322,7 @@ KernelArgs base_args(const msda_problem *p, const void *value, const int64_t *sh
     a.L = p->num_levels;
     a.K = p->num_points;
     a.withhold_copy = (p->flags & MSDA_TEST_WITHHOLD_COPY) ? 1 : 0;
+    a.stage = (p->flags & MSDA_STAGE_INPUTS) ? 1 : 0;
     a.order = (p->batch * p->num_queries > 0) ? p->query_order : nullptr;
     a.scale = p->value_dtype == MSDA_S8 ? p->value_scale : nullptr;
     return a;

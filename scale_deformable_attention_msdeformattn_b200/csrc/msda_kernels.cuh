@@ -41,20 +41,21 @@
 
 namespace msda {
 
-// Tuning knobs (compile-time).  The forward gathers float32 rows with 32-byte
-// lane vectors, one sample in flight per lane and 3 CTAs per SM, and bf16
+// Tuning knobs (compile-time).  The forward gathers float32 rows with 16-byte
+// lane vectors, one sample in flight per lane and 4 CTAs per SM, and bf16
 // rows with 16-byte vectors and four samples in flight; the backward uses
 // 16-byte vectors (whole-sector grad_value reductions, more rows per warp).
-// TMA staging of the set-up inputs pays off in the float32 forward only (the
-// others measured slower with it).
+// Bulk-copy staging of the set-up inputs measured slower everywhere with
+// these layouts; it stays available per call (MSDA_STAGE_INPUTS, general
+// kernels) and by these switches.
 #ifndef MSDA_FWD_VB_F32
-#define MSDA_FWD_VB_F32 32
+#define MSDA_FWD_VB_F32 16
 #endif
 #ifndef MSDA_FWD_INFLIGHT_F32
 #define MSDA_FWD_INFLIGHT_F32 1
 #endif
 #ifndef MSDA_FWD_MIN_CTAS_F32
-#define MSDA_FWD_MIN_CTAS_F32 3
+#define MSDA_FWD_MIN_CTAS_F32 4
 #endif
 #ifndef MSDA_FWD_VB_BF16
 #define MSDA_FWD_VB_BF16 16
@@ -66,7 +67,7 @@ namespace msda {
 #define MSDA_FWD_MIN_CTAS_BF16 2
 #endif
 #ifndef MSDA_FWD_STAGE_F32           // TMA-staged set-up inputs (see "input staging")
-#define MSDA_FWD_STAGE_F32 1
+#define MSDA_FWD_STAGE_F32 0
 #endif
 #ifndef MSDA_FWD_STAGE_BF16
 #define MSDA_FWD_STAGE_BF16 0
@@ -129,6 +130,7 @@ struct KernelArgs {
     int64_t S;
     int Q, M, L, K;
     int withhold_copy;      // testing: arm the input copies but never issue them
+    int stage;              // forward: stage set-up inputs by bulk copies (general kernels)
     const int32_t *order;   // optional processing order of the B*Q queries
     const float *scale;     // INT8 value: dequantization scale per (batch, head)
     // DCNv3 core (non-fused kernels): levels are the kh kernel rows, points
@@ -1062,6 +1064,7 @@ forward_kernel(const KernelArgs a_in)
     if constexpr (!GEN) {
         a.order = nullptr;
         a.dcn = 0;
+        a.stage = 0;
     }
     using Lay = Layout<T, D, FwdTune<T>::kVB>;
     using Raw = typename Lay::Raw;
@@ -1083,7 +1086,8 @@ forward_kernel(const KernelArgs a_in)
     int4 *off = reinterpret_cast<int4 *>(smem_raw) + a.rows_per_tile * stride + slot * stride;
     const uint64_t pol = stream_policy();
     constexpr int RPW = Lay::kRowsPerWarp;
-    const int cap = a.order ? 0 : stage_cap(FwdTune<T>::kStage, RPW, P);  // staged slices are contiguous rows
+    // staged slices are contiguous rows: not with a query order
+    const int cap = a.order ? 0 : stage_cap(FwdTune<T>::kStage || a.stage, RPW, P);
     const WarpStage ws = warp_stage(smem_raw + align16((size_t)a.rows_per_tile * stride * 32), warp,
                                     blockDim.x >> 5, cap);
     if (cap) {
@@ -1251,6 +1255,7 @@ backward_kernel(const KernelArgs a_in)
     if constexpr (!GEN) {
         a.order = nullptr;
         a.dcn = 0;
+        a.stage = 0;
     }
     using Lay = Layout<T, D, BwdVB<T>::kVB>;
     using R = typename RowOf<T>::type;  // grad_output element

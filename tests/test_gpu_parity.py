@@ -294,9 +294,9 @@ def test_nondefault_stream():
 
 
 def test_bounded_wait_reports_timeout_and_context_survives():
-    """The float32 forward stages its inputs with bulk copies and waits for
-    them with a bounded poll.  With MSDA_TEST_WITHHOLD_COPY the copy is armed
-    but never issued: the wait runs out, the kernel reports
+    """With MSDA_STAGE_INPUTS the forward stages its inputs with bulk copies
+    and waits for them with a bounded poll.  With MSDA_TEST_WITHHOLD_COPY the
+    copy is armed but never issued: the wait runs out, the kernel reports
     MSDA_ERR_DEVICE_TIMEOUT and returns, and the next call works."""
     import ctypes
     from scale_deformable_attention_msdeformattn_b200 import _lib
@@ -304,7 +304,8 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     x = wl.generate(w)
     t = upload(x)
     out = torch.empty((1, 64, 2, 32), device="cuda")
-    prob = _lib.Problem(1, w.S, 64, 2, 32, 2, 2, _lib.MSDA_F32, _lib.MSDA_TEST_WITHHOLD_COPY)
+    prob = _lib.Problem(1, w.S, 64, 2, 32, 2, 2, _lib.MSDA_F32,
+                        _lib.MSDA_STAGE_INPUTS | _lib.MSDA_TEST_WITHHOLD_COPY)
     p = lambda z: ctypes.c_void_p(z.data_ptr())
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     assert msda.device_status() == 0
@@ -313,8 +314,15 @@ def test_bounded_wait_reports_timeout_and_context_survives():
                                   p(t["attention_weights"]), p(out), stream)
     assert st == 0
     assert msda.device_status() == _lib.MSDA_ERR_DEVICE_TIMEOUT
-    # the context is intact: a normal call succeeds and is correct
+    # the context is intact: a normal call succeeds and is correct, staged too
     out2 = msda.forward(t["value"], t["spatial_shapes"], t["level_start_index"],
                         t["sampling_locations"], t["attention_weights"])
     assert msda.device_status() == 0
     assert_close(out2, oracle_nonfused(x)[0], 1e-5, "after timeout")
+    prob.flags = _lib.MSDA_STAGE_INPUTS
+    out3 = torch.empty_like(out)
+    st = _lib.load().msda_forward(ctypes.byref(prob), p(t["value"]), p(t["spatial_shapes"]),
+                                  p(t["level_start_index"]), p(t["sampling_locations"]),
+                                  p(t["attention_weights"]), p(out3), stream)
+    assert st == 0 and msda.device_status() == 0
+    assert_close(out3, oracle_nonfused(x)[0], 1e-5, "staged forward")
