@@ -87,6 +87,9 @@ namespace msda {
 #ifndef MSDA_BWD_VB
 #define MSDA_BWD_VB 16
 #endif
+#ifndef MSDA_BWD_MIN_CTAS_F32       // backward CTAs per SM (register budget) by value type
+#define MSDA_BWD_MIN_CTAS_F32 3
+#endif
 #ifndef MSDA_BWD_MIN_CTAS
 #define MSDA_BWD_MIN_CTAS 2
 #endif
@@ -210,6 +213,7 @@ __device__ __forceinline__ U8 ld_vec(const U8 *p)
                  : "l"(p));
     return r;
 }
+__device__ __forceinline__ void st_vec(uint2 *p, const uint2 &v) { *p = v; }
 __device__ __forceinline__ void st_vec(uint4 *p, const uint4 &v) { *p = v; }
 __device__ __forceinline__ void st_vec(U8 *p, const U8 &v)
 {
@@ -309,9 +313,12 @@ template <typename T, int D, int VB> struct Layout {
     }
 };
 
-// Lane vector width of the backward for each value type.
+// Lane vector width and resident CTAs per SM of the backward for each value
+// type.
 template <typename T> struct BwdVB { static constexpr int kVB = MSDA_BWD_VB; };
 template <> struct BwdVB<S8> { static constexpr int kVB = 8; };
+template <typename T> struct BwdMinCtas { static constexpr int kN = MSDA_BWD_MIN_CTAS; };
+template <> struct BwdMinCtas<float> { static constexpr int kN = MSDA_BWD_MIN_CTAS_F32; };
 
 template <int G>
 __device__ __forceinline__ float group_sum(float v)
@@ -936,7 +943,10 @@ __device__ __forceinline__ void warp_sample(const KernelArgs &a, const Geometry 
     }
 }
 
-constexpr int kWarpSetupRounds = 8;  // rounds whose loads are issued together
+#ifndef MSDA_WARP_SETUP_ROUNDS
+#define MSDA_WARP_SETUP_ROUNDS 8
+#endif
+constexpr int kWarpSetupRounds = MSDA_WARP_SETUP_ROUNDS;  // rounds whose loads are issued together
 
 // Backward records of the warp's rows (inactive rows and pad slots inert).
 template <bool FUSED>
@@ -1248,7 +1258,7 @@ __device__ __forceinline__ void reduce_scatter3(float (&v)[C][3], int gl)
 template <int G> struct BwdChunk { static constexpr int kC = G < 4 ? G : 4; };
 
 template <typename T, int D, bool FUSED, bool GEN>
-__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, MSDA_BWD_MIN_CTAS)
+__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, BwdMinCtas<T>::kN)
 backward_kernel(const KernelArgs a_in)
 {
     KernelArgs a = a_in;
