@@ -1255,10 +1255,7 @@ __device__ __forceinline__ void reduce_scatter3(float (&v)[C][3], int gl)
 }
 
 // Samples per backward reduce-scatter chunk for G lanes per row.
-#ifndef MSDA_BWD_CHUNK
-#define MSDA_BWD_CHUNK 4
-#endif
-template <int G> struct BwdChunk { static constexpr int kC = G < MSDA_BWD_CHUNK ? G : MSDA_BWD_CHUNK; };
+template <int G> struct BwdChunk { static constexpr int kC = G < 4 ? G : 4; };
 
 template <typename T, int D, bool FUSED, bool GEN>
 __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, BwdMinCtas<T>::kN)
