@@ -76,8 +76,11 @@ typedef enum msda_status {
     MSDA_ERR_UNSUPPORTED = 2,   /* valid, but outside the supported sizes */
     MSDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
     MSDA_ERR_DEVICE_CHECK = 4,  /* a kernel found inconsistent geometry or a bad query_order entry */
-    MSDA_ERR_DEVICE_TIMEOUT = 5 /* a kernel gave up waiting for an input copy
+    MSDA_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up waiting for an input copy
                                    (bounded wait; the call's outputs are invalid) */
+    MSDA_ERR_DEVICE_BOUNDS = 6  /* checked build only (MSDA_BOUNDS_CHECK): a kernel
+                                   found a corner row outside its tensor and
+                                   skipped the access */
 } msda_status;
 
 typedef enum msda_dtype {

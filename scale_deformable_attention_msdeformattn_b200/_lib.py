@@ -16,6 +16,7 @@ MSDA_ERR_UNSUPPORTED = 2
 MSDA_ERR_CUDA = 3
 MSDA_ERR_DEVICE_CHECK = 4
 MSDA_ERR_DEVICE_TIMEOUT = 5
+MSDA_ERR_DEVICE_BOUNDS = 6
 
 MSDA_F32 = 0
 MSDA_BF16 = 1

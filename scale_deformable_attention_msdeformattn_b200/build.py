@@ -19,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmsda.so")
+CHECKED = os.path.join(PKG, "libmsda_checked.so")  # MSDA_BOUNDS_CHECK=1 variant (tests)
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
@@ -41,11 +42,19 @@ def _deps():
         sorted(glob.glob(os.path.join(INCLUDE, "*.h"))) + [os.path.abspath(__file__)]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(path: str = LIB) -> bool:
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(p) <= t for p in _deps())
+
+
+def build_checked(force: bool = False) -> str:
+    """The checked variant: every corner row a kernel reads or reduces into is
+    tested against its tensor (MSDA_BOUNDS_CHECK=1); the tests run it."""
+    if not force and up_to_date(CHECKED):
+        return CHECKED
+    return build(force=True, out=CHECKED, defines=("MSDA_BOUNDS_CHECK=1",))
 
 
 def build(force: bool = False, verbose: bool = False, out: str = LIB, defines=()) -> str:

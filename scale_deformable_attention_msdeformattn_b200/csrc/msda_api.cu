@@ -3,13 +3,15 @@
 //
 // Launch shape.  Every compute kernel runs as one persistent wave: the grid is
 // (SM count) x (resident CTAs per SM, from the occupancy calculator), walking
-// the row tiles band by band (see the scheduling notes in msda_kernels.cuh).  CTAs have up to 8 warps; fewer when
+// the row tiles grid-stride (tile_walk in msda_kernels.cuh).  CTAs have up to 8 warps; fewer when
 // the shared-memory records of the L*K samples of each row would exceed the
 // per-CTA budget.
 #include "msda.h"
 #include "msda_kernels.cuh"
 
 #include <mutex>
+
+#include <nvtx3/nvToolsExt.h>
 
 namespace {
 
@@ -457,6 +459,16 @@ void dcn_args(const msda_dcn_problem *d, int64_t wo, KernelArgs &a)
     a.dil_w = d->dilation_w;
 }
 
+// NVTX range around each entry point that enqueues work, so that a profiler
+// timeline shows the library calls (no-ops when no tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+#define MSDA_TRACE() NvtxRange msda_trace_range_(__func__)
+
 }  // namespace
 
 extern "C" {
@@ -478,6 +490,7 @@ msda_status msda_dcn_output_size(const msda_dcn_problem *problem, int64_t *out_h
 msda_status msda_dcn_forward(const msda_dcn_problem *problem, const void *input, const float *offset,
                              const float *mask, void *output, msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_problem p;
     int64_t ho = 0, wo = 0;
     msda_status st = dcn_to_problem(problem, p, ho, wo);
@@ -502,6 +515,7 @@ msda_status msda_dcn_backward(const msda_dcn_problem *problem, const void *input
                               float *grad_offset, float *grad_mask, void *workspace,
                               size_t workspace_bytes, msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_problem p;
     int64_t ho = 0, wo = 0;
     msda_status st = dcn_to_problem(problem, p, ho, wo);
@@ -538,6 +552,7 @@ msda_status msda_forward(const msda_problem *problem, const void *value,
                          const float *sampling_locations, const float *attention_weights,
                          void *output, msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
@@ -562,6 +577,7 @@ msda_status msda_backward(const msda_problem *problem, const void *value,
                           float *grad_sampling_locations, float *grad_attention_weights,
                           void *workspace, size_t workspace_bytes, msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
@@ -587,6 +603,7 @@ msda_status msda_fused_forward(const msda_problem *problem, const void *value,
                                const float *attention_logits, void *output,
                                float *attention_weights_out, msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
@@ -615,6 +632,7 @@ msda_status msda_fused_backward(const msda_problem *problem, const void *value,
                                 float *grad_sampling_offsets, float *grad_attention_logits,
                                 void *workspace, size_t workspace_bytes, msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
@@ -641,6 +659,7 @@ msda_status msda_fused_backward(const msda_problem *problem, const void *value,
 msda_status msda_zero_grads(const msda_problem *problem, float *grad_value,
                             float *grad_reference_points, msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
@@ -659,6 +678,7 @@ msda_status msda_backward_noalloc(const msda_problem *problem, const void *value
                                   float *grad_sampling_locations, float *grad_attention_weights,
                                   msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
@@ -703,6 +723,7 @@ msda_status msda_backward_noalloc(const msda_problem *problem, const void *value
 msda_status msda_quantize_value_s8(const msda_problem *problem, const void *value, void *value_s8,
                                    float *value_scale, msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
@@ -756,6 +777,7 @@ msda_status msda_quantize_value_s8(const msda_problem *problem, const void *valu
 msda_status msda_sort_queries(const msda_problem *problem, const float *points, int32_t *query_order,
                               msda_stream_t stream)
 {
+    MSDA_TRACE();
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
@@ -806,6 +828,7 @@ const char *msda_status_string(msda_status status)
     case MSDA_ERR_CUDA: return "CUDA runtime error";
     case MSDA_ERR_DEVICE_CHECK: return "kernel found inconsistent spatial_shapes / level_start_index or a query_order entry out of range";
     case MSDA_ERR_DEVICE_TIMEOUT: return "kernel gave up waiting for an input copy";
+    case MSDA_ERR_DEVICE_BOUNDS: return "checked build: a kernel found a row index outside its tensor";
     }
     return "unknown status";
 }

@@ -106,8 +106,33 @@ namespace msda {
 constexpr int kMaxLevels = 16;
 constexpr int kMaxWarpsPerCta = 8;
 
+#ifndef MSDA_BOUNDS_CHECK            // 1: checked build (every corner row tested)
+#define MSDA_BOUNDS_CHECK 0
+#endif
+
 // Per-device status word; kernels record inconsistent geometry here.
 __device__ int g_device_status;
+
+// Checked build (MSDA_BOUNDS_CHECK): the corner row offset `off` (key * M,
+// relative to the row's (batch, head) slice) that a kernel is about to read
+// or reduce into must lie in [0, S*M); a violation is recorded
+// (MSDA_ERR_DEVICE_BOUNDS = 6) and the access skipped.  By construction the
+// set-up only produces in-range offsets, so a clean run of the checked build
+// is evidence that every access stays inside value / grad_value.
+__device__ __forceinline__ bool row_in_bounds(int64_t S, int M, int off)
+{
+#if MSDA_BOUNDS_CHECK
+    if (off < 0 || (int64_t)off >= S * M) {
+        atomicExch(&g_device_status, 6 /* MSDA_ERR_DEVICE_BOUNDS */);
+        return false;
+    }
+#else
+    (void)S;
+    (void)M;
+    (void)off;
+#endif
+    return true;
+}
 
 struct KernelArgs {
     const void *value;
@@ -1180,7 +1205,9 @@ forward_kernel(const KernelArgs a_in)
                         for (int c = 0; c < 4; ++c)
 #pragma unroll
                             for (int j = 0; j < CH; ++j)
-                                v[u][c][j] = ld_vec(vbase + (int64_t)oc[c] * Lay::kNvec + j * G);
+                                v[u][c][j] = row_in_bounds(a.S, a.M, oc[c])
+                                                 ? ld_vec(vbase + (int64_t)oc[c] * Lay::kNvec + j * G)
+                                                 : Raw{};
                     }
                 }
 #pragma unroll
@@ -1411,7 +1438,10 @@ backward_kernel(const KernelArgs a_in)
 #pragma unroll
                         for (int j = 0; j < CH; ++j) {
                             float f[EPV];
-                            Lay::widen(ld_vec(vbase + (int64_t)oc[c] * Lay::kNvec + j * G), f);
+                            Lay::widen(row_in_bounds(a.S, a.M, oc[c])
+                                           ? ld_vec(vbase + (int64_t)oc[c] * Lay::kNvec + j * G)
+                                           : Raw{},
+                                       f);
 #pragma unroll
                             for (int e = 0; e < EPV; e += 2)
                                 dp = fma2(g2[(j * EPV + e) / 2], make_float2(f[e], f[e + 1]), dp);
@@ -1438,6 +1468,8 @@ backward_kernel(const KernelArgs a_in)
                     if (!(inm & (1u << c)))
                         continue;
                     const float awc = A * w[c];
+                    if (!row_in_bounds(a.S, a.M, ocs[c]))
+                        continue;
                     float4 *q = gvbase + (int64_t)ocs[c] * (D / 4);
                     const float2 ww = make_float2(awc, awc);
 #pragma unroll

@@ -27,7 +27,7 @@ def test_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     assert lib.msda_version().decode() == "0.1.0"
-    for code in range(5):
+    for code in range(7):
         assert lib.msda_status_string(code)
     assert b"unknown" in lib.msda_status_string(99)
 
