@@ -468,10 +468,13 @@ def version() -> str:
 
 class MSDeformAttnFunction(torch.autograd.Function):
     """Autograd wrapper over msda_forward / msda_backward (grad_value in the
-    value's dtype)."""
+    value's dtype).  Same argument order as the operator's usual autograd
+    function; a trailing im2col_step is accepted and ignored (the kernels
+    have no column buffer to chunk), so existing call sites need no change."""
 
     @staticmethod
-    def forward(ctx, value, spatial_shapes, level_start_index, sampling_locations, attention_weights):
+    def forward(ctx, value, spatial_shapes, level_start_index, sampling_locations, attention_weights,
+                im2col_step=None):
         ctx.save_for_backward(value, spatial_shapes, level_start_index, sampling_locations,
                               attention_weights)
         return forward(value, spatial_shapes, level_start_index, sampling_locations,
@@ -482,7 +485,7 @@ class MSDeformAttnFunction(torch.autograd.Function):
         value, shapes, starts, loc, attn = ctx.saved_tensors
         gv, gl, ga = backward(value, shapes, starts, loc, attn, grad_output.contiguous(),
                               grad_value_dtype=value.dtype)
-        return gv, None, None, gl, ga
+        return gv, None, None, gl, ga, None
 
 
 class MSDeformAttnFusedFunction(torch.autograd.Function):
@@ -504,11 +507,12 @@ class MSDeformAttnFusedFunction(torch.autograd.Function):
         return gv, None, None, gref, goff, glog.reshape(logits.shape)
 
 
-def ms_deform_attn(value, spatial_shapes, level_start_index, sampling_locations, attention_weights):
+def ms_deform_attn(value, spatial_shapes, level_start_index, sampling_locations, attention_weights,
+                   im2col_step=None):
     """Differentiable core operator; output [B, Q, M*D] like the module's
-    reshape before output_proj."""
+    reshape before output_proj (im2col_step accepted and ignored)."""
     out = MSDeformAttnFunction.apply(value, spatial_shapes, level_start_index, sampling_locations,
-                                     attention_weights)
+                                     attention_weights, im2col_step)
     return out.flatten(2)
 
 

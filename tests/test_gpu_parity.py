@@ -265,6 +265,10 @@ def test_autograd_wrappers():
     ref = oracle_nonfused(x)
     assert_close(v.grad, ref[1], 1e-5, "autograd grad_value")
     assert_close(loc.grad, ref[2], 1e-5, "autograd grad_loc")
+    # the usual call site with a trailing im2col_step (accepted, ignored)
+    out64 = msda.MSDeformAttnFunction.apply(t["value"], t["spatial_shapes"], t["level_start_index"],
+                                            t["sampling_locations"], t["attention_weights"], 64)
+    assert torch.equal(out64.flatten(2), out.detach())
     assert_close(a.grad, ref[3], 1e-5, "autograd grad_attn")
     ref_pts = t["reference_points"].clone().requires_grad_(True)
     off = t["sampling_offsets"].clone().requires_grad_(True)
