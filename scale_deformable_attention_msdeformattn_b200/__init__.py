@@ -2,8 +2,10 @@
 
 The operator runs in libmsda.so (hand-written CUDA kernels behind the C ABI of
 include/msda.h); this package is its Python binding.  PyTorch only provides
-device memory and the current stream.
+device memory and the current stream, and, in the optional MSDeformAttn layer,
+the linear projections around the operator.
 """
+from .module import MSDeformAttn  # noqa: F401
 from .binding import (  # noqa: F401
     MsdaError,
     MSDeformAttnFunction,
