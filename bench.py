@@ -51,6 +51,9 @@ NCU_TRAFFIC = {
     # profiles/detr_encoder_f32_fused_kernels.md: 107.71 MB read + 20.30 MB written
     ("fused_backward", "detr_encoder_f32"): {"bytes": 128009728, "csrc": "b307ee533b6790b5"},
     ("fused_forward", "detr_encoder_f32"): {"bytes": 60423168, "csrc": "b307ee533b6790b5"},
+    # profiles/dcnv3_stage1_f32_kernels.md: 122.60 MB read + 21.93 MB written
+    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 144524544, "csrc": "b307ee533b6790b5"},
+    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 73908992, "csrc": "b307ee533b6790b5"},
 }
 
 
@@ -997,7 +1000,9 @@ def run_dcn(args):
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4),
-                         "bytes_per_launch": nb[dom], "traffic": None},
+                         "bytes_per_launch": nb[dom],
+                         "traffic": (lambda tr: tr["bytes"] if tr and tr.get("csrc") == csrc_hash()
+                                     else None)(NCU_TRAFFIC.get((dom, w.name)))},
             "gpu_launches": (3 + (3 if int8 else 0)) * args.steps,
             "clocks": clocks.summary(),
         }
