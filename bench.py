@@ -689,6 +689,18 @@ def _oracle_step(oracle, smp):
                           smp["attention_logits"], smp["grad_output"])
 
 
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(w: wl.Workload, x: wl.Inputs, seconds: float) -> dict:
     """The fp64 oracle (plain C loops, one thread), fused forward + backward on
     a bounded sample of the workload, timed on this host's cores."""
@@ -708,7 +720,7 @@ def cpu_baseline(w: wl.Workload, x: wl.Inputs, seconds: float) -> dict:
     return {"value": round(rate / 1e9, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"every {stride}th query ({smp['queries']} of {w.num_queries}, "
                       f"{smp['samples']} samples) x {passes} passes of fused fwd+bwd, "
-                      f"{el:.1f} s", "host_cpus": os.cpu_count(),
+                      f"{el:.1f} s", "host_cpus": os.cpu_count(), "cpu_model": _cpu_model(),
             "full_step_ms_extrapolated": round(w.samples / rate * 1e3, 1)}
 
 
