@@ -262,11 +262,22 @@ msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
             MSDA_FWD_CASE(float, 64) MSDA_FWD_CASE(float, 128) MSDA_FWD_CASE(float, 256)
         }
     } else if (p->value_dtype == MSDA_BF16) {
+        // bf16 rows of at most 16 samples take the SHORT tuning (msda_kernels.cuh)
+        const bool short_rows = a.L * a.K <= 16;
+#define MSDA_FWD_CASE_BF16(DD)                                                                     \
+    case DD:                                                                                        \
+        return launch_rows(                                                                         \
+            short_rows ? (gen ? (const void *)msda::forward_kernel<__nv_bfloat16, DD, FUSED, true, true>    \
+                              : (const void *)msda::forward_kernel<__nv_bfloat16, DD, FUSED, false, true>)  \
+                       : (gen ? (const void *)msda::forward_kernel<__nv_bfloat16, DD, FUSED, true, false>   \
+                              : (const void *)msda::forward_kernel<__nv_bfloat16, DD, FUSED, false, false>), \
+            msda::forward_rows_per_warp<__nv_bfloat16, DD>(), kForwardRecordBytes, a.L * a.K,     \
+            msda::forward_stages<__nv_bfloat16>() || (a.stage && !a.order), a, s);
         switch (p->head_dim) {
-            MSDA_FWD_CASE(__nv_bfloat16, 8) MSDA_FWD_CASE(__nv_bfloat16, 16)
-            MSDA_FWD_CASE(__nv_bfloat16, 32) MSDA_FWD_CASE(__nv_bfloat16, 64)
-            MSDA_FWD_CASE(__nv_bfloat16, 128) MSDA_FWD_CASE(__nv_bfloat16, 256)
+            MSDA_FWD_CASE_BF16(8) MSDA_FWD_CASE_BF16(16) MSDA_FWD_CASE_BF16(32)
+            MSDA_FWD_CASE_BF16(64) MSDA_FWD_CASE_BF16(128) MSDA_FWD_CASE_BF16(256)
         }
+#undef MSDA_FWD_CASE_BF16
     } else {
         switch (p->head_dim) {
             MSDA_FWD_CASE(msda::S8, 8) MSDA_FWD_CASE(msda::S8, 16) MSDA_FWD_CASE(msda::S8, 32)
