@@ -26,7 +26,7 @@
  *              1-3: normalized coordinates, align_corners=False (pixels are
  *              cell centres), softmax over all L*K points.
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent:
  *   - pixel coordinate of a normalized location: x = loc_x * W - 0.5,
  *     y = loc_y * H - 0.5 (what grid_sample with align_corners=False does to
  *     grid = 2*loc - 1, [cf-1] §5.3, [csdn] §3 note 2);

@@ -72,8 +72,8 @@ def test_int8_full_size(name):
     x = wl.generate(w)
     t, q, scale = _check(w, x)
     # accuracy of INT8 storage against the bf16 value it was quantised from
-    # (information for the reader; the pages give no criterion, see the
-    # design notes): the fused forward output differs by a few hundredths
+    # (information for the reader: the pages give no accuracy criterion for
+    # INT8 storage): the fused forward output differs by a few hundredths
     out_bf16 = msda.fused_forward(t["value"], t["spatial_shapes"], t["level_start_index"],
                                   t["reference_points"], t["sampling_offsets"], t["attention_logits"])
     out_s8 = msda.fused_forward(q, t["spatial_shapes"], t["level_start_index"], t["reference_points"],
