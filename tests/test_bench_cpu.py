@@ -65,3 +65,26 @@ def test_clock_summary_decodes_reasons():
     s = c.summary()
     assert s["sm_mhz"] == 1965 and s["sm_mhz_min"] == 1950
     assert set(s["reasons"]) == {"sw_power_cap", "hw_thermal_slowdown"}  # gpu_idle dropped
+
+
+def test_dcn_workload_sizes_agree_with_the_oracle_and_the_library():
+    """Output grid of each DCNv3 workload: the workload table, the oracle and
+    the C ABI's msda_dcn_output_size agree; the draws are reproducible."""
+    import ctypes
+
+    import oracle
+    from scale_deformable_attention_msdeformattn_b200 import _lib, build
+    build.build()
+    lib = _lib.load()
+    for w in wl.DCN_WORKLOADS.values():
+        ho, wo = w.out_hw
+        assert (ho, wo) == oracle.dcn_output_size(w.H, w.W, w.kernel, w.stride, w.pad, w.dil)
+        p = _lib.DcnProblem(w.N, w.H, w.W, w.G, w.C, w.kernel[0], w.kernel[1], w.stride[0],
+                            w.stride[1], w.pad[0], w.pad[1], w.dil[0], w.dil[1], _lib.MSDA_F32, 0)
+        a, b = ctypes.c_int64(0), ctypes.c_int64(0)
+        assert lib.msda_dcn_output_size(ctypes.byref(p), ctypes.byref(a), ctypes.byref(b)) == 0
+        assert (a.value, b.value) == (ho, wo)
+    w = wl.custom_dcn("repro", 1, 6, 7, 2, 8, (3, 3))
+    x1, x2 = wl.generate_dcn(w), wl.generate_dcn(w)
+    assert np.array_equal(x1.offset, x2.offset) and np.array_equal(x1.mask, x2.mask)
+    np.testing.assert_allclose(x1.mask.sum(-1), 1.0, rtol=1e-5)
