@@ -373,9 +373,10 @@ MSDA_API msda_status msda_dcn_backward_workspace_size(const msda_dcn_problem *pr
 
 /*
  * Synchronizes `stream`, then returns in *code the status the kernels recorded
- * on the current device since the last call (MSDA_OK, MSDA_ERR_DEVICE_CHECK or
- * MSDA_ERR_DEVICE_TIMEOUT), and clears it.  Returns MSDA_ERR_CUDA if the
- * synchronization or the read fails.
+ * on the current device since the last call (MSDA_OK, MSDA_ERR_DEVICE_CHECK,
+ * MSDA_ERR_DEVICE_TIMEOUT, or MSDA_ERR_DEVICE_BOUNDS in the checked build), and
+ * clears it.  The word belongs to the loaded library (the checked build has its
+ * own).  Returns MSDA_ERR_CUDA if the synchronization or the read fails.
  */
 MSDA_API msda_status msda_get_device_status(msda_stream_t stream, int32_t *code);
 
