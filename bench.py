@@ -80,6 +80,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-nonfused", action="store_true")
+    ap.add_argument("--merge-reductions", action="store_true",
+                    help="backward merges each tile's grad_value contributions per corner "
+                         "row before reducing them (MSDA_MERGE_REDUCTIONS)")
     ap.add_argument("--sorted", action="store_true",
                     help="order the queries by the Morton cell of their reference point "
                          "(msda_sort_queries, inside the timed step) and process them in that order")
@@ -328,7 +331,8 @@ def run_ours(args):
                             grad_value=o["grad_value"], grad_reference_points=o["grad_reference_points"],
                             grad_sampling_offsets=o["grad_sampling_offsets"],
                             grad_attention_logits=o["grad_attention_logits"],
-                            query_order=order, value_scale=qs)
+                            query_order=order, value_scale=qs,
+                            merge_reductions=args.merge_reductions)
         ev[3].record(stream)
         return o
 
@@ -434,6 +438,15 @@ def run_ours(args):
             result["nonfused"] = _time_nonfused(msda, t, w, nbytes, flush, min(args.steps, 50),
                                                 qv if int8 else t["value"], qs)
         if world == 1:
+            # the fused backward with the other grad_value reduction path
+            result["bwd_other_reductions"] = _time_bwd(
+                msda, t, o=outputs, flush=flush, n=min(args.steps, 50),
+                value=qv if int8 else t["value"], value_scale=qs, order=order,
+                merge=not args.merge_reductions)
+            result["config"]["grad_value_reductions"] = (
+                "merged per tile of consecutive queries of one head"
+                if args.merge_reductions and not args.sorted
+                else "direct (one vector reduction per corner contribution)")
             result["warm_l2"] = _time_warm(w, step, min(args.steps, 50))
             result["graph"] = _time_graph(w.samples, step, flush, min(args.steps, 100), 7)
         stats = _input_stats(w, x)
@@ -506,6 +519,33 @@ def _time_nonfused(msda, t, w, nbytes, flush, n, value, value_scale=None):
             "fwd_hbm_frac": round(nbytes["forward"] / (fwd * 1e-3) / 1e9 / peak, 4),
             "bwd_hbm_frac": round(nbytes["backward"] / (bwd * 1e-3) / 1e9 / peak, 4),
             "fwd_gsamples_per_s": round(w.samples / (fwd * 1e-3) / 1e9, 4), "launches": n}
+
+
+def _time_bwd(msda, t, o, flush, n, value, value_scale, order, merge):
+    """msda_fused_backward alone (zero-fill outside the events, L2 flushed
+    before each launch) with the given grad_value reduction path."""
+    import torch
+    stream = torch.cuda.current_stream()
+    ts = []
+    for i in range(n + 3):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        msda.zero_grads(o["grad_value"], o["grad_reference_points"])
+        flush.fill_(float(i))
+        e[0].record(stream)
+        msda.fused_backward(value, t["spatial_shapes"], t["level_start_index"],
+                            t["reference_points"], t["sampling_offsets"], t["attention_logits"],
+                            t["grad_output"], accumulate=True, grad_value=o["grad_value"],
+                            grad_reference_points=o["grad_reference_points"],
+                            grad_sampling_offsets=o["grad_sampling_offsets"],
+                            grad_attention_logits=o["grad_attention_logits"],
+                            query_order=order, value_scale=value_scale, merge_reductions=merge)
+        e[1].record(stream)
+        if i >= 3:
+            ts.append(e)
+    torch.cuda.synchronize()
+    ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ts)
+    return {"reductions": "merged" if merge and order is None else "direct",
+            "bwd_ms": round(ms, 5), "launches": n}
 
 
 def _time_graph(samples, step, flush, n, nev):

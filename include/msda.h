@@ -111,6 +111,18 @@ typedef enum msda_dtype {
                                           L*K <= 32, natural query order.  A
                                           performance option (off by default:
                                           slower with the default lane layout) */
+#define MSDA_MERGE_REDUCTIONS (1u << 3) /* backward: per tile of consecutive
+                                          queries of one head, merge in shared
+                                          memory the grad_value contributions
+                                          that share a corner row before
+                                          reducing them (one reduction per
+                                          distinct row instead of one per
+                                          corner).  Results agree within float32
+                                          rounding.  A performance option, off
+                                          by default: on B200 the merge costs
+                                          more than the reductions it saves on
+                                          every workload measured.  Ignored with
+                                          a query_order */
 #define MSDA_TEST_WITHHOLD_COPY (1u << 31) /* testing only: kernels that stage
                                           their inputs with bulk copies arm
                                           the copy but never issue it, so

@@ -25,6 +25,7 @@ MSDA_S8 = 2
 MSDA_GRAD_VALUE_BF16 = 1 << 0
 MSDA_ACCUMULATE_GRADS = 1 << 1
 MSDA_STAGE_INPUTS = 1 << 2
+MSDA_MERGE_REDUCTIONS = 1 << 3
 MSDA_TEST_WITHHOLD_COPY = 1 << 31
 
 

@@ -139,11 +139,14 @@ def backward(value, spatial_shapes, level_start_index, sampling_locations, atten
              workspace: Optional[torch.Tensor] = None,
              accumulate: bool = False,
              query_order: Optional[torch.Tensor] = None,
-             value_scale: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+             value_scale: Optional[torch.Tensor] = None,
+             merge_reductions: bool = False) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """msda_backward: (grad_value, grad_sampling_locations, grad_attention_weights).
 
     accumulate=True adds into the given float32 grad_value instead of
-    overwriting it (MSDA_ACCUMULATE_GRADS)."""
+    overwriting it (MSDA_ACCUMULATE_GRADS); merge_reductions=True merges the
+    grad_value contributions of each tile per corner row before reducing them
+    (MSDA_MERGE_REDUCTIONS, a performance option)."""
     _need(value, "value", None)
     L = _geometry(value, spatial_shapes, level_start_index)
     B, S, M, D = value.shape
@@ -159,6 +162,8 @@ def backward(value, spatial_shapes, level_start_index, sampling_locations, atten
         if grad_value is None:
             raise ValueError("accumulate=True needs the grad_value buffer to add into")
         flags |= _lib.MSDA_ACCUMULATE_GRADS
+    if merge_reductions:
+        flags |= _lib.MSDA_MERGE_REDUCTIONS
     if grad_value is None:
         grad_value = torch.empty((B, S, M, D), dtype=grad_value_dtype, device=dev)
     if grad_sampling_locations is None:
@@ -228,12 +233,15 @@ def fused_backward(value, spatial_shapes, level_start_index, reference_points, s
                    grad_sampling_offsets: Optional[torch.Tensor] = None,
                    grad_attention_logits: Optional[torch.Tensor] = None,
                    query_order: Optional[torch.Tensor] = None,
-                   value_scale: Optional[torch.Tensor] = None):
+                   value_scale: Optional[torch.Tensor] = None,
+                   merge_reductions: bool = False):
     """msda_fused_backward: (grad_value, grad_reference_points or None,
     grad_sampling_offsets, grad_attention_logits [B, Q, M, L*K]).
 
     accumulate=True adds into the given float32 grad_value (and
-    grad_reference_points) instead of overwriting them."""
+    grad_reference_points) instead of overwriting them; merge_reductions=True
+    merges each tile's grad_value contributions per corner row first
+    (MSDA_MERGE_REDUCTIONS, a performance option)."""
     _need(value, "value", None)
     L = _geometry(value, spatial_shapes, level_start_index)
     B, S, M, D = value.shape
@@ -250,6 +258,8 @@ def fused_backward(value, spatial_shapes, level_start_index, reference_points, s
         if grad_value is None or (want_grad_reference_points and grad_reference_points is None):
             raise ValueError("accumulate=True needs the buffers to add into")
         flags |= _lib.MSDA_ACCUMULATE_GRADS
+    if merge_reductions:
+        flags |= _lib.MSDA_MERGE_REDUCTIONS
     if grad_value is None:
         grad_value = torch.empty((B, S, M, D), dtype=grad_value_dtype, device=dev)
     _need(grad_value, "grad_value", grad_value_dtype, (B, S, M, D), dev)
@@ -384,8 +394,11 @@ def dcn_backward(input, offset, mask, grad_output, kernel=3, stride=1, pad=1, di
                  grad_input_dtype=torch.float32, grad_input: Optional[torch.Tensor] = None,
                  accumulate: bool = False, value_scale: Optional[torch.Tensor] = None,
                  grad_offset: Optional[torch.Tensor] = None,
-                 grad_mask: Optional[torch.Tensor] = None):
-    """msda_dcn_backward: (grad_input, grad_offset, grad_mask)."""
+                 grad_mask: Optional[torch.Tensor] = None,
+                 merge_reductions: bool = False):
+    """msda_dcn_backward: (grad_input, grad_offset, grad_mask);
+    merge_reductions=True merges each tile's contributions per input row
+    before reducing them (MSDA_MERGE_REDUCTIONS)."""
     _need(input, "input", None)
     if grad_input_dtype not in (torch.float32, torch.bfloat16):
         raise TypeError("grad_input_dtype must be float32 or bfloat16")
@@ -394,6 +407,8 @@ def dcn_backward(input, offset, mask, grad_output, kernel=3, stride=1, pad=1, di
         if grad_input is None:
             raise ValueError("accumulate=True needs the grad_input buffer to add into")
         flags |= _lib.MSDA_ACCUMULATE_GRADS
+    if merge_reductions:
+        flags |= _lib.MSDA_MERGE_REDUCTIONS
     prob, Ho, Wo = _dcn_problem(input, kernel, stride, pad, dilation, flags, value_scale)
     N, H, W, G, C = input.shape
     K = prob.kernel_h * prob.kernel_w

@@ -3,11 +3,12 @@
     python -m scale_deformable_attention_msdeformattn_b200.build [--verbose]
 
 The library links only the CUDA runtime (statically, nvcc's default); it has
-no PyTorch dependency.  The build is skipped when the .so is newer than every
-source file.
+no PyTorch dependency.  Its .cu files compile in parallel.  The build is
+skipped when the .so is newer than every source file.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -22,8 +23,9 @@ LIB = os.path.join(PKG, "libmsda.so")
 CHECKED = os.path.join(PKG, "libmsda_checked.so")  # MSDA_BOUNDS_CHECK=1 variant (tests)
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-         "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]
+COMPILE_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+                 "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]
+LINK_FLAGS = ["-shared", "-Xcompiler", "-fPIC"]
 
 
 def nvcc() -> str:
@@ -57,23 +59,52 @@ def build_checked(force: bool = False) -> str:
     return build(force=True, out=CHECKED, defines=("MSDA_BOUNDS_CHECK=1",))
 
 
+def _compile(args):
+    cmd, verbose = args
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    return cmd, res.returncode, res.stdout, res.stderr
+
+
 def build(force: bool = False, verbose: bool = False, out: str = LIB, defines=()) -> str:
-    """Compiles the library to `out`; `defines` are extra -D tuning knobs."""
+    """Compiles the library to `out`; `defines` are extra -D tuning knobs.
+
+    Each .cu file (the C ABI and one file per group of kernel instantiations)
+    compiles to an object in parallel; nvcc then links the shared library."""
     if not force and out == LIB and not defines and up_to_date():
         return LIB
-    tmp = out + ".%d.tmp" % os.getpid()
-    cmd = [nvcc()] + ARCH + FLAGS + ["-D" + d for d in defines] + \
-        ["-I", INCLUDE, "-I", CSRC, "-o", tmp] + sources()
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-        print(" ".join(cmd))
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if verbose or res.returncode != 0:
-        sys.stdout.write(res.stdout)
-        sys.stderr.write(res.stderr)
-    if res.returncode != 0:
-        raise RuntimeError("nvcc failed (exit %d)" % res.returncode)
-    os.replace(tmp, out)
+    objdir = out + ".%d.obj" % os.getpid()
+    os.makedirs(objdir, exist_ok=True)
+    try:
+        jobs = []
+        for src in sources():
+            obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
+            cmd = [nvcc()] + ARCH + COMPILE_FLAGS + ["-D" + d for d in defines] + \
+                ["-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+            if verbose:
+                cmd += ["-Xptxas", "-v"]
+            jobs.append((cmd, verbose))
+        workers = max(1, min(len(jobs), os.cpu_count() or 1))
+        objs = []
+        with concurrent.futures.ThreadPoolExecutor(workers) as pool:
+            for cmd, rc, so, se in pool.map(_compile, jobs):
+                if verbose or rc != 0:
+                    print(" ".join(cmd))
+                    sys.stdout.write(so)
+                    sys.stderr.write(se)
+                if rc != 0:
+                    raise RuntimeError("nvcc failed (exit %d)" % rc)
+                objs.append(cmd[cmd.index("-o") + 1])
+        tmp = out + ".%d.tmp" % os.getpid()
+        link = [nvcc()] + ARCH + LINK_FLAGS + ["-o", tmp] + objs
+        res = subprocess.run(link, capture_output=True, text=True)
+        if verbose or res.returncode != 0:
+            sys.stdout.write(res.stdout)
+            sys.stderr.write(res.stderr)
+        if res.returncode != 0:
+            raise RuntimeError("nvcc link failed (exit %d)" % res.returncode)
+        os.replace(tmp, out)
+    finally:
+        shutil.rmtree(objdir, ignore_errors=True)
     return out
 
 

@@ -7,9 +7,18 @@
 // the shared-memory records of the L*K samples of each row would exceed the
 // per-CTA budget.
 #include "msda.h"
-#include "msda_kernels.cuh"
+#include "msda_aux.cuh"
+#include "msda_instances.cuh"
 
 #include <mutex>
+
+namespace msda {
+// the operator kernels are instantiated in the msda_inst_*.cu units
+MSDA_ALL_INSTANCES(extern)
+
+// Per-device status word; kernels record failures through KernelArgs::status.
+__device__ int g_device_status;
+}  // namespace msda
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -59,7 +68,7 @@ msda_status check_problem(const msda_problem *p)
         (!p->value_scale || (reinterpret_cast<uintptr_t>(p->value_scale) & 3u)))
         return MSDA_ERR_INVALID_ARG;
     if (p->flags & ~(uint32_t)(MSDA_GRAD_VALUE_BF16 | MSDA_ACCUMULATE_GRADS | MSDA_STAGE_INPUTS |
-                               MSDA_TEST_WITHHOLD_COPY))
+                               MSDA_MERGE_REDUCTIONS | MSDA_TEST_WITHHOLD_COPY))
         return MSDA_ERR_INVALID_ARG;
     if ((p->flags & MSDA_GRAD_VALUE_BF16) && (p->flags & MSDA_ACCUMULATE_GRADS))
         return MSDA_ERR_INVALID_ARG;
@@ -92,23 +101,32 @@ msda_status check_problem(const msda_problem *p)
 
 struct DeviceInfo {
     int sm_count = 0;
+    int *status = nullptr;  // device address of msda::g_device_status
 };
 
 std::mutex g_mutex;
 DeviceInfo g_devices[kMaxDevices];
 
-msda_status current_device(int &dev, int &sm_count)
+// SM count and status-word address of the current device, looked up once per
+// device (with that device current) on its first call.
+msda_status current_device(int &dev, int &sm_count, int **status = nullptr)
 {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return MSDA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mutex);
     if (g_devices[dev].sm_count == 0) {
         int n = 0;
+        void *st = nullptr;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             return MSDA_ERR_CUDA;
+        if (cudaGetSymbolAddress(&st, msda::g_device_status) != cudaSuccess || !st)
+            return MSDA_ERR_CUDA;
+        g_devices[dev].status = static_cast<int *>(st);
         g_devices[dev].sm_count = n;
     }
     sm_count = g_devices[dev].sm_count;
+    if (status)
+        *status = g_devices[dev].status;
     return MSDA_OK;
 }
 
@@ -179,7 +197,7 @@ msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, int pa
                         bool stages, KernelArgs &a, cudaStream_t stream)
 {
     int dev = 0, sms = 0;
-    msda_status st = current_device(dev, sms);
+    msda_status st = current_device(dev, sms, &a.status);
     if (st != MSDA_OK)
         return st;
     // records of the warp's rows, then (power-of-two L*K up to 32) the warp's
@@ -197,6 +215,69 @@ msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, int pa
     a.rows_per_tile = (int64_t)warps * rpw;
     a.ntiles = (a.rows + a.rows_per_tile - 1) / a.rows_per_tile;
     // one resident wave, but no more CTAs than there are tiles
+    int64_t ctas = (int64_t)sms * blocks_per_sm;
+    if (ctas > a.ntiles)
+        ctas = a.ntiles;
+    void *params[] = {&a};
+    if (cudaLaunchKernel(kernel, dim3((unsigned)ctas), dim3(threads), params, smem, stream) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    return MSDA_OK;
+}
+
+// Shared-memory budget of one CTA of the merged backward: float32 value runs
+// three CTAs per SM (its register budget), the others two.
+constexpr size_t kMergeSmemBudgetF32 = 72 * 1024;
+constexpr size_t kMergeSmemBudget = 108 * 1024;
+
+// Launches the merged backward (tiles of one head of merge_qb consecutive
+// queries of one batch; msda_kernels.cuh "merged reductions") as a
+// persistent wave.  The tile takes as many warps (up to 8) as fit the budget
+// with a hash table of at least one slot per contribution and 16-bit
+// contribution ids; `fits` is false when not even one warp does (the caller
+// then takes the direct path).
+msda_status launch_merge(const void *kernel, int rpw, size_t record_bytes, int padded_samples, int D,
+                         size_t budget, KernelArgs &a, const msda_problem *p, cudaStream_t stream,
+                         bool &fits)
+{
+    fits = false;
+    int dev = 0, sms = 0;
+    msda_status st = current_device(dev, sms, &a.status);
+    if (st != MSDA_OK)
+        return st;
+    const int stride = msda::record_stride(padded_samples);
+    // no more warps than the queries of one batch need
+    const int64_t need = (p->num_queries + rpw - 1) / rpw;
+    int warps = need < msda::kMaxWarpsPerCta ? (int)need : msda::kMaxWarpsPerCta;
+    int tslots = 0, tbits = 0;
+    size_t smem = 0;
+    for (; warps >= 1; --warps) {
+        const int64_t rows = (int64_t)warps * rpw;
+        const int64_t ids = rows * stride * 4;
+        const int64_t items = rows * padded_samples * 4;
+        tbits = 2;
+        while ((int64_t(1) << tbits) < items)
+            ++tbits;
+        tslots = 1 << tbits;
+        if (ids > 0xFFFF || tslots > 0x10000)
+            continue;
+        smem = msda::merge_layout((size_t)rows * stride * record_bytes, rows, stride, D, tslots).total;
+        if (smem <= budget)
+            break;
+    }
+    if (warps < 1)
+        return MSDA_OK;
+    fits = true;
+    const int threads = warps * 32;
+    int blocks_per_sm = 0;
+    st = occupancy(kernel, dev, threads, smem, blocks_per_sm);
+    if (st != MSDA_OK)
+        return st;
+    a.rows_per_tile = (int64_t)warps * rpw;
+    a.merge_qb = a.rows_per_tile;
+    a.merge_nqb = (p->num_queries + a.merge_qb - 1) / a.merge_qb;
+    a.merge_tslots = tslots;
+    a.merge_tbits = tbits;
+    a.ntiles = p->batch * a.merge_nqb * p->num_heads;
     int64_t ctas = (int64_t)sms * blocks_per_sm;
     if (ctas > a.ntiles)
         ctas = a.ntiles;
@@ -288,18 +369,36 @@ msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
     return MSDA_ERR_UNSUPPORTED;
 }
 
+// Backward kernel for (T, D): direct grad_value reductions, or merged ones
+// when the caller asks (MSDA_MERGE_REDUCTIONS), no query order is given
+// (merged tiles follow the natural order) and a merged tile fits.
+template <typename T, int D, bool FUSED>
+msda_status launch_backward_td(const msda_problem *p, KernelArgs &a, cudaStream_t s)
+{
+    const bool gen = a.order != nullptr || a.dcn != 0;
+    const int rpw = msda::backward_rows_per_warp<T, D>();
+    const size_t rec = FUSED ? kFusedBackwardRecordBytes : kBackwardRecordBytes;
+    const int pp = msda::backward_padded_samples<T, D>(a.L * a.K);
+    if (!a.order && (p->flags & MSDA_MERGE_REDUCTIONS)) {
+        const void *k = gen ? (const void *)msda::backward_kernel<T, D, FUSED, true, true>
+                            : (const void *)msda::backward_kernel<T, D, FUSED, false, true>;
+        bool fits = false;
+        const size_t budget = std::is_same<T, float>::value ? kMergeSmemBudgetF32 : kMergeSmemBudget;
+        msda_status st = launch_merge(k, rpw, rec, pp, D, budget, a, p, s, fits);
+        if (st != MSDA_OK || fits)
+            return st;
+    }
+    const void *k = gen ? (const void *)msda::backward_kernel<T, D, FUSED, true, false>
+                        : (const void *)msda::backward_kernel<T, D, FUSED, false, false>;
+    return launch_rows(k, rpw, rec, pp, false, a, s);
+}
+
 template <bool FUSED>
 msda_status launch_backward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 {
-    const bool gen = a.order != nullptr || a.dcn != 0 || a.stage != 0;
-#define MSDA_BWD_CASE(T, DD)                                                                       \
-    case DD:                                                                                        \
-        return launch_rows(gen ? (const void *)msda::backward_kernel<T, DD, FUSED, true>         \
-                               : (const void *)msda::backward_kernel<T, DD, FUSED, false>,       \
-                           msda::backward_rows_per_warp<T, DD>(),                                \
-                           FUSED ? kFusedBackwardRecordBytes : kBackwardRecordBytes,             \
-                           msda::backward_padded_samples<T, DD>(a.L * a.K), msda::backward_stages(), \
-                           a, s);
+#define MSDA_BWD_CASE(T, DD) \
+    case DD:                 \
+        return launch_backward_td<T, DD, FUSED>(p, a, s);
     if (p->value_dtype == MSDA_F32) {
         switch (p->head_dim) {
             MSDA_BWD_CASE(float, 8) MSDA_BWD_CASE(float, 16) MSDA_BWD_CASE(float, 32)
@@ -693,7 +792,7 @@ msda_status msda_backward_noalloc(const msda_problem *problem, const void *value
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
-    if (problem->flags & ~(uint32_t)MSDA_GRAD_VALUE_BF16)
+    if (problem->flags & ~(uint32_t)(MSDA_GRAD_VALUE_BF16 | MSDA_MERGE_REDUCTIONS))
         return MSDA_ERR_INVALID_ARG;
     const Sizes z = sizes_of(problem);
     if (z.value > kNoAllocScratchFloats)

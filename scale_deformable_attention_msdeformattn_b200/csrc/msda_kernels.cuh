@@ -78,9 +78,6 @@ namespace msda {
 #ifndef MSDA_FWD_STAGE_BF16
 #define MSDA_FWD_STAGE_BF16 0
 #endif
-#ifndef MSDA_BWD_STAGE
-#define MSDA_BWD_STAGE 0
-#endif
 #ifndef MSDA_FWD_VB_S8               // INT8 value: bytes per lane vector
 #define MSDA_FWD_VB_S8 8
 #endif
@@ -99,11 +96,8 @@ namespace msda {
 #ifndef MSDA_BWD_MIN_CTAS
 #define MSDA_BWD_MIN_CTAS 2
 #endif
-#ifndef MSDA_CONTIGUOUS_TILES        // 1: each CTA walks one contiguous run of tiles
-#define MSDA_CONTIGUOUS_TILES 0
-#endif
-#ifndef MSDA_HEAD_MAJOR              // 1: process rows head-major
-#define MSDA_HEAD_MAJOR 0
+#ifndef MSDA_MERGE_FLUSH_CHAINS      // merged backward: slot lists a lane group walks together
+#define MSDA_MERGE_FLUSH_CHAINS 1
 #endif
 #ifndef MSDA_STREAM_HINTS            // 1: L2 evict-first on streaming arrays
 #define MSDA_STREAM_HINTS 1
@@ -115,30 +109,6 @@ constexpr int kMaxWarpsPerCta = 8;
 #ifndef MSDA_BOUNDS_CHECK            // 1: checked build (every corner row tested)
 #define MSDA_BOUNDS_CHECK 0
 #endif
-
-// Per-device status word; kernels record inconsistent geometry here.
-__device__ int g_device_status;
-
-// Checked build (MSDA_BOUNDS_CHECK): the corner row offset `off` (key * M,
-// relative to the row's (batch, head) slice) that a kernel is about to read
-// or reduce into must lie in [0, S*M); a violation is recorded
-// (MSDA_ERR_DEVICE_BOUNDS = 6) and the access skipped.  By construction the
-// set-up only produces in-range offsets, so a clean run of the checked build
-// is evidence that every access stays inside value / grad_value.
-__device__ __forceinline__ bool row_in_bounds(int64_t S, int M, int off)
-{
-#if MSDA_BOUNDS_CHECK
-    if (off < 0 || (int64_t)off >= S * M) {
-        atomicExch(&g_device_status, 6 /* MSDA_ERR_DEVICE_BOUNDS */);
-        return false;
-    }
-#else
-    (void)S;
-    (void)M;
-    (void)off;
-#endif
-    return true;
-}
 
 struct KernelArgs {
     const void *value;
@@ -174,7 +144,35 @@ struct KernelArgs {
     int dcn;
     int dcn_h, dcn_w, dcn_wo;
     int stride_h, stride_w, pad_h, pad_w, dil_h, dil_w;
+    // backward grad_value merge (see "merged reductions"): queries per tile,
+    // query blocks per batch, hash-table slots (a power of two) and log2
+    int64_t merge_qb, merge_nqb;
+    int merge_tslots, merge_tbits;
+    int *status;            // per-device status word (device address)
 };
+
+// Records a device-side failure code in the status word (msda_status values).
+__device__ __forceinline__ void report(const KernelArgs &a, int code) { atomicExch(a.status, code); }
+
+// Checked build (MSDA_BOUNDS_CHECK): the corner row offset `off` (key * M,
+// relative to the row's (batch, head) slice) that a kernel is about to read
+// or reduce into must lie in [0, S*M); a violation is recorded
+// (MSDA_ERR_DEVICE_BOUNDS = 6) and the access skipped.  By construction the
+// set-up only produces in-range offsets, so a clean run of the checked build
+// is evidence that every access stays inside value / grad_value.
+__device__ __forceinline__ bool row_in_bounds(const KernelArgs &a, int off)
+{
+#if MSDA_BOUNDS_CHECK
+    if (off < 0 || (int64_t)off >= a.S * a.M) {
+        report(a, 6 /* MSDA_ERR_DEVICE_BOUNDS */);
+        return false;
+    }
+#else
+    (void)a;
+    (void)off;
+#endif
+    return true;
+}
 
 struct Geometry {
     int H[kMaxLevels];
@@ -215,7 +213,7 @@ __device__ __forceinline__ bool load_geometry(const KernelArgs &a, Geometry &geo
             good = 0;
         ok = good;
         if (!good)
-            atomicExch(&g_device_status, 4 /* MSDA_ERR_DEVICE_CHECK */);
+            report(a, 4 /* MSDA_ERR_DEVICE_CHECK */);
     }
     __syncthreads();
     return ok != 0;
@@ -477,6 +475,14 @@ __device__ __forceinline__ void st_stream2(float2 *ptr, float2 v, uint64_t pol)
 #endif
 }
 
+// grad_value reduction of one 16-byte chunk: a vector reduction that returns
+// nothing (no wait for the L2 round trip).
+__device__ __forceinline__ void red_add_v4(float4 *p, float4 v)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
+                 :: "l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+}
+
 // 4 consecutive grad_output channels starting at element `e` of a row,
 // widened to float32.
 template <typename T>
@@ -497,11 +503,11 @@ __device__ __forceinline__ float4 ld_grad4<__nv_bfloat16>(const __nv_bfloat16 *r
 
 // ------------------------------------------------------------- scheduling --
 //
-// Persistent grid: one resident wave of CTAs walks the row tiles (see
-// tile_walk for the two walks).
+// Persistent grid: one resident wave of CTAs walks the row tiles grid-stride
+// (tile c, c + gridDim.x, ...).
 //
-// Processing row p maps to memory row (b * Q + q) * M + m; head-major order
-// takes p = (m * B + b) * Q + q; with a query order the p-th query is order[p / M].
+// Processing row p maps to memory row (b * Q + q) * M + m = p in the natural
+// order; with a query order the p-th query is order[p / M].
 
 __device__ __forceinline__ int64_t memory_row(const KernelArgs &a, int64_t p)
 {
@@ -511,20 +517,12 @@ __device__ __forceinline__ int64_t memory_row(const KernelArgs &a, int64_t p)
         const int64_t qi = p / a.M;
         int64_t q = __ldg(a.order + qi);
         if (q < 0 || q * a.M >= a.rows) {
-            atomicExch(&g_device_status, 4 /* MSDA_ERR_DEVICE_CHECK */);
+            report(a, 4 /* MSDA_ERR_DEVICE_CHECK */);
             q = 0;
         }
         return q * a.M + (p - qi * a.M);
     }
-#if MSDA_HEAD_MAJOR
-    const int64_t BQ = a.rows / a.M;
-    const int64_t m = p / BQ;
-    const int64_t bq = p - m * BQ;
-    return bq * a.M + m;
-#else
-    (void)a;
     return p;
-#endif
 }
 
 // ----------------------------------------------------------------- set-up --
@@ -545,24 +543,40 @@ __device__ __forceinline__ int64_t memory_row(const KernelArgs &a, int64_t p)
 
 __host__ __device__ __forceinline__ int record_stride(int P) { return (P & 1) ? P + 2 : P + 1; }
 
-// Non-fused: x = loc_x * W - 0.5 in float64 (the product of a float32 and an
-// integer below 2^16 is exact, so this equals the double-precision formula).
+// Non-fused: x = loc_x * W - 0.5 in float64.  The product of a float32 and
+// an integer below 2^16 is exact in float64, so one fused multiply-add rounds
+// exactly as the double-precision formula (product, then subtraction) does.
 __device__ __forceinline__ void pixel_from_location(float lx, float ly, int H, int W,
                                                     double &x, double &y)
 {
-    x = __dsub_rn(__dmul_rn((double)lx, (double)W), 0.5);
-    y = __dsub_rn(__dmul_rn((double)ly, (double)H), 0.5);
+    x = __fma_rn((double)lx, (double)W, -0.5);
+    y = __fma_rn((double)ly, (double)H, -0.5);
 }
 
-// Fused: loc = ref + off / (W, H) then x = loc * W - 0.5, each operation
-// rounded in float64 exactly as the formula reads.
+// Fused: the formula reads loc = ref + off / W, then x = loc * W - 0.5, each
+// step rounded in float64 (the oracle's chain).  Algebraically x = ref * W +
+// off - 0.5, which the kernel forms with one float64 fused multiply-add and
+// one subtraction, without the division.  For |off| + |ref| * W < 2^20 the two
+// values differ by less than 2^-30 (each chain rounds a few times at 2^-53
+// relative to that magnitude), so they have the same floor and the same
+// order against -1 and W (integers) unless the value lies within 1e-9 of an
+// integer; there, and for larger magnitudes, the formula's own chain is
+// evaluated, so that the corner choice is always that of the float64 formula.
+__device__ __forceinline__ double fused_coord(float r, float o, int W)
+{
+    const double Wd = (double)W;
+    const double x = __dsub_rn(__fma_rn((double)r, Wd, (double)o), 0.5);
+    const double f = x - floor(x);
+    if (f > 1e-9 && f < 1.0 - 1e-9 && fabsf(o) + fabsf(r) * (float)W < 1048576.f)
+        return x;
+    return __dsub_rn(__dmul_rn(__dadd_rn((double)r, __ddiv_rn((double)o, Wd)), Wd), 0.5);
+}
+
 __device__ __forceinline__ void pixel_from_offset(float rx, float ry, float ox, float oy,
                                                   int H, int W, double &x, double &y)
 {
-    double lx = __dadd_rn((double)rx, __ddiv_rn((double)ox, (double)W));
-    double ly = __dadd_rn((double)ry, __ddiv_rn((double)oy, (double)H));
-    x = __dsub_rn(__dmul_rn(lx, (double)W), 0.5);
-    y = __dsub_rn(__dmul_rn(ly, (double)H), 0.5);
+    x = fused_coord(rx, ox, W);
+    y = fused_coord(ry, oy, H);
 }
 
 // DCNv3: sample s = r * kw + c of memory row `row` (= (b * Q + q) * G + g,
@@ -670,6 +684,28 @@ __device__ __forceinline__ void sample_input(const KernelArgs &a, int64_t base, 
 
 // Builds the forward records of one row; lane gl of the group does samples
 // gl, gl + G, ...
+// One forward record: the four corner weights A * w_c (0 outside the map)
+// and the corner rows.
+__device__ __forceinline__ void write_forward_record(const KernelArgs &a, const Geometry &geo, int l,
+                                                     double x, double y, float A, float4 *wa, int4 *off)
+{
+    const Corners c = corners_of(x, y, geo.H[l], geo.W[l], geo.start[l]);
+    const float ay1 = A * c.fy, ay0 = A - ay1;
+    float4 w;
+    w.x = c.in[0] ? ay0 * (1.f - c.fx) : 0.f;
+    w.y = c.in[1] ? ay0 * c.fx : 0.f;
+    w.z = c.in[2] ? ay1 * (1.f - c.fx) : 0.f;
+    w.w = c.in[3] ? ay1 * c.fx : 0.f;
+    *wa = w;
+    *off = c.valid ? make_int4(c.key[0] * a.M, c.key[1] * a.M, c.key[2] * a.M, c.key[3] * a.M)
+                   : make_int4(-1, 0, 0, 0);
+}
+
+// Samples of a row a lane of the fused forward keeps in registers between
+// the softmax statistics and the records (rows of up to kFwdCache * G
+// samples read each logit once and take one expf per sample).
+constexpr int kFwdCache = 4;
+
 template <int G, bool FUSED>
 __device__ __forceinline__ void setup_forward_row(const KernelArgs &a, const Geometry &geo,
                                                   int64_t row, bool active, int gl, uint64_t pol,
@@ -677,6 +713,48 @@ __device__ __forceinline__ void setup_forward_row(const KernelArgs &a, const Geo
 {
     const int P = a.L * a.K;
     const int64_t base = row * P;
+    if constexpr (FUSED) {
+        if (P <= kFwdCache * G) {
+            float z[kFwdCache];
+            float2 o[kFwdCache];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kFwdCache; ++i) {
+                const int s = gl + i * G;
+                const bool on = active && s < P;
+                z[i] = on ? ld_stream(a.logits + base + s, pol) : -INFINITY;
+                o[i] = on ? ld_stream2(reinterpret_cast<const float2 *>(a.off) + base + s, pol)
+                          : make_float2(0.f, 0.f);
+                mx = fmaxf(mx, z[i]);
+            }
+            mx = group_max<G>(mx);
+            float sum = 0.f;
+#pragma unroll
+            for (int i = 0; i < kFwdCache; ++i) {
+                z[i] = (active && gl + i * G < P) ? expf(z[i] - mx) : 0.f;
+                sum += z[i];
+            }
+            sum = group_sum<G>(sum);
+            if (!active)
+                return;
+            const float inv_sum = 1.0f / sum;
+            const float2 r = __ldg(reinterpret_cast<const float2 *>(a.ref) + row / a.M);
+#pragma unroll
+            for (int i = 0; i < kFwdCache; ++i) {
+                const int s = gl + i * G;
+                if (s >= P)
+                    break;
+                const int l = s / a.K;
+                double x, y;
+                pixel_from_offset(r.x, r.y, o[i].x, o[i].y, geo.H[l], geo.W[l], x, y);
+                const float A = z[i] * inv_sum;
+                if (a.attn_out)
+                    st_stream(a.attn_out + base + s, A, pol);
+                write_forward_record(a, geo, l, x, y, A, wa + s, off + s);
+            }
+            return;
+        }
+    }
     float mx = 0.f, inv_sum = 0.f, rx = 0.f, ry = 0.f;
     if (FUSED)
         fused_row_stats<G>(a, row, active, gl, mx, inv_sum, rx, ry);
@@ -690,28 +768,22 @@ __device__ __forceinline__ void setup_forward_row(const KernelArgs &a, const Geo
         sample_input<FUSED>(a, base, s, H, W, mx, inv_sum, rx, ry, pol, x, y, A);
         if (FUSED && a.attn_out)
             st_stream(a.attn_out + base + s, A, pol);
-        const Corners c = corners_of(x, y, H, W, geo.start[l]);
-        const float ay1 = A * c.fy, ay0 = A - ay1;
-        float4 w;
-        w.x = c.in[0] ? ay0 * (1.f - c.fx) : 0.f;
-        w.y = c.in[1] ? ay0 * c.fx : 0.f;
-        w.z = c.in[2] ? ay1 * (1.f - c.fx) : 0.f;
-        w.w = c.in[3] ? ay1 * c.fx : 0.f;
-        wa[s] = w;
-        off[s] = c.valid ? make_int4(c.key[0] * a.M, c.key[1] * a.M, c.key[2] * a.M, c.key[3] * a.M)
-                         : make_int4(-1, 0, 0, 0);
+        write_forward_record(a, geo, l, x, y, A, wa + s, off + s);
     }
 }
 
 // Builds the backward records of one row, padded to Pp >= P samples with
 // inert records (no load, no reduction); lane gl of the group does samples
 // gl, gl + G, ...  For an inactive row every record is inert.  Record of
-// sample s: fa = {fx, fy, A, in-map bits of the four corners}, off = corner
-// rows (key * M) with off.x = -1 when the sample is skipped.
+// sample s: fa = {fx, fy, A, in-map bits of the four corners | tag}, off =
+// corner rows (key * M) with off.x = -1 when the sample is skipped; `tag`
+// (bits 8 and up) is the row's slot in the CTA tile, which the merged
+// reductions use to find the row's grad_output.
 template <int G, bool FUSED>
 __device__ __forceinline__ void setup_backward_row(const KernelArgs &a, const Geometry &geo,
                                                    int64_t row, bool active, int gl, uint64_t pol,
-                                                   int Pp, float4 *fa, int4 *off, float *As)
+                                                   int Pp, float4 *fa, int4 *off, float *As,
+                                                   unsigned tag)
 {
     const int P = a.L * a.K;
     const int64_t base = row * P;
@@ -732,7 +804,7 @@ __device__ __forceinline__ void setup_backward_row(const KernelArgs &a, const Ge
         const Corners c = corners_of(x, y, H, W, geo.start[l]);
         const unsigned bits = (c.in[0] ? 1u : 0u) | (c.in[1] ? 2u : 0u) | (c.in[2] ? 4u : 0u) |
                               (c.in[3] ? 8u : 0u);
-        fa[s] = make_float4(c.fx, c.fy, A, __uint_as_float(bits));
+        fa[s] = make_float4(c.fx, c.fy, A, __uint_as_float(bits | tag));
         off[s] = c.valid ? make_int4(c.key[0] * a.M, c.key[1] * a.M, c.key[2] * a.M, c.key[3] * a.M)
                          : make_int4(-1, 0, 0, 0);
         if (FUSED)
@@ -811,7 +883,7 @@ struct WarpStage {
 // inputs are never staged; bytes of a warp's stages and barriers.
 __host__ __device__ __forceinline__ int stage_cap(bool enabled, int rpw, int P)
 {
-    return (enabled && MSDA_HEAD_MAJOR == 0 && P <= 32 && (P & (P - 1)) == 0) ? ((rpw * P + 3) & ~3) : 0;
+    return (enabled && P <= 32 && (P & (P - 1)) == 0) ? ((rpw * P + 3) & ~3) : 0;
 }
 __host__ __device__ __forceinline__ size_t stage_bytes_per_warp(bool enabled, int rpw, int P)
 {
@@ -834,23 +906,17 @@ __device__ __forceinline__ WarpStage warp_stage(unsigned char *base, int warp, i
     return ws;
 }
 
-// Next tile of this CTA in the banded walk.
-// Tiles of this CTA: a grid-stride walk (c, c + G, c + 2G, ...) or, with
-// MSDA_CONTIGUOUS_TILES, the contiguous run [c*T/G, (c+1)*T/G) of the T tiles
-// (consecutive queries then stay on one SM, where the corner rows they share
-// can hit in L1).  The host launches at most T CTAs.
+// Tiles of this CTA: a grid-stride walk (c, c + G, c + 2G, ...), so that the
+// resident wave sweeps one narrow band of queries at a time and the corner
+// rows it gathers and reduces into stay in L2.  The host launches at most
+// ntiles CTAs.
 struct TileWalk {
     int64_t first, end, step;
 };
 
 __device__ __forceinline__ TileWalk tile_walk(const KernelArgs &a)
 {
-    const int64_t c = blockIdx.x, G = gridDim.x;
-#if MSDA_CONTIGUOUS_TILES
-    return TileWalk{c * a.ntiles / G, (c + 1) * a.ntiles / G, 1};
-#else
-    return TileWalk{c, a.ntiles, G};
-#endif
+    return TileWalk{(int64_t)blockIdx.x, a.ntiles, (int64_t)gridDim.x};
 }
 
 __device__ __forceinline__ bool stage_ok(int64_t prow0, int nv, int P)
@@ -881,8 +947,7 @@ __device__ __forceinline__ void stage_issue(const KernelArgs &a, const WarpStage
 // of round t takes sample (32 t + L) % P of the warp's row (32 t + L) / P, so
 // every input array is read with one contiguous load per round (the loads of
 // up to kWarpSetupRounds rounds are issued together), and the softmax of a row
-// is a reduction over its P lanes (one expf per sample).  Rows of the warp are
-// consecutive processing rows prow0 ..; nrows of them.  (The forward keeps the
+// is a reduction over its P lanes (one expf per sample).  (The forward keeps the
 // per-group set-up: its register budget is spent on gathers in flight, and the
 // warp-wide form measured slower there.)
 
@@ -980,37 +1045,37 @@ __device__ __forceinline__ void warp_sample(const KernelArgs &a, const Geometry 
 constexpr int kWarpSetupRounds = MSDA_WARP_SETUP_ROUNDS;  // rounds whose loads are issued together
 
 // Backward records of the warp's rows (inactive rows and pad slots inert).
-template <bool FUSED>
-__device__ __forceinline__ void setup_backward_warp(const KernelArgs &a, const Geometry &geo,
-                                                    int64_t prow0, int nrows, int lane, uint64_t pol,
-                                                    int Pp, float4 *fa0, int4 *off0, float *As0,
-                                                    int stride, const float2 *sp, const float *sz)
+// row_of(rr) is the memory row of the warp's rr-th row, or -1 when that row
+// is inactive; record k = rr * stride + s; tag0 + (rr << 8) tags the records
+// of row rr with the row's slot in the CTA tile (see setup_backward_row).
+// ROUNDS: rounds whose loads are issued together; nrows <= ROUNDS * 32 / P
+// rows fit one batch of rounds when ROUNDS >= nrows.
+template <bool FUSED, int ROUNDS, typename RowFn>
+__device__ __forceinline__ void setup_backward_warp(const KernelArgs &a, const Geometry &geo, RowFn row_of,
+                                                    int nrows, int lane, uint64_t pol, int Pp, float4 *fa0,
+                                                    int4 *off0, float *As0, int stride, unsigned tag0)
 {
     const int P = a.L * a.K;
     const int per_round = 32 / P;
-    for (int rb = 0; rb < nrows; rb += per_round * kWarpSetupRounds) {
-        WarpIn in[kWarpSetupRounds];
+    for (int rb = 0; rb < nrows; rb += per_round * ROUNDS) {
+        WarpIn in[ROUNDS];
 #pragma unroll
-        for (int t = 0; t < kWarpSetupRounds; ++t) {
+        for (int t = 0; t < ROUNDS; ++t) {
             const int rr = rb + t * per_round + lane / P;
-            const int64_t prow = prow0 + rr;
-            const bool active = rr < nrows && prow < a.rows;
-            const int64_t row = active ? memory_row(a, prow) : 0;
-            in[t] = sp ? warp_load_staged<FUSED>(a, sp, sz, rr * P + lane % P, row, active)
-                       : warp_load<FUSED>(a, row, active, lane % P, P, pol);
+            const int64_t row = rr < nrows ? row_of(rr) : -1;
+            in[t] = warp_load<FUSED>(a, row >= 0 ? row : 0, row >= 0, lane % P, P, pol);
         }
 #pragma unroll
-        for (int t = 0; t < kWarpSetupRounds; ++t) {
+        for (int t = 0; t < ROUNDS; ++t) {
             if (rb + t * per_round >= nrows)
                 break;
             const int rr = rb + t * per_round + lane / P, s = lane % P;
-            const int64_t prow = prow0 + rr;
-            const bool active = rr < nrows && prow < a.rows;
+            const int64_t row = rr < nrows ? row_of(rr) : -1;
+            const bool active = row >= 0;
             int l;
             double x, y;
             float A;
-            const int64_t row = (a.dcn && active) ? memory_row(a, prow) : 0;  // DCN grid point
-            warp_sample<FUSED>(a, geo, in[t], active, row, s, P, l, x, y, A);
+            warp_sample<FUSED>(a, geo, in[t], active, active ? row : 0, s, P, l, x, y, A);
             if (rr >= nrows)
                 continue;
             const int k = rr * stride + s;
@@ -1022,7 +1087,7 @@ __device__ __forceinline__ void setup_backward_warp(const KernelArgs &a, const G
             const Corners c = corners_of(x, y, geo.H[l], geo.W[l], geo.start[l]);
             const unsigned bits = (c.in[0] ? 1u : 0u) | (c.in[1] ? 2u : 0u) | (c.in[2] ? 4u : 0u) |
                                   (c.in[3] ? 8u : 0u);
-            fa0[k] = make_float4(c.fx, c.fy, A, __uint_as_float(bits));
+            fa0[k] = make_float4(c.fx, c.fy, A, __uint_as_float(bits | (tag0 + ((unsigned)rr << 8))));
             off0[k] = c.valid ? make_int4(c.key[0] * a.M, c.key[1] * a.M, c.key[2] * a.M, c.key[3] * a.M)
                               : make_int4(-1, 0, 0, 0);
             if (FUSED)
@@ -1182,7 +1247,7 @@ forward_kernel(const KernelArgs a_in)
             const bool ok = __all_sync(0xffffffffu, mbar_wait(ws.bar + st, (phase >> st) & 1u));
             if (!ok) {
                 if (lane == 0)
-                    atomicExch(&g_device_status, 5 /* MSDA_ERR_DEVICE_TIMEOUT */);
+                    report(a, 5 /* MSDA_ERR_DEVICE_TIMEOUT */);
                 if (next_staged && !a.withhold_copy)
                     mbar_wait(ws.bar + (st ^ 1), (phase >> (st ^ 1)) & 1u);
                 return;
@@ -1222,7 +1287,7 @@ forward_kernel(const KernelArgs a_in)
                         for (int c = 0; c < 4; ++c)
 #pragma unroll
                             for (int j = 0; j < CH; ++j)
-                                v[u][c][j] = row_in_bounds(a.S, a.M, oc[c])
+                                v[u][c][j] = row_in_bounds(a, oc[c])
                                                  ? ld_vec(vbase + (int64_t)oc[c] * Lay::kNvec + j * G)
                                                  : Raw{};
                     }
@@ -1301,7 +1366,94 @@ __device__ __forceinline__ void reduce_scatter3(float (&v)[C][3], int gl)
 // Samples per backward reduce-scatter chunk for G lanes per row.
 template <int G> struct BwdChunk { static constexpr int kC = G < 4 ? G : 4; };
 
-template <typename T, int D, bool FUSED, bool GEN>
+// ------------------------------------------------------ merged reductions --
+//
+// grad_value receives A * w_c * g for every in-map corner of every sample.
+// Neighbouring queries of one head sample largely the same corner rows (on
+// the encoder workloads only about a third of the contributions of 32
+// consecutive queries of one head go to distinct rows), so in the MERGE
+// kernels a CTA tile is one head m of Qb consecutive queries of one batch
+// and the CTA merges the tile's contributions before they reach L2:
+//   1. each warp keeps its rows' grad_output in shared memory and enters the
+//      in-map corners of its records into a shared-memory open-addressing
+//      table keyed by corner row (multiplicative hash, linear probing, slots
+//      claimed with atomicCAS); each contribution is linked into its row's
+//      list with atomicExch on the list head, and a newly claimed slot is
+//      appended to the tile's list of occupied slots;
+//   2. after a CTA barrier, groups of FG lanes take the occupied slots, walk
+//      each list summing A * w_c * g (the weights are recomputed from the
+//      record, the row's grad_output read from shared memory) and reduce the
+//      sum into grad_value with one whole-sector vector reduction per lane;
+//      each walked slot is reset for the next tile;
+//   3. a second barrier closes the tile.
+// The table has at least as many slots as the tile has contributions, so a
+// free slot always exists; the probe loop is bounded all the same, and a
+// contribution that finds no slot is reduced directly.  Contribution ids
+// (record * 4 + corner) and slots are 16-bit; the host sizes tiles so that
+// they fit.
+//
+// Measured on B200, the merge costs more than the L2 reductions it saves
+// (fused backward, direct / merged: encoder float32 270 / 469 us, 1080p K = 8
+// bf16 2045 / 6439 us, DCNv3 7 x 7 bf16 697 / 2711 us): a shared-memory
+// atomic takes about one L1 wavefront per lane, and the list walks are
+// latency-bound between the CTA barriers.  It is therefore an option
+// (MSDA_MERGE_REDUCTIONS); the default reduces each contribution directly.
+
+constexpr int kMergeEmpty = -1;         // free table slot
+constexpr unsigned kMergeEnd = 0xFFFFu;  // end of a contribution list
+
+// Byte offsets of the merge arrays after the records (host and device agree).
+struct MergeLayout {
+    size_t gsm, tkey, thead, occ, next, total;
+};
+
+__host__ __device__ __forceinline__ MergeLayout merge_layout(size_t record_bytes, int64_t rows, int stride,
+                                                            int D, int tslots)
+{
+    MergeLayout m;
+    size_t o = align16(record_bytes);
+    m.gsm = o;      // float32 grad_output rows of the tile [rows][D]
+    o += (size_t)rows * D * 4;
+    m.tkey = o;     // int   [tslots]: corner row (key * M) or kMergeEmpty
+    o += (size_t)tslots * 4;
+    m.thead = o;    // int   [tslots]: first contribution id of the slot's list
+    o += (size_t)tslots * 4;
+    m.occ = o;      // u16   [tslots]: occupied slots in claim order
+    o += align16((size_t)tslots * 2);
+    m.next = o;     // u16   [rows * stride * 4]: next contribution id
+    o += align16((size_t)rows * stride * 4 * 2);
+    m.total = o;
+    return m;
+}
+
+// Enters contribution `id` (record id >> 2, corner id & 3) of corner row
+// `key` into the table; false when no slot was found.
+__device__ __forceinline__ bool merge_insert(int *tkey, int *thead, uint16_t *occ, uint16_t *next, int *nocc,
+                                             int tslots, int tbits, int key, int id)
+{
+    unsigned h = ((unsigned)key * 2654435761u) >> (32 - tbits);
+    for (int probe = 0; probe < tslots; ++probe) {
+        const int prev = atomicCAS(tkey + h, kMergeEmpty, key);
+        if (prev == kMergeEmpty)
+            occ[atomicAdd(nocc, 1)] = (uint16_t)h;
+        if (prev == kMergeEmpty || prev == key) {
+            next[id] = (uint16_t)atomicExch(thead + h, id);
+            return true;
+        }
+        h = (h + 1) & (unsigned)(tslots - 1);
+    }
+    return false;
+}
+
+// --------------------------------------------------------------- backward --
+
+// GEN = false: the plain attention kernel (natural query order, no DCN grid);
+// GEN = true honours KernelArgs::order (without MERGE only) and ::dcn.
+// MERGE = true: a CTA tile is one head of merge_qb consecutive queries of one
+// batch and grad_value contributions are merged per tile (above); MERGE =
+// false: a tile is rows_per_tile consecutive processing rows and every
+// contribution is reduced into grad_value directly.
+template <typename T, int D, bool FUSED, bool GEN, bool MERGE>
 __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, BwdMinCtas<T>::kN)
 backward_kernel(const KernelArgs a_in)
 {
@@ -1309,8 +1461,10 @@ backward_kernel(const KernelArgs a_in)
     if constexpr (!GEN) {
         a.order = nullptr;
         a.dcn = 0;
-        a.stage = 0;
     }
+    if constexpr (MERGE)
+        a.order = nullptr;  // merged tiles follow the natural order (host-checked)
+    a.stage = 0;
     using Lay = Layout<T, D, BwdVB<T>::kVB>;
     using R = typename RowOf<T>::type;  // grad_output element
     using Raw = typename Lay::Raw;
@@ -1322,10 +1476,12 @@ backward_kernel(const KernelArgs a_in)
     constexpr int NR = D / 4 / G;
     static_assert(NR >= 1 && (D / 4) % G == 0, "reduction layout");
     static_assert(EPV % 2 == 0, "pairs");
+    constexpr int RPW = Lay::kRowsPerWarp;
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ Geometry geo;
     __shared__ int geo_ok;
+    __shared__ int nocc[2];
     if (!load_geometry(a, geo, geo_ok))
         return;
 
@@ -1333,79 +1489,78 @@ backward_kernel(const KernelArgs a_in)
     const int Pp = (P + C - 1) / C * C;
     const int stride = record_stride(Pp);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
     const int grp = lane / G, gl = lane % G;
-    const int slot = warp * Lay::kRowsPerWarp + grp;
+    const int slot = warp * RPW + grp;
     const int64_t arr = a.rows_per_tile * stride;  // one record array, in 16-byte units
-    float4 *fa = reinterpret_cast<float4 *>(smem_raw) + slot * stride;
-    int4 *off = reinterpret_cast<int4 *>(reinterpret_cast<float4 *>(smem_raw) + arr) + slot * stride;
+    float4 *fa_all = reinterpret_cast<float4 *>(smem_raw);
+    int4 *off_all = reinterpret_cast<int4 *>(fa_all + arr);
+    float4 *fa = fa_all + slot * stride;
+    int4 *off = off_all + slot * stride;
     // fused: grad_A and A of each sample, kept for the softmax Jacobian.
     // Layout in floats: fa, off: 4 * arr each; gA, As: arr each (10 * arr
     // floats = 40 bytes per record slot, as the host sizes it).
-    float *gA = reinterpret_cast<float *>(reinterpret_cast<float4 *>(smem_raw) + 2 * arr) + slot * stride;
+    float *gA = reinterpret_cast<float *>(fa_all + 2 * arr) + slot * stride;
     float *As = gA + arr;
     const uint64_t pol = stream_policy();
-    constexpr int RPW = Lay::kRowsPerWarp;
-    const int cap = a.order ? 0 : stage_cap(MSDA_BWD_STAGE != 0, RPW, P);
-    const WarpStage ws = warp_stage(smem_raw + align16((size_t)arr * (FUSED ? 40 : 32)), warp,
-                                    blockDim.x >> 5, cap);
-    if (cap) {
-        if (lane == 0) {
-            mbar_init(ws.bar);
-            mbar_init(ws.bar + 1);
+
+    // merge arrays (MERGE only)
+#define MSDA_MERGE_ARRAYS                                                                             \
+    const MergeLayout ml = merge_layout((size_t)arr * (FUSED ? 40 : 32), a.rows_per_tile, stride, D, \
+                                        a.merge_tslots);                                             \
+    float4 *gsm = reinterpret_cast<float4 *>(smem_raw + ml.gsm);                                     \
+    int *tkey = reinterpret_cast<int *>(smem_raw + ml.tkey);                                         \
+    int *thead = reinterpret_cast<int *>(smem_raw + ml.thead);                                       \
+    uint16_t *occ = reinterpret_cast<uint16_t *>(smem_raw + ml.occ);                                 \
+    uint16_t *cnext = reinterpret_cast<uint16_t *>(smem_raw + ml.next);                              \
+    (void)gsm, (void)tkey, (void)thead, (void)occ, (void)cnext;
+    if constexpr (MERGE) {
+        MSDA_MERGE_ARRAYS
+        for (int i = threadIdx.x; i < a.merge_tslots; i += blockDim.x) {
+            tkey[i] = kMergeEmpty;
+            thead[i] = (int)kMergeEnd;
         }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        __syncwarp();
+        if (threadIdx.x == 0)
+            nocc[0] = nocc[1] = 0;
+        __syncthreads();
     }
-    unsigned phase = 0;  // bit st: parity of the next completion of stage st
+
     int k = 0;
-    const TileWalk tw = tile_walk(a);
-    int64_t tile = tw.first;
-    if (cap && tile < tw.end) {
-        const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
-        const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
-        if (stage_ok(p0, nv, P))
-            stage_issue<FUSED>(a, ws, 0, p0, nv, lane, pol);
-    }
-    for (; tile < tw.end; tile += tw.step, ++k) {
-        const int st = k & 1;
-        const int64_t nxt = tile + tw.step;
-        bool next_staged = false;
-        if (cap && nxt < tw.end) {
-            const int64_t p0n = nxt * a.rows_per_tile + warp * RPW;
-            const int nvn = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0n));
-            next_staged = stage_ok(p0n, nvn, P);
-            if (next_staged) {
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                stage_issue<FUSED>(a, ws, st ^ 1, p0n, nvn, lane, pol);
-            }
-        }
-        const int64_t prow = tile * a.rows_per_tile + slot;
-        const bool active = prow < a.rows;
-        const int64_t row = active ? memory_row(a, prow) : prow;
-        const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
-        const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
-        if (cap && stage_ok(p0, nv, P)) {
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(ws.bar + st, (phase >> st) & 1u));
-            if (!ok) {
-                if (lane == 0)
-                    atomicExch(&g_device_status, 5 /* MSDA_ERR_DEVICE_TIMEOUT */);
-                if (next_staged && !a.withhold_copy)
-                    mbar_wait(ws.bar + (st ^ 1), (phase >> (st ^ 1)) & 1u);
-                return;
-            }
-            phase ^= 1u << st;
-            setup_backward_warp<FUSED>(a, geo, p0, RPW, lane, pol, Pp, fa - grp * stride,
-                                       off - grp * stride, As - grp * stride, stride, ws.p + st * cap,
-                                       ws.z + st * cap);
-        } else if (warp_setup_ok(P)) {
-            setup_backward_warp<FUSED>(a, geo, p0, RPW, lane, pol, Pp, fa - grp * stride,
-                                       off - grp * stride, As - grp * stride, stride, nullptr, nullptr);
+    for (int64_t tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x, ++k) {
+        // rows of this warp: row_of(rr) for rr < RPW, -1 when inactive
+        int64_t tb = 0, tm = 0, mrow0 = 0, prow0 = 0;
+        int nact;
+        if constexpr (MERGE) {
+            tm = tile % a.M;
+            const int64_t rest = tile / a.M;
+            const int64_t qblk = rest % a.merge_nqb;
+            tb = rest / a.merge_nqb;
+            const int64_t q0 = qblk * a.merge_qb + warp * RPW;
+            nact = (int)max((int64_t)0, min((int64_t)RPW, (int64_t)a.Q - q0));
+            mrow0 = (tb * a.Q + q0) * a.M + tm;
         } else {
-            setup_backward_row<G, FUSED>(a, geo, row, active, gl, pol, Pp, fa, off, As);
+            prow0 = tile * a.rows_per_tile + warp * RPW;
+            nact = (int)max((int64_t)0, min((int64_t)RPW, a.rows - prow0));
         }
+        auto row_of = [&](int rr) -> int64_t {
+            if (rr >= nact)
+                return -1;
+            return MERGE ? mrow0 + (int64_t)rr * a.M : memory_row(a, prow0 + rr);
+        };
+        const int64_t row0 = row_of(grp);
+        const bool active = row0 >= 0;
+        const int64_t row = active ? row0 : 0;
+        const unsigned tag0 = (unsigned)(warp * RPW) << 8;
+        if (warp_setup_ok(P))
+            setup_backward_warp<FUSED, (RPW < kWarpSetupRounds ? RPW : kWarpSetupRounds)>(
+                a, geo, row_of, RPW, lane, pol, Pp, fa - grp * stride,
+                                       off - grp * stride, As - grp * stride, stride, tag0);
+        else
+            setup_backward_row<G, FUSED>(a, geo, row, active, gl, pol, Pp, fa, off, As,
+                                         tag0 + ((unsigned)grp << 8));
         __syncwarp();
-        const int64_t bq = active ? row / a.M : 0;
-        const int m = active ? (int)(row - bq * a.M) : 0;
+        const int64_t bq = row / a.M;
+        const int m = (int)(row - bq * a.M);
         const int64_t b = bq / a.Q;
         const int64_t rbase = b * a.S * a.M + m;  // (b, key 0, m) row
         const Raw *vbase = reinterpret_cast<const Raw *>(static_cast<const T *>(a.value) + rbase * D) + gl;
@@ -1435,6 +1590,43 @@ backward_kernel(const KernelArgs a_in)
             for (int h = 0; h < NR; ++h)
                 gr[h] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        if constexpr (MERGE) {
+            MSDA_MERGE_ARRAYS
+            // the tile's grad_output rows, then this warp's contributions
+            float4 *gvt = reinterpret_cast<float4 *>(a.grad_value + (tb * a.S * a.M + tm) * D);
+#pragma unroll
+            for (int h = 0; h < NR; ++h)
+                gsm[slot * (D / 4) + h * G + gl] = gr[h];
+            __syncwarp();
+            for (int e = lane; e < nact * Pp; e += 32) {
+                const int rr = e / Pp, s = e - rr * Pp;
+                const int rec = (warp * RPW + rr) * stride + s;
+                const unsigned bits = __float_as_uint(fa_all[rec].w) & 15u;
+                if (!bits)
+                    continue;
+                const int4 o = off_all[rec];
+                const int oc[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (!(bits & (1u << c)))
+                        continue;
+                    if (!merge_insert(tkey, thead, occ, cnext, &nocc[k & 1], a.merge_tslots, a.merge_tbits,
+                                      oc[c], rec * 4 + c) &&
+                        row_in_bounds(a, oc[c])) {
+                        // no slot (never with the host's table size): reduce directly
+                        const float4 r = fa_all[rec];
+                        const float wxy = ((c & 1) ? r.x : 1.f - r.x) * ((c & 2) ? r.y : 1.f - r.y);
+                        const float coef = r.z * wxy;
+                        const float4 *gq = gsm + (warp * RPW + rr) * (D / 4);
+                        for (int f = 0; f < D / 4; ++f) {
+                            const float4 g4 = gq[f];
+                            red_add_v4(gvt + (int64_t)oc[c] * (D / 4) + f,
+                                      make_float4(coef * g4.x, coef * g4.y, coef * g4.z, coef * g4.w));
+                        }
+                    }
+                }
+            }
+        }
         const int64_t base = row * P;
         float dot = 0.f, ref_gx = 0.f, ref_gy = 0.f;  // fused: per-owner partial sums
         float vsc = 1.f;  // INT8 value: the dot products are in quantized units
@@ -1455,7 +1647,7 @@ backward_kernel(const KernelArgs a_in)
 #pragma unroll
                         for (int j = 0; j < CH; ++j) {
                             float f[EPV];
-                            Lay::widen(row_in_bounds(a.S, a.M, oc[c])
+                            Lay::widen(row_in_bounds(a, oc[c])
                                            ? ld_vec(vbase + (int64_t)oc[c] * Lay::kNvec + j * G)
                                            : Raw{},
                                        f);
@@ -1477,23 +1669,25 @@ backward_kernel(const KernelArgs a_in)
                 part[i][0] = w[0] * d[0] + w[1] * d[1] + w[2] * d[2] + w[3] * d[3];
                 part[i][1] = A * (ey * (d[1] - d[0]) + fy * (d[3] - d[2]));
                 part[i][2] = A * (ex * (d[2] - d[0]) + fx * (d[3] - d[1]));
-                // scatter A * w_c * g into grad_value (in-map corners of taken
-                // samples; skipped samples have no in-map bits)
-                const int ocs[4] = {o.x, o.y, o.z, o.w};
+                if constexpr (!MERGE) {
+                    // scatter A * w_c * g into grad_value (in-map corners of
+                    // taken samples; skipped samples have no in-map bits)
+                    const int ocs[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    if (!(inm & (1u << c)))
-                        continue;
-                    const float awc = A * w[c];
-                    if (!row_in_bounds(a.S, a.M, ocs[c]))
-                        continue;
-                    float4 *q = gvbase + (int64_t)ocs[c] * (D / 4);
-                    const float2 ww = make_float2(awc, awc);
+                    for (int c = 0; c < 4; ++c) {
+                        if (!(inm & (1u << c)))
+                            continue;
+                        const float awc = A * w[c];
+                        if (!row_in_bounds(a, ocs[c]))
+                            continue;
+                        float4 *q = gvbase + (int64_t)ocs[c] * (D / 4);
+                        const float2 ww = make_float2(awc, awc);
 #pragma unroll
-                    for (int h = 0; h < NR; ++h) {
-                        const float2 lo = mul2(ww, make_float2(gr[h].x, gr[h].y));
-                        const float2 hi = mul2(ww, make_float2(gr[h].z, gr[h].w));
-                        atomicAdd(q + h * G, make_float4(lo.x, lo.y, hi.x, hi.y));
+                        for (int h = 0; h < NR; ++h) {
+                            const float2 lo = mul2(ww, make_float2(gr[h].x, gr[h].y));
+                            const float2 hi = mul2(ww, make_float2(gr[h].z, gr[h].w));
+                            red_add_v4(q + h * G, make_float4(lo.x, lo.y, hi.x, hi.y));
+                        }
                     }
                 }
             }
@@ -1534,238 +1728,89 @@ backward_kernel(const KernelArgs a_in)
                 }
             }
         }
-        __syncwarp();
-    }
-}
-
-// ----------------------------------------------------------------- helpers --
-
-// Zeroes n4 float4 of `a` and n floats of `b` (grid-stride).
-__global__ void zero_kernel(float4 *a, int64_t n4, float *b, int64_t n)
-{
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride)
-        a[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
-        b[i] = 0.f;
-}
-
-// float32 -> bf16 (round to nearest even), 8 elements per thread step.
-__global__ void f32_to_bf16_kernel(const float4 *src, uint4 *dst, int64_t n8)
-{
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
-        const float4 x = src[2 * i], y = src[2 * i + 1];
-        const float f[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
-        uint4 r;
-        Elem<__nv_bfloat16>::narrow<4>(f, reinterpret_cast<uint32_t *>(&r));
-        dst[i] = r;
-    }
-}
-
-// ------------------------------------------------------ INT8 quantisation --
-//
-// value [B, S, M, D] (float32 or bf16) -> int8 with one symmetric scale per
-// (batch, head): amax = max |value[b, :, m, :]|, scale = amax / 127 (1 when
-// amax = 0), q = value / scale rounded half to even, clipped to +-127.  Three
-// kernels: per-(b, m) absmax (into the scale array as float bits, zeroed by
-// the host), scale = amax / 127 in place, quantise.
-
-// Eight consecutive channels starting at p, widened to float32.
-__device__ __forceinline__ void load8(const float *p, float (&f)[8])
-{
-    const float4 x = __ldg(reinterpret_cast<const float4 *>(p));
-    const float4 y = __ldg(reinterpret_cast<const float4 *>(p) + 1);
-    f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
-    f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
-}
-__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&f)[8])
-{
-    const uint4 r = __ldg(reinterpret_cast<const uint4 *>(p));
-    Elem<__nv_bfloat16>::widen<4>(reinterpret_cast<const uint32_t *>(&r), f);
-}
-
-// CTA blockIdx.x covers (b, m) = blockIdx.x / chunks and the chunk
-// blockIdx.x % chunks of the S keys; one atomicMax per CTA.  |x| >= 0, so the
-// float bit patterns order like the values.
-template <typename T>
-__global__ void __launch_bounds__(256) absmax_kernel(const T *v, int64_t S, int M, int D, int chunks,
-                                                     unsigned *amax)
-{
-    __shared__ float part[8];
-    const int64_t bm = blockIdx.x / chunks;
-    const int64_t chunk = blockIdx.x % chunks;
-    const int64_t b = bm / M, m = bm % M;
-    const int nv = D / 8;
-    const int64_t s0 = S * chunk / chunks, s1 = S * (chunk + 1) / chunks;
-    float mx = 0.f;
-    for (int64_t i = threadIdx.x; i < (s1 - s0) * nv; i += blockDim.x) {
-        const int64_t s = s0 + i / nv;
-        const int j = (int)(i % nv);
-        float f[8];
-        load8(v + ((b * S + s) * M + m) * D + j * 8, f);
+        if constexpr (MERGE) {
+            // every warp's contributions are in the table: reduce one sum per
+            // occupied slot, FG lanes per grad_value row
+            MSDA_MERGE_ARRAYS
+            __syncthreads();
+            const int n = nocc[k & 1];
+            if (threadIdx.x == 0)
+                nocc[(k + 1) & 1] = 0;  // last read in the previous tile, before its second barrier
+            constexpr int FG = (D / 4) < 32 ? (D / 4) : 32, NRF = D / 4 / FG, GPW = 32 / FG;
+            const int fg = lane / FG, fl = lane % FG;
+            float4 *gvt = reinterpret_cast<float4 *>(a.grad_value + (tb * a.S * a.M + tm) * D) + fl;
+            const int limit = (int)(arr * 4);
+            // NCH slots per lane group at a time, their lists walked in step so
+            // that the dependent shared-memory loads of different lists overlap
+            constexpr int NCH = MSDA_MERGE_FLUSH_CHAINS;
+            // (warp-uniform trip count: the __syncwarp below is reached by every lane)
+            for (int jw = warp * GPW * NCH; jw < n; jw += nwarps * GPW * NCH) {
+                const int j0 = jw + fg * NCH;
+                int hs[NCH], id[NCH];
+                float4 acc[NCH][NRF];
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            mx = fmaxf(mx, fabsf(f[e]));
-    }
+                for (int u = 0; u < NCH; ++u) {
+                    hs[u] = j0 + u < n ? occ[j0 + u] : -1;
+                    id[u] = hs[u] >= 0 ? thead[hs[u]] : (int)kMergeEnd;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if ((threadIdx.x & 31) == 0)
-        part[threadIdx.x >> 5] = mx;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
-            mx = fmaxf(mx, part[w]);
-        atomicMax(amax + bm, __float_as_uint(mx));
-    }
-}
-
-__global__ void s8_scale_kernel(float *scale, int64_t n)
-{
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n) {
-        const float amax = scale[i];
-        scale[i] = amax > 0.f ? __fdiv_rn(amax, 127.f) : 1.f;
-    }
-}
-
-// Eight channels per thread step (D is a multiple of 8).
-template <typename T>
-__global__ void quantize_s8_kernel(const T *v, const float *scale, int64_t n8, int64_t S, int M, int D,
-                                   uint2 *q)
-{
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
-        const int64_t row = i * 8 / D;  // (b * S + s) * M + m
-        const int64_t m = row % M, b = row / ((int64_t)S * M);
-        const float sc = __ldg(scale + b * M + m);
-        float f[8];
-        load8(v + i * 8, f);
-        uint32_t w[2] = {0u, 0u};
+                    for (int f = 0; f < NRF; ++f)
+                        acc[u][f] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                for (int guard = 0; guard < limit; ++guard) {
+                    bool more = false;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            int r = __float2int_rn(__fdiv_rn(f[e], sc));  // half to even
-            r = r > 127 ? 127 : (r < -127 ? -127 : r);
-            w[e >> 2] |= ((uint32_t)r & 0xffu) << (8 * (e & 3));
-        }
-        q[i] = make_uint2(w[0], w[1]);
-    }
-}
-
-// ------------------------------------------------------------ query order --
-//
-// Counting sort of each batch's queries by the Morton code of the 64 x 64 cell
-// of [0,1]^2 holding their point, in one kernel: one CTA of 1024 threads per
-// batch counts the queries per cell in shared memory, scans the counts, then
-// hands each query the next slot of its cell.  Each pass reads the batch's
-// points with kSortInFlight loads in flight per thread.
-
-constexpr int kSortCells = 64;  // cells per axis of [0,1]^2
-constexpr int kSortThreads = 1024, kSortInFlight = 8;
-
-__device__ __forceinline__ uint32_t spread_bits6(uint32_t v)  // 6 bits -> even bit positions
-{
-    v &= 63u;
-    v = (v | (v << 4)) & 0x0f0fu;
-    v = (v | (v << 2)) & 0x3333u;
-    v = (v | (v << 1)) & 0x5555u;
-    return v;
-}
-
-__device__ __forceinline__ uint32_t cell_code(float2 p)
-{
-    // fminf / fmaxf map NaN to the other operand, so every point gets a cell
-    const float fx = fminf(fmaxf(p.x * kSortCells, 0.f), kSortCells - 1.f);
-    const float fy = fminf(fmaxf(p.y * kSortCells, 0.f), kSortCells - 1.f);
-    return spread_bits6((uint32_t)fx) | (spread_bits6((uint32_t)fy) << 1);
-}
-
-// Cell codes of the points i0 + j * kSortThreads + t (j < kSortInFlight);
-// ~0u past the end.
-__device__ __forceinline__ void cell_codes(const float2 *p, int64_t Q, int64_t i0, int t,
-                                           uint32_t (&code)[kSortInFlight])
-{
-    float2 v[kSortInFlight];
+                    for (int u = 0; u < NCH; ++u) {
+                        if (id[u] == (int)kMergeEnd)
+                            continue;
+                        more = true;
+                        const float4 r = fa_all[id[u] >> 2];
+                        const int c = id[u] & 3;
+                        const float wxy = ((c & 1) ? r.x : 1.f - r.x) * ((c & 2) ? r.y : 1.f - r.y);
+                        const float coef = r.z * wxy;
+                        const float4 *gq = gsm + (__float_as_uint(r.w) >> 8) * (D / 4) + fl;
 #pragma unroll
-    for (int j = 0; j < kSortInFlight; ++j) {
-        const int64_t i = i0 + (int64_t)j * kSortThreads + t;
-        v[j] = i < Q ? __ldg(p + i) : make_float2(0.f, 0.f);
-    }
+                        for (int f = 0; f < NRF; ++f) {
+                            const float4 g4 = gq[f * FG];
+                            acc[u][f].x = fmaf(coef, g4.x, acc[u][f].x);
+                            acc[u][f].y = fmaf(coef, g4.y, acc[u][f].y);
+                            acc[u][f].z = fmaf(coef, g4.z, acc[u][f].z);
+                            acc[u][f].w = fmaf(coef, g4.w, acc[u][f].w);
+                        }
+                        id[u] = cnext[id[u]];
+                    }
+                    if (!more)
+                        break;
+                }
 #pragma unroll
-    for (int j = 0; j < kSortInFlight; ++j)
-        code[j] = i0 + (int64_t)j * kSortThreads + t < Q ? cell_code(v[j]) : ~0u;
-}
-
-__global__ void __launch_bounds__(kSortThreads) sort_queries_kernel(const float2 *pts, int64_t Q,
-                                                                    int32_t *order)
-{
-    constexpr int kCells = kSortCells * kSortCells;
-    static_assert(kCells == 4 * kSortThreads, "the scan takes 4 counters per thread");
-    __shared__ __align__(16) int cnt[kCells];
-    __shared__ int warp_base[kSortThreads / 32];
-    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
-    const int64_t base = (int64_t)blockIdx.x * Q;  // first query of this batch
-    const float2 *p = pts + base;
-    reinterpret_cast<int4 *>(cnt)[t] = make_int4(0, 0, 0, 0);
-    __syncthreads();
-    for (int64_t i0 = 0; i0 < Q; i0 += (int64_t)kSortThreads * kSortInFlight) {
-        uint32_t code[kSortInFlight];
-        cell_codes(p, Q, i0, t, code);
+                for (int u = 0; u < NCH; ++u) {
+                    if (hs[u] < 0)
+                        continue;
+                    const int key = tkey[hs[u]];
+                    if (row_in_bounds(a, key)) {
 #pragma unroll
-        for (int j = 0; j < kSortInFlight; ++j)
-            if (code[j] != ~0u)
-                atomicAdd(cnt + code[j], 1);
-    }
-    __syncthreads();
-    // exclusive scan of the counters: 4 per thread, warp shuffles, warp totals
-    const int4 c = reinterpret_cast<const int4 *>(cnt)[t];
-    const int own = c.x + c.y + c.z + c.w;
-    int incl = own;
+                        for (int f = 0; f < NRF; ++f)
+                            red_add_v4(gvt + (int64_t)key * (D / 4) + f * FG, acc[u][f]);
+                    }
+                }
+                __syncwarp();  // every lane of the group has read tkey before the reset
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o)
-            incl += y;
-    }
-    if (lane == 31)
-        warp_base[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-        const int tot = warp_base[lane];
-        int x = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o)
-                x += y;
-        }
-        warp_base[lane] = x - tot;
-    }
-    __syncthreads();
-    int4 r;
-    r.x = warp_base[wid] + incl - own;
-    r.y = r.x + c.x;
-    r.z = r.y + c.y;
-    r.w = r.z + c.z;
-    reinterpret_cast<int4 *>(cnt)[t] = r;
-    __syncthreads();
-    for (int64_t i0 = 0; i0 < Q; i0 += (int64_t)kSortThreads * kSortInFlight) {
-        uint32_t code[kSortInFlight];
-        cell_codes(p, Q, i0, t, code);
-#pragma unroll
-        for (int j = 0; j < kSortInFlight; ++j)
-            if (code[j] != ~0u) {
-                const int slot = atomicAdd(cnt + code[j], 1);
-                order[base + slot] = (int32_t)(base + i0 + (int64_t)j * kSortThreads + t);
+                for (int u = 0; u < NCH; ++u)
+                    if (hs[u] >= 0 && fl == 0) {
+                        tkey[hs[u]] = kMergeEmpty;
+                        thead[hs[u]] = (int)kMergeEnd;
+                    }
             }
+            __syncthreads();
+        } else {
+            __syncwarp();
+        }
     }
+#undef MSDA_MERGE_ARRAYS
 }
 
 // Rows per warp of each kernel (the host sizes CTAs and shared memory by it).
 template <typename T, int D> constexpr int forward_rows_per_warp() { return Layout<T, D, FwdTune<T, false>::kVB>::kRowsPerWarp; }
 template <typename T> constexpr bool forward_stages() { return FwdTune<T, false>::kStage; }
-constexpr bool backward_stages() { return MSDA_BWD_STAGE != 0; }
 template <typename T, int D> constexpr int backward_rows_per_warp() { return Layout<T, D, BwdVB<T>::kVB>::kRowsPerWarp; }
 // Record slots of a backward row: L*K rounded up to the reduce-scatter chunk.
 template <typename T, int D> inline int backward_padded_samples(int P)

@@ -7,7 +7,9 @@ started.  msda_backward_noalloc serves them by summing into a float32 buffer
 the library owns.  These tests call it through the C ABI and compare it with
 msda_backward given a caller workspace (the existing path), on two calls in a
 row, so that a buffer left dirty by the first call would show up in the
-second.  This file is collected last on purpose.
+second, and with the fp64 oracle (grad_value against the oracle's rounded to
+bf16, the other gradients at the workload's tolerance, both metrics).  This
+file is collected last on purpose.
 """
 import ctypes
 
@@ -16,7 +18,7 @@ import torch
 
 from scale_deformable_attention_msdeformattn_b200 import _lib
 from scale_deformable_attention_msdeformattn_b200 import workloads as wl
-from tests.gpu_util import TOL, rel_err, upload
+from tests.gpu_util import TOL, assert_close, bf16_round, oracle_nonfused, rel_err, upload
 
 pytestmark = pytest.mark.gpu
 
@@ -70,6 +72,7 @@ def test_noalloc_matches_workspace_backward(spec):
     assert st == 0
     torch.cuda.synchronize()
 
+    _, o_gv, o_gl, o_ga = oracle_nonfused(x)
     for call in range(2):
         gv, gl, ga = _outputs(w, dev)
         st = lib.msda_backward_noalloc(ctypes.byref(prob), *args, _p(gv), _p(gl), _p(ga), _stream())
@@ -79,6 +82,13 @@ def test_noalloc_matches_workspace_backward(spec):
         assert rel_err(gv, ref) <= TOL["bf16"], f"call {call}: grad_value"
         assert rel_err(gl, ref_gl.double().cpu().numpy()) <= TOL[w.dtype], f"call {call}: grad_loc"
         assert rel_err(ga, ref_ga.double().cpu().numpy()) <= TOL[w.dtype], f"call {call}: grad_attn"
+        # against the oracle: grad_value is its float64 sum rounded to bf16 up
+        # to one rounding step (at most 2^-7 of the value), the other
+        # gradients at the workload's bounds
+        assert_close(gv, bf16_round(o_gv), 2.0 ** -7, f"call {call}: grad_value vs rounded oracle",
+                     elem_tol=2.0 ** -7)
+        assert_close(gl, o_gl, TOL[w.dtype], f"call {call}: grad_loc vs oracle")
+        assert_close(ga, o_ga, TOL[w.dtype], f"call {call}: grad_attn vs oracle")
 
     code = ctypes.c_int32(-1)
     assert lib.msda_get_device_status(_stream(), ctypes.byref(code)) == 0 and code.value == 0
