@@ -707,10 +707,18 @@ def _time_e2e(hin, step, make_outputs, flush, n, samples, dev, nev):
 
 # ------------------------------------------------------- the oracle legs --
 
-def _oracle_sample(w: wl.Workload, x: wl.Inputs, stride: int):
-    """Every `stride`-th query of the workload (all levels stay represented),
-    with the full value map: the inputs of a bounded oracle pass."""
-    qs = np.arange(0, w.num_queries, stride)
+def _oracle_sample(w: wl.Workload, x: wl.Inputs, frac: float, block: int = 512):
+    """About `frac` of the workload's queries in contiguous blocks of `block`
+    queries spread evenly over the query axis (all levels stay represented,
+    and each block keeps the access locality of a full pass), with the full
+    value map: the inputs of a bounded oracle pass.  frac >= 1: every query."""
+    Q = w.num_queries
+    if frac >= 1.0 or block >= Q:
+        qs = np.arange(Q)
+    else:
+        nblk = max(1, int(round(frac * Q / block)))
+        starts = np.linspace(0, Q - block, nblk).astype(np.int64)
+        qs = np.unique(np.concatenate([np.arange(s0, s0 + block) for s0 in starts]))
     return {
         "value": x.value_f64(), "grad_output": np.ascontiguousarray(x.grad_output_f64()[:, qs]),
         "spatial_shapes": x.spatial_shapes, "level_start_index": x.level_start_index,
@@ -718,7 +726,19 @@ def _oracle_sample(w: wl.Workload, x: wl.Inputs, stride: int):
         "sampling_offsets": np.ascontiguousarray(x.sampling_offsets[:, qs]),
         "attention_logits": np.ascontiguousarray(x.attention_logits[:, qs]),
         "samples": w.B * len(qs) * w.M * w.L * w.K, "queries": len(qs),
+        "what": ("every query" if len(qs) == Q else
+                 f"{len(qs)} of {Q} queries in contiguous blocks of {block}"),
     }
+
+
+def _sample_fraction(oracle, w: wl.Workload, x: wl.Inputs, seconds: float, passes: int = 3) -> float:
+    """Fraction of the workload's queries whose fused fwd+bwd the oracle runs
+    `passes` times within about `seconds` (one timed probe on a small block)."""
+    probe = _oracle_sample(w, x, min(1.0, 1024 / w.num_queries))
+    t0 = time.perf_counter()
+    _oracle_step(oracle, probe)
+    per_query = (time.perf_counter() - t0) / probe["queries"]
+    return min(1.0, seconds / passes / (per_query * w.num_queries))
 
 
 def _oracle_step(oracle, smp):
@@ -743,11 +763,11 @@ def _cpu_model() -> str:
 
 def cpu_baseline(w: wl.Workload, x: wl.Inputs, seconds: float) -> dict:
     """The fp64 oracle (plain C loops, one thread), fused forward + backward on
-    a bounded sample of the workload, timed on this host's cores."""
+    the whole workload when a few passes fit in `seconds`, else on contiguous
+    blocks of its queries, timed on this host's cores."""
     import oracle
     oracle.build()
-    stride = max(1, int(round(w.num_queries / 2048)))
-    smp = _oracle_sample(w, x, stride)
+    smp = _oracle_sample(w, x, _sample_fraction(oracle, w, x, seconds))
     t0 = time.perf_counter()
     passes = 0
     while True:
@@ -758,9 +778,8 @@ def cpu_baseline(w: wl.Workload, x: wl.Inputs, seconds: float) -> dict:
             break
     rate = smp["samples"] * passes / el
     return {"value": round(rate / 1e9, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"every {stride}th query ({smp['queries']} of {w.num_queries}, "
-                      f"{smp['samples']} samples) x {passes} passes of fused fwd+bwd, "
-                      f"{el:.1f} s", "host_cpus": os.cpu_count(), "cpu_model": _cpu_model(),
+            "sample": f"{smp['what']} ({smp['samples']} samples) x {passes} passes of fused "
+                      f"fwd+bwd, {el:.1f} s", "host_cpus": os.cpu_count(), "cpu_model": _cpu_model(),
             "full_step_ms_extrapolated": round(w.samples / rate * 1e3, 1)}
 
 
@@ -793,8 +812,7 @@ def cpu_baseline_all_cores(w: wl.Workload, x: wl.Inputs, one_thread: dict, secon
     import oracle
     oracle.build()
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    stride = max(1, int(round(w.num_queries / (2048 * max(1, cores // 4)))))
-    smp = _oracle_sample(w, x, stride)
+    smp = _oracle_sample(w, x, min(1.0, _sample_fraction(oracle, w, x, seconds) * cores))
     nq = smp["queries"]
     nproc = max(1, min(cores, nq))
     rate1 = one_thread["value"] * 1e9
@@ -812,9 +830,8 @@ def cpu_baseline_all_cores(w: wl.Workload, x: wl.Inputs, one_thread: dict, secon
     total = sum(n for _, n in res)
     return {"value": round(total / slowest / 1e9, 6), "unit": UNIT, "cores": nproc,
             "kind": "oracle",
-            "sample": f"every {stride}th query ({nq} of {w.num_queries}) split over {nproc} "
-                      f"spawned processes x {passes} passes of fused fwd+bwd, slowest "
-                      f"{slowest:.1f} s"}
+            "sample": f"{smp['what']} split over {nproc} spawned processes x {passes} "
+                      f"passes of fused fwd+bwd, slowest {slowest:.1f} s"}
 
 
 def run_reference(args):
@@ -827,15 +844,10 @@ def run_reference(args):
     oracle.build()
     w = wl.WORKLOADS[args.workload]
     x = wl.generate(w, with_nonfused=False)
-    # size the per-step sample so that warm-up + steps stay within ~2 minutes
-    probe = _oracle_sample(w, x, max(1, w.num_queries // 256))
-    t0 = time.perf_counter()
-    _oracle_step(oracle, probe)
-    per_sample = (time.perf_counter() - t0) / probe["samples"]
-    budget = 120.0 / (args.steps + args.warmup)
-    want = max(64 * w.M * w.L * w.K * w.B, budget / per_sample)
-    stride = max(1, int(np.ceil(w.samples / want)))
-    smp = _oracle_sample(w, x, stride)
+    # size the per-step sample so that warm-up + steps stay within ~2 minutes:
+    # the whole workload when it fits, else contiguous blocks of its queries
+    frac = _sample_fraction(oracle, w, x, 120.0, passes=args.steps + args.warmup)
+    smp = _oracle_sample(w, x, frac)
     for _ in range(args.warmup):
         _oracle_step(oracle, smp)
     t0 = time.perf_counter()
@@ -844,8 +856,7 @@ def run_reference(args):
     el = time.perf_counter() - t0
     rate = smp["samples"] * args.steps / el
     value = rate / 1e9
-    sample = (f"every {stride}th query ({smp['queries']} of {w.num_queries}, {smp['samples']} "
-              f"samples) per step, fused fwd+bwd")
+    sample = f"{smp['what']} ({smp['samples']} samples) per step, fused fwd+bwd"
     result = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,

@@ -49,6 +49,12 @@
  *     B*Q < 2^31;
  *     B*Q*M*L*K < 2^40; B or Q may be 0 (nothing to sample).
  *   - No C++ exception crosses this boundary.
+ *   - Per-device state: on its first call on a device (with that device
+ *     current) the library looks up the device's SM count and the device
+ *     addresses of its status word and of the msda_backward_noalloc buffer,
+ *     and keeps them for the life of the process.  cudaDeviceReset() destroys
+ *     the context those addresses belong to: after a reset of a device, do not
+ *     call the library on that device again in the same process.
  */
 #ifndef MSDA_H_
 #define MSDA_H_
@@ -77,7 +83,10 @@ typedef enum msda_status {
     MSDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
     MSDA_ERR_DEVICE_CHECK = 4,  /* a kernel found inconsistent geometry or a bad query_order entry */
     MSDA_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up waiting for an input copy
-                                   (bounded wait; the call's outputs are invalid) */
+                                   (bounded wait) and read its inputs directly
+                                   instead; a copy that may still be in flight
+                                   is waited for (bounded) before the kernel
+                                   ends */
     MSDA_ERR_DEVICE_BOUNDS = 6  /* checked build only (MSDA_BOUNDS_CHECK): a kernel
                                    found a corner row outside its tensor and
                                    skipped the access */
@@ -128,7 +137,7 @@ typedef enum msda_dtype {
                                           the copy but never issue it, so
                                           their bounded wait runs out and
                                           they report MSDA_ERR_DEVICE_TIMEOUT
-                                          (outputs are then invalid) */
+                                          (and finish on direct loads) */
 
 /* Sizes of one call.  S = sum_l H_l * W_l. */
 typedef struct msda_problem {
@@ -258,8 +267,9 @@ MSDA_API msda_status msda_zero_grads(const msda_problem *problem, float *grad_va
  * pages on the operator have no counterpart of this entry point; it is an
  * interface convenience of this library.
  *   Arguments: as msda_backward, without the workspace; grad_value is
- *   [B, S, M, D] bf16 (overwritten).  problem->flags may be 0 or
- *   MSDA_GRAD_VALUE_BF16 (the output is bf16 either way).
+ *   [B, S, M, D] bf16 (overwritten).  problem->flags may hold
+ *   MSDA_GRAD_VALUE_BF16 (the output is bf16 either way) and
+ *   MSDA_MERGE_REDUCTIONS, nothing else.
  *   Scratch: the float32 sums are kept in one buffer owned by the library,
  *   4 Mi floats (16 MiB) per GPU, held until the process exits.  Problems with
  *   B*S*M*D > 4 * 2^20 are rejected with MSDA_ERR_UNSUPPORTED before anything
@@ -267,7 +277,9 @@ MSDA_API msda_status msda_zero_grads(const msda_problem *problem, float *grad_va
  *   allocating library routine.
  *   The first call on a device looks up the buffer's device address (a CUDA
  *   runtime query, once per device, with that device current); make that
- *   first call before any stream capture.
+ *   first call before any stream capture.  The address is kept until the
+ *   process exits: after cudaDeviceReset() of the device it is stale (see
+ *   "Per-device state" above).
  *   Every call on a device shares the one buffer and clears it before use:
  *   calls that overlap on the GPU (different streams, no ordering between
  *   them) race on it and give wrong results.  Serialize them.

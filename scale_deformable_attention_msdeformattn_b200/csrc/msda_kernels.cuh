@@ -822,8 +822,10 @@ __device__ __forceinline__ void setup_backward_row(const KernelArgs &a, const Ge
 // A copy needs 16-byte aligned source and size: a warp slice qualifies when
 // (first row * P) and (rows * P) are multiples of 4; other slices (ragged
 // tails) and other P read global memory directly.  Waits are bounded: after
-// kStageSpinLimit polls the kernel records MSDA_ERR_DEVICE_TIMEOUT (5), gives
-// its other copy in flight a bounded chance to land, and returns.
+// kStageSpinLimit polls the kernel records MSDA_ERR_DEVICE_TIMEOUT (5), stops
+// staging and reads the rest of its inputs directly; before the CTA exits it
+// waits (bounded again) for every copy it issued and has not seen complete,
+// so that no copy is left writing the shared memory of a finished CTA.
 
 constexpr int kStageSpinLimit = 1 << 22;
 
@@ -1215,27 +1217,32 @@ forward_kernel(const KernelArgs a_in)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         __syncwarp();
     }
-    unsigned phase = 0;  // bit st: parity of the next completion of stage st
+    unsigned phase = 0;    // bit st: parity of the next completion of stage st
+    unsigned pending = 0;  // bit st: a copy into stage st was issued and not yet seen complete
+    bool live = cap != 0;  // staging on; off after a wait ran out
     int k = 0;
     const TileWalk tw = tile_walk(a);
     int64_t tile = tw.first;
-    if (cap && tile < tw.end) {
+    if (live && tile < tw.end) {
         const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
         const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
-        if (stage_ok(p0, nv, P))
+        if (stage_ok(p0, nv, P)) {
             stage_issue<FUSED>(a, ws, 0, p0, nv, lane, pol);
+            if (!a.withhold_copy)
+                pending |= 1u;
+        }
     }
     for (; tile < tw.end; tile += tw.step, ++k) {
         const int st = k & 1;
         const int64_t nxt = tile + tw.step;
-        bool next_staged = false;
-        if (cap && nxt < tw.end) {
+        if (live && nxt < tw.end) {
             const int64_t p0n = nxt * a.rows_per_tile + warp * RPW;
             const int nvn = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0n));
-            next_staged = stage_ok(p0n, nvn, P);
-            if (next_staged) {
+            if (stage_ok(p0n, nvn, P)) {
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 stage_issue<FUSED>(a, ws, st ^ 1, p0n, nvn, lane, pol);
+                if (!a.withhold_copy)
+                    pending |= 1u << (st ^ 1);
             }
         }
         const int64_t prow = tile * a.rows_per_tile + slot;
@@ -1243,21 +1250,26 @@ forward_kernel(const KernelArgs a_in)
         const int64_t row = active ? memory_row(a, prow) : prow;
         const int64_t p0 = tile * a.rows_per_tile + warp * RPW;
         const int nv = (int)max((int64_t)0, min((int64_t)RPW, a.rows - p0));
-        if (cap && stage_ok(p0, nv, P)) {
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(ws.bar + st, (phase >> st) & 1u));
-            if (!ok) {
+        bool staged = false;
+        if (live && stage_ok(p0, nv, P)) {
+            staged = __all_sync(0xffffffffu, mbar_wait(ws.bar + st, (phase >> st) & 1u));
+            if (staged) {
+                pending &= ~(1u << st);
+                phase ^= 1u << st;
+            } else {
+                // the copy did not land in time: report it, stop staging and
+                // read the inputs directly from here on (the copies still in
+                // flight are waited for before the CTA exits)
                 if (lane == 0)
                     report(a, 5 /* MSDA_ERR_DEVICE_TIMEOUT */);
-                if (next_staged && !a.withhold_copy)
-                    mbar_wait(ws.bar + (st ^ 1), (phase >> (st ^ 1)) & 1u);
-                return;
+                live = false;
             }
-            phase ^= 1u << st;
+        }
+        if (staged)
             setup_forward_staged<FUSED>(a, geo, p0, RPW, lane, pol, wa - grp * stride, off - grp * stride,
                                         stride, ws.p + st * cap, ws.z + st * cap);
-        } else {
+        else
             setup_forward_row<G, FUSED>(a, geo, row, active, gl, pol, wa, off);
-        }
         __syncwarp();
         if (active) {
             const int64_t bq = row / a.M;
@@ -1332,6 +1344,11 @@ forward_kernel(const KernelArgs a_in)
         }
         __syncwarp();
     }
+    // no copy may still be writing this CTA's shared memory when it exits:
+    // after a time-out, wait (bounded) for the copies issued and not yet seen
+    for (int st = 0; st < 2; ++st)
+        if (pending & (1u << st))
+            mbar_wait(ws.bar + st, (phase >> st) & 1u);
 }
 
 // --------------------------------------------------------------- backward --
