@@ -61,10 +61,14 @@ def _load():
             DD = ctypes.POINTER(_DcnDims)
             lib.msda_oracle_dcn_forward.argtypes = [DD, P, P, P, P]
             lib.msda_oracle_dcn_backward.argtypes = [DD, P, P, P, P, P, P, P]
+            I = ctypes.c_int64
+            lib.msda_oracle_linear.argtypes = [I, I, I, P, P, P, P]
+            lib.msda_oracle_linear_backward.argtypes = [I, I, I, P, P, P, P, P, P]
             for f in ("msda_oracle_forward", "msda_oracle_backward", "msda_oracle_sampling_locations",
                       "msda_oracle_softmax", "msda_oracle_fused_chain",
                       "msda_oracle_quantize_value_s8", "msda_oracle_dcn_forward",
-                      "msda_oracle_dcn_backward"):
+                      "msda_oracle_dcn_backward", "msda_oracle_linear",
+                      "msda_oracle_linear_backward"):
                 getattr(lib, f).restype = None
             _lib = lib
     return _lib
@@ -237,3 +241,60 @@ def dcn_backward(x, offset, mask, grad_y, kernel, stride=(1, 1), pad=(0, 0), dil
     _load().msda_oracle_dcn_backward(ctypes.byref(d), _p(xv), _p(off), _p(m), _p(gy), _p(gx),
                                      _p(goff), _p(gm))
     return gx, goff, gm
+
+
+# ------------------------------------------------ the module's dense layers --
+
+def linear(x, weight, bias=None):
+    """y = x @ weight^T + bias in float64 (nn.Linear's convention): x [..., K],
+    weight [N, K], bias [N] or None; returns [..., N].  The module's value and
+    output projections and its query head (discosf.com §2.2, §3.1;
+    cf-1.com §3.2)."""
+    x, w = _f64(x), _f64(weight)
+    K = x.shape[-1]
+    N = w.shape[0]
+    assert w.shape == (N, K)
+    rows = int(np.prod(x.shape[:-1]))
+    b = _f64(bias) if bias is not None else None
+    y = np.empty(x.shape[:-1] + (N,), np.float64)
+    _load().msda_oracle_linear(rows, K, N, _p(x), _p(w), _p(b) if b is not None else None, _p(y))
+    return y
+
+
+def linear_backward(x, weight, grad_y):
+    """(grad_x, grad_weight, grad_bias) of linear() for an upstream grad_y."""
+    x, w, gy = _f64(x), _f64(weight), _f64(grad_y)
+    K, N = x.shape[-1], w.shape[0]
+    rows = int(np.prod(x.shape[:-1]))
+    gx = np.empty_like(x)
+    gw = np.empty((N, K), np.float64)
+    gb = np.empty(N, np.float64)
+    _load().msda_oracle_linear_backward(rows, K, N, _p(x), _p(w), _p(gy), _p(gx), _p(gw), _p(gb))
+    return gx, gw, gb
+
+
+def query_head(query, weight, bias, reference_points, spatial_shapes, M: int, L: int, K: int):
+    """The query head as the pages compose it (cf-1.com §3.2): one linear
+    layer to 3*M*L*K outputs, the first 2*M*L*K the sampling offsets in level
+    pixels in [M, L, K, 2] order, the last M*L*K the attention logits in
+    [M, L*K] order; then locations = ref + offsets / (W_l, H_l) and the
+    softmax over each (b, q, m)'s L*K logits.  query [B, Q, C].
+    Returns (sampling_locations [B,Q,M,L,K,2], attention_weights [B,Q,M,L,K])."""
+    y = linear(query, weight, bias)
+    B, Q = y.shape[0], y.shape[1]
+    P = M * L * K
+    assert y.shape[2] == 3 * P
+    off = np.ascontiguousarray(y[:, :, :2 * P]).reshape(B, Q, M, L, K, 2)
+    logits = np.ascontiguousarray(y[:, :, 2 * P:]).reshape(B, Q, M, L * K)
+    return sampling_locations(spatial_shapes, reference_points, off), softmax(logits, L, K)
+
+
+def query_head_backward(spatial_shapes, attention_weights, grad_loc, grad_attn):
+    """Gradient of the query head's linear outputs [B, Q, 3*M*L*K] (offsets
+    then logits, the weight's row order) and of the reference points
+    [B, Q, 2], from the core's grad_sampling_locations and
+    grad_attention_weights: the chain rule of query_head's location and
+    softmax steps (fused_chain)."""
+    goff, gref, glog = fused_chain(spatial_shapes, attention_weights, grad_loc, grad_attn, True)
+    B, Q = goff.shape[0], goff.shape[1]
+    return np.concatenate([goff.reshape(B, Q, -1), glog.reshape(B, Q, -1)], axis=2), gref

@@ -453,3 +453,53 @@ void msda_oracle_dcn_backward(const dcn_dims *d, const double *x, const double *
         }
     }
 }
+
+/*
+ * Dense layer of the module around the operator: the value projection W'_m
+ * and the output projection W_m of the formula ([discosf] §2.2, §3.1) and the
+ * query head that predicts the sampling offsets and attention logits
+ * ([cf-1] §3.2; [discosf] §3.1).  nn.Linear's convention:
+ *   y[r, n] = sum_k x[r, k] * w[n, k] + b[n]      (b may be NULL)
+ * x [rows, K], w [N, K], y [rows, N].
+ */
+void msda_oracle_linear(int64_t rows, int64_t K, int64_t N, const double *x, const double *w,
+                        const double *b, double *y)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t n = 0; n < N; ++n) {
+            double s = b ? b[n] : 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                s += x[r * K + k] * w[n * K + k];
+            y[r * N + n] = s;
+        }
+}
+
+/*
+ * Its exact derivative for an upstream gradient gy [rows, N]:
+ *   gx[r, k] = sum_n gy[r, n] * w[n, k]
+ *   gw[n, k] = sum_r gy[r, n] * x[r, k]
+ *   gb[n]    = sum_r gy[r, n]
+ */
+void msda_oracle_linear_backward(int64_t rows, int64_t K, int64_t N, const double *x, const double *w,
+                                 const double *gy, double *gx, double *gw, double *gb)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                s += gy[r * N + n] * w[n * K + k];
+            gx[r * K + k] = s;
+        }
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t r = 0; r < rows; ++r)
+                s += gy[r * N + n] * x[r * K + k];
+            gw[n * K + k] = s;
+        }
+        double s = 0.0;
+        for (int64_t r = 0; r < rows; ++r)
+            s += gy[r * N + n];
+        gb[n] = s;
+    }
+}

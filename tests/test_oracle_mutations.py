@@ -15,6 +15,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_dcn as dcn_pins
+from tests import test_oracle_linear as linear_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "msda_oracle.c")
@@ -67,6 +68,14 @@ DCN_MUTATIONS = {
                            "const double py = (double)(i - d->pad_h + r * d->dil_h) + dp[1];"),
 }
 
+# mistakes in the dense layer and the query head, caught by their own pins
+LINEAR_MUTATIONS = {
+    "linear_weight_transposed": ("s += x[r * K + k] * w[n * K + k];", "s += x[r * K + k] * w[(k * N + n) % (N * K)];"),
+    "linear_bias_dropped": ("double s = b ? b[n] : 0.0;", "double s = 0.0;"),
+    "linear_grad_x_row_of_w": ("s += gy[r * N + n] * w[n * K + k];", "s += gy[r * N + n] * w[(k * N + n) % (N * K)];"),
+    "linear_grad_w_from_gx": ("s += gy[r * N + n] * x[r * K + k];", "s += gy[r * N + n] * gx[r * K + k];"),
+}
+
 PIN_CHECKS = [
     pins.test_golden_worked_bilinear,
     pins.test_golden_worked_two_level_fused,
@@ -89,6 +98,15 @@ DCN_PIN_CHECKS = [
 ]
 
 
+LINEAR_PIN_CHECKS = [
+    linear_pins.test_golden_worked_linear,
+    linear_pins.test_identity_and_zero_weights,
+    linear_pins.test_adjoint_identities,
+    linear_pins.test_query_head_column_order,
+    linear_pins.test_query_head_backward_central_differences,
+]
+
+
 @contextlib.contextmanager
 def _swapped(lib_path):
     oracle._load()
@@ -96,7 +114,7 @@ def _swapped(lib_path):
     lib = ctypes.CDLL(lib_path)
     for name in ("msda_oracle_forward", "msda_oracle_backward", "msda_oracle_sampling_locations",
                  "msda_oracle_softmax", "msda_oracle_fused_chain", "msda_oracle_dcn_forward",
-                 "msda_oracle_dcn_backward"):
+                 "msda_oracle_dcn_backward", "msda_oracle_linear", "msda_oracle_linear_backward"):
         f, ref = getattr(lib, name), getattr(saved, name)
         f.argtypes, f.restype = ref.argtypes, ref.restype
     oracle._lib = lib
@@ -106,10 +124,14 @@ def _swapped(lib_path):
         oracle._lib = saved
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(DCN_MUTATIONS))
+ALL_MUTATIONS = {**MUTATIONS, **DCN_MUTATIONS, **LINEAR_MUTATIONS}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(DCN_MUTATIONS) + sorted(LINEAR_MUTATIONS))
 def test_planted_mistake_is_caught(name, tmp_path):
-    old, new = MUTATIONS[name] if name in MUTATIONS else DCN_MUTATIONS[name]
-    checks = PIN_CHECKS if name in MUTATIONS else DCN_PIN_CHECKS
+    old, new = ALL_MUTATIONS[name]
+    checks = (PIN_CHECKS if name in MUTATIONS else
+              DCN_PIN_CHECKS if name in DCN_MUTATIONS else LINEAR_PIN_CHECKS)
     src = open(SRC).read()
     assert src.count(old) == 1, name
     mutated = tmp_path / "mut.c"
