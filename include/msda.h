@@ -395,6 +395,80 @@ MSDA_API msda_status msda_dcn_backward(const msda_dcn_problem *problem, const vo
 MSDA_API msda_status msda_dcn_backward_workspace_size(const msda_dcn_problem *problem,
                                                       size_t *bytes);
 
+/* ------------------------------------------------------------------------
+ * Dense layers around the operator, on the tensor cores (tcgen05, sm_100a).
+ *
+ * The module the pages build around the core (discosf.com/news/5175395
+ * §2.2 and §3.1; cf-1.com/news/4799680 §3.1-3.2) has four linear layers: the
+ * value projection W'_m (value_proj), the sampling-offset and attention-
+ * weight heads that read the query, and the output projection W_m
+ * (output_proj).  These entry points run them with bf16 operands and
+ * float32 accumulation; the layer weights use nn.Linear's layout
+ * [out_features, in_features] (row-major, in_features contiguous).
+ * ------------------------------------------------------------------------ */
+
+/*
+ * out[r, n] = sum_k x[r, k] * weight[n, k] + bias[n], r < rows, n < out_features.
+ *   x       [rows, in_features] bf16, device, 16-byte aligned
+ *   weight  [out_features, in_features] bf16, device, 16-byte aligned
+ *   bias    [out_features] float32 or NULL
+ *   out     [rows, out_features] in out_dtype (MSDA_F32 or MSDA_BF16),
+ *           16-byte aligned.  With MSDA_BF16 output and out_features = M*D,
+ *           value_proj writes the operator's value tensor [B, S, M, D]
+ *           directly (rows = B*S).
+ *   in_features and out_features >= 8 and multiples of 8 (16-byte rows for
+ *   the tensor-memory copies); rows < 2^31; out_features < 2^20.
+ * Errors: MSDA_ERR_INVALID_ARG (null / misaligned pointer, bad size or
+ * dtype), MSDA_ERR_CUDA (launch or tensor-map set-up failed).  A kernel that
+ * gives up a bounded wait records MSDA_ERR_DEVICE_TIMEOUT in the status word.
+ */
+MSDA_API msda_status msda_linear(int64_t rows, int32_t in_features, int32_t out_features,
+                                 const void *x, const void *weight, const float *bias,
+                                 void *out, int32_t out_dtype, msda_stream_t stream);
+
+/*
+ * The query-side head: one linear layer from the query to the 3*M*L*K
+ * outputs the module's two heads predict (cf-1.com/news/4799680 §3.2:
+ * 2*M*L*K sampling offsets, M*L*K attention logits), fused with the steps
+ * that turn them into the core's inputs: sampling locations
+ * loc = ref + off / (W_l, H_l) and attention weights A = softmax over the
+ * L*K logits of each (b, q, m).  The offsets and logits are never written.
+ *   problem      sizes (B, Q, M, L, K; S, D and value_dtype unused)
+ *   query        [B, Q, in_features] bf16
+ *   weight       [3*M*L*K, in_features] bf16: rows 0 .. 2P-1 are the offset
+ *                head in the core's [M, L, K, 2] order, rows 2P .. 3P-1 the
+ *                logit head in [M, L*K] order (P = M*L*K)
+ *   bias         [3*M*L*K] float32 or NULL
+ *   reference_points [B, Q, 2] float32 (normalized)
+ *   spatial_shapes   [L, 2] int64 (H, W), device
+ *   sampling_locations [B, Q, M, L, K, 2] float32, attention_weights
+ *                [B, Q, M, L, K] float32: outputs, the core's layouts
+ *   Needs L*K a power of two of at most 32 and M*L*K a multiple of 32;
+ *   in_features as for msda_linear.
+ */
+MSDA_API msda_status msda_query_head(const msda_problem *problem, int32_t in_features,
+                                     const void *query, const void *weight, const float *bias,
+                                     const float *reference_points, const int64_t *spatial_shapes,
+                                     float *sampling_locations, float *attention_weights,
+                                     msda_stream_t stream);
+
+/*
+ * Backward of msda_query_head's location and softmax step: from the core's
+ * grad_sampling_locations [B, Q, M, L, K, 2] and grad_attention_weights
+ * [B, Q, M, L, K] (and the attention weights the forward produced) it
+ * writes grad_head [B, Q, 3*M*L*K] float32, the gradient of the head's
+ * linear outputs in the weight's row order: grad_loc / (W_l, H_l) for the
+ * offsets, A_j (gA_j - sum_i A_i gA_i) over each run of L*K for the logits.
+ * grad_reference_points [B, Q, 2] (sum of grad_loc over the query's
+ * samples) is written when not NULL.  Same size limits as msda_query_head.
+ */
+MSDA_API msda_status msda_query_head_backward(const msda_problem *problem,
+                                              const float *attention_weights,
+                                              const float *grad_sampling_locations,
+                                              const float *grad_attention_weights,
+                                              const int64_t *spatial_shapes, float *grad_head,
+                                              float *grad_reference_points, msda_stream_t stream);
+
 /*
  * Synchronizes `stream`, then returns in *code the status the kernels recorded
  * on the current device since the last call (MSDA_OK, MSDA_ERR_DEVICE_CHECK,

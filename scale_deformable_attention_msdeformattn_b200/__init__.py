@@ -20,8 +20,11 @@ from .binding import (  # noqa: F401
     forward,
     fused_backward,
     fused_forward,
+    linear,
     ms_deform_attn,
     quantize_value_s8,
+    query_head,
+    query_head_backward,
     sort_queries,
     version,
     zero_grads,

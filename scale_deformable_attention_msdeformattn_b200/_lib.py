@@ -85,6 +85,9 @@ _SIGNATURES = {
     "msda_dcn_forward": [_DCN, _P, _P, _P, _P, _P],
     "msda_dcn_backward": [_DCN, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "msda_dcn_backward_workspace_size": [_DCN, ctypes.POINTER(ctypes.c_size_t)],
+    "msda_linear": [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, _P, _P, _P, ctypes.c_int32, _P],
+    "msda_query_head": [_PROB, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P],
+    "msda_query_head_backward": [_PROB, _P, _P, _P, _P, _P, _P, _P],
     "msda_get_device_status": [_P, ctypes.POINTER(ctypes.c_int32)],
     "msda_status_string": [ctypes.c_int],
     "msda_version": [],

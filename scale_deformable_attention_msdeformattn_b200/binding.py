@@ -435,6 +435,97 @@ def dcn_backward(input, offset, mask, grad_output, kernel=3, stride=1, pad=1, di
     return grad_input, goff, gmask
 
 
+# ------------------------------------------------ dense layers (tcgen05) --
+
+def linear(x: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None,
+           out: Optional[torch.Tensor] = None, out_dtype=torch.float32) -> torch.Tensor:
+    """msda_linear: x [..., K] bf16 @ weight[N, K]^T (+ bias [N] float32) on the
+    tensor cores, float32 accumulation; returns [..., N] in out_dtype (float32
+    or bfloat16).  K must be a multiple of 8."""
+    if x.dtype != torch.bfloat16 or weight.dtype != torch.bfloat16:
+        raise TypeError("x and weight must be bfloat16")
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    N, K = weight.shape
+    if x.shape[-1] != K:
+        raise ValueError(f"x has {x.shape[-1]} features, weight expects {K}")
+    dev = x.device
+    _need(x, "x", torch.bfloat16, None, dev)
+    _need(weight, "weight", torch.bfloat16, (N, K), dev)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (N,), dev)
+    rows = x.numel() // K if K else 0
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=out_dtype, device=dev)
+    _need(out, "out", out_dtype, tuple(x.shape[:-1]) + (N,), dev)
+    st = _lib.load().msda_linear(rows, K, N, _ptr(x), _ptr(weight), _ptr(bias), _ptr(out),
+                                 _DTYPES[out_dtype], _stream())
+    _check(st, "msda_linear")
+    return out
+
+
+def _head_problem(B, Q, M, L, K):
+    return _lib.Problem(B, 0, Q, M, 0, L, K, _lib.MSDA_F32, 0)
+
+
+def query_head(query: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor],
+               reference_points: torch.Tensor, spatial_shapes: torch.Tensor, num_heads: int,
+               num_points: int, sampling_locations: Optional[torch.Tensor] = None,
+               attention_weights: Optional[torch.Tensor] = None):
+    """msda_query_head: the offset / logit head (weight [3*M*L*K, C] bf16, rows
+    in [offsets (M, L, K, 2) | logits (M, L*K)] order) fused with the location
+    step and the softmax.  query [B, Q, C] bf16.  Returns
+    (sampling_locations [B,Q,M,L,K,2], attention_weights [B,Q,M,L,K])."""
+    if query.dtype != torch.bfloat16 or weight.dtype != torch.bfloat16:
+        raise TypeError("query and weight must be bfloat16")
+    B, Q, C = query.shape
+    L = spatial_shapes.shape[0]
+    M, K = num_heads, num_points
+    P = M * L * K
+    dev = query.device
+    _need(query, "query", torch.bfloat16, (B, Q, C), dev)
+    _need(weight, "weight", torch.bfloat16, (3 * P, C), dev)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (3 * P,), dev)
+    _need(reference_points, "reference_points", torch.float32, (B, Q, 2), dev)
+    _need(spatial_shapes, "spatial_shapes", torch.int64, (L, 2), dev)
+    loc = sampling_locations if sampling_locations is not None else \
+        torch.empty((B, Q, M, L, K, 2), dtype=torch.float32, device=dev)
+    attn = attention_weights if attention_weights is not None else \
+        torch.empty((B, Q, M, L, K), dtype=torch.float32, device=dev)
+    _need(loc, "sampling_locations", torch.float32, (B, Q, M, L, K, 2), dev)
+    _need(attn, "attention_weights", torch.float32, (B, Q, M, L, K), dev)
+    prob = _head_problem(B, Q, M, L, K)
+    st = _lib.load().msda_query_head(ctypes.byref(prob), C, _ptr(query), _ptr(weight), _ptr(bias),
+                                     _ptr(reference_points), _ptr(spatial_shapes), _ptr(loc),
+                                     _ptr(attn), _stream())
+    _check(st, "msda_query_head")
+    return loc, attn
+
+
+def query_head_backward(attention_weights: torch.Tensor, grad_sampling_locations: torch.Tensor,
+                        grad_attention_weights: torch.Tensor, spatial_shapes: torch.Tensor,
+                        want_grad_reference_points: bool = False):
+    """msda_query_head_backward: (grad_head [B, Q, 3*M*L*K] float32, the
+    gradient of the head's linear outputs; grad_reference_points [B, Q, 2] or
+    None)."""
+    B, Q, M, L, K = attention_weights.shape
+    P = M * L * K
+    dev = attention_weights.device
+    _need(attention_weights, "attention_weights", torch.float32, (B, Q, M, L, K), dev)
+    _need(grad_sampling_locations, "grad_sampling_locations", torch.float32, (B, Q, M, L, K, 2), dev)
+    _need(grad_attention_weights, "grad_attention_weights", torch.float32, (B, Q, M, L, K), dev)
+    _need(spatial_shapes, "spatial_shapes", torch.int64, (L, 2), dev)
+    gh = torch.empty((B, Q, 3 * P), dtype=torch.float32, device=dev)
+    gref = torch.empty((B, Q, 2), dtype=torch.float32, device=dev) if want_grad_reference_points else None
+    prob = _head_problem(B, Q, M, L, K)
+    st = _lib.load().msda_query_head_backward(ctypes.byref(prob), _ptr(attention_weights),
+                                              _ptr(grad_sampling_locations), _ptr(grad_attention_weights),
+                                              _ptr(spatial_shapes), _ptr(gh), _ptr(gref), _stream())
+    _check(st, "msda_query_head_backward")
+    return gh, gref
+
+
 def sort_queries(points: torch.Tensor, query_order: Optional[torch.Tensor] = None) -> torch.Tensor:
     """msda_sort_queries: int32 [B*Q] order of the queries by batch, then by
     the Morton code of the 64 x 64 cell of [0,1]^2 holding points[b, q]

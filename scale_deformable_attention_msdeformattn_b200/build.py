@@ -23,8 +23,12 @@ LIB = os.path.join(PKG, "libmsda.so")
 CHECKED = os.path.join(PKG, "libmsda_checked.so")  # MSDA_BOUNDS_CHECK=1 variant (tests)
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# -static-global-template-stub=false: msda_api.cu launches kernel templates
+# that other units instantiate (extern template), which whole-program mode
+# supports only with non-static template stubs
 COMPILE_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
-                 "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]
+                 "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
+                 "-static-global-template-stub=false"]
 LINK_FLAGS = ["-shared", "-Xcompiler", "-fPIC"]
 
 

@@ -8,7 +8,10 @@
 // per-CTA budget.
 #include "msda.h"
 #include "msda_aux.cuh"
+#include "msda_gemm.cuh"
 #include "msda_instances.cuh"
+
+#include <cudaTypedefs.h>
 
 #include <mutex>
 
@@ -569,6 +572,154 @@ void dcn_args(const msda_dcn_problem *d, int64_t wo, KernelArgs &a)
     a.dil_w = d->dilation_w;
 }
 
+// Tensor-core dense layers (msda_gemm.cuh) ------------------------------------
+
+// Widest output tile, in 128-column MMAs (1 or 2; a tuning knob).
+#ifndef MSDA_GEMM_MAX_SUB
+#define MSDA_GEMM_MAX_SUB 2
+#endif
+constexpr int kGemmMaxSub = MSDA_GEMM_MAX_SUB;
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (the library links no driver library).
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+
+msda_status tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000 &fn)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_encode_tiled) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !f)
+            return MSDA_ERR_CUDA;
+        g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    fn = g_encode_tiled;
+    return MSDA_OK;
+}
+
+// Tensor map of a row-major matrix [rows, cols] of `dtype` moved in boxes of
+// box_rows x box_cols elements (box_cols * element size = 128 bytes) with the
+// 128-byte swizzle the MMA descriptors and the epilogue boxes use; rows and
+// columns outside the matrix read as zero and are not written.
+msda_status tile_map(CUtensorMap &map, const void *ptr, CUtensorMapDataType dtype, int64_t rows, int64_t cols,
+                     int box_cols, int box_rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    msda_status st = tensor_map_encoder(encode);
+    if (st != MSDA_OK)
+        return st;
+    const int esize = dtype == CU_TENSOR_MAP_DATA_TYPE_FLOAT32 ? 4 : 2;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * esize};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(&map, dtype, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MSDA_OK : MSDA_ERR_CUDA;
+}
+
+// Operand map: bf16 [rows, cols] in 128-row x 64-column boxes.
+msda_status operand_map(CUtensorMap &map, const void *ptr, int64_t rows, int64_t cols)
+{
+    return tile_map(map, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rows, cols, msda_gemm::kBK, msda_gemm::kBM);
+}
+
+// Output map: 32-row boxes of 128 bytes (32 float32 or 64 bf16 columns).
+msda_status output_map(CUtensorMap &map, void *ptr, bool bf16, int64_t rows, int64_t cols)
+{
+    return tile_map(map, ptr, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rows,
+                    cols, bf16 ? 64 : 32, 32);
+}
+
+template <int NSUB, bool WRES>
+msda_status launch_gemm_n(const CUtensorMap &mx, const CUtensorMap &mw, const CUtensorMap &mo0,
+                          const CUtensorMap &mo1, msda_gemm::Params &p, int sms, int dev, cudaStream_t s)
+{
+    using C = msda_gemm::Cfg<NSUB, WRES>;
+    const void *k = (const void *)msda_gemm::gemm_kernel<NSUB, WRES>;
+    int optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, k) != cudaSuccess)
+        return MSDA_ERR_CUDA;
+    msda_status st;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        st = raise_smem_limit(k, dev);
+    }
+    if (st != MSDA_OK)
+        return st;
+    // as many stages as the shared memory left after the w area holds
+    const int avail = optin - (int)fa.sharedSizeBytes;
+    p.stages = (avail - C::smem_bytes(p.w_bytes, 0)) / C::kStageBytes;
+    if (p.stages > msda_gemm::kMaxStages)
+        p.stages = msda_gemm::kMaxStages;
+    if (p.stages < 2)
+        return MSDA_ERR_UNSUPPORTED;
+    const int smem = C::smem_bytes(p.w_bytes, p.stages);
+    const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+    // one persistent CTA per SM (the shared memory admits one); with the
+    // weight resident, a multiple of n_tiles CTAs, so that each CTA keeps
+    // one column tile
+    int64_t grid = WRES ? (int64_t)(sms / p.n_tiles) * p.n_tiles : sms;
+    if (grid > tiles)
+        grid = tiles;
+    msda_gemm::gemm_kernel<NSUB, WRES><<<(unsigned)grid, msda_gemm::kThreads, smem, s>>>(mx, mw, mo0, mo1, p);
+    return cudaGetLastError() == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
+}
+
+template <int NSUB>
+msda_status launch_gemm_nsub(const CUtensorMap &mx, const CUtensorMap &mw, const CUtensorMap &mo0,
+                             const CUtensorMap &mo1, msda_gemm::Params &p, cudaStream_t s)
+{
+    using C = msda_gemm::Cfg<NSUB, true>;
+    int dev = 0, sms = 0;
+    msda_status st = current_device(dev, sms, &p.status);
+    if (st != MSDA_OK)
+        return st;
+    p.m_tiles = (p.rows + msda_gemm::kBM - 1) / msda_gemm::kBM;
+    p.n_tiles = (p.N + C::kBN - 1) / C::kBN;
+    const int nkb = (p.K + msda_gemm::kBK - 1) / msda_gemm::kBK;
+    // the weight stays in shared memory when its K blocks fit the area
+    if (nkb <= C::kMaxKBlocks && p.n_tiles <= sms) {
+        p.w_bytes = nkb * NSUB * msda_gemm::kBSubBytes;
+        return launch_gemm_n<NSUB, true>(mx, mw, mo0, mo1, p, sms, dev, s);
+    }
+    p.w_bytes = 0;
+    return launch_gemm_n<NSUB, false>(mx, mw, mo0, mo1, p, sms, dev, s);
+}
+
+msda_status launch_gemm(int nsub, const CUtensorMap &mx, const CUtensorMap &mw, const CUtensorMap &mo0,
+                        const CUtensorMap &mo1, msda_gemm::Params &p, cudaStream_t s)
+{
+    switch (nsub) {
+    case 1: return launch_gemm_nsub<1>(mx, mw, mo0, mo1, p, s);
+    case 2: return launch_gemm_nsub<2>(mx, mw, mo0, mo1, p, s);
+    }
+    return MSDA_ERR_UNSUPPORTED;
+}
+
+// Query-head sizes: P = M*L*K with L*K a power of two <= 32 and P a multiple
+// of 32 (a 32-column chunk of the head is all offsets or whole softmax runs).
+msda_status head_sizes(const msda_problem *p, int64_t &rows, int &P, int &LK)
+{
+    if (!p || p->batch < 0 || p->num_queries < 0 || p->num_heads < 1 || p->num_levels < 1 ||
+        p->num_levels > msda::kMaxLevels || p->num_points < 1)
+        return MSDA_ERR_INVALID_ARG;
+    LK = p->num_levels * p->num_points;
+    const int64_t P64 = (int64_t)p->num_heads * LK;
+    if (LK > 32 || (LK & (LK - 1)) != 0 || P64 % 32 != 0 || 3 * P64 > (int64_t(1) << 20))
+        return MSDA_ERR_UNSUPPORTED;
+    rows = p->batch * p->num_queries;
+    if (rows >= (int64_t(1) << 31))
+        return MSDA_ERR_UNSUPPORTED;
+    P = (int)P64;
+    return MSDA_OK;
+}
+
 // NVTX range around each entry point that enqueues work, so that a profiler
 // timeline shows the library calls (no-ops when no tool is attached).
 struct NvtxRange {
@@ -899,6 +1050,120 @@ msda_status msda_sort_queries(const msda_problem *problem, const float *points, 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     msda::sort_queries_kernel<<<(unsigned)problem->batch, msda::kSortThreads, 0, s>>>(
         reinterpret_cast<const float2 *>(points), problem->num_queries, query_order);
+    return cudaGetLastError() == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
+}
+
+msda_status msda_linear(int64_t rows, int32_t in_features, int32_t out_features, const void *x,
+                        const void *weight, const float *bias, void *out, int32_t out_dtype,
+                        msda_stream_t stream)
+{
+    MSDA_TRACE();
+    if (rows < 0 || rows >= (int64_t(1) << 31) || in_features < 8 || in_features % 8 != 0 ||
+        out_features < 8 || out_features % 8 != 0 || out_features >= (1 << 20) ||
+        (out_dtype != MSDA_F32 && out_dtype != MSDA_BF16))
+        return MSDA_ERR_INVALID_ARG;
+    if (rows == 0)
+        return MSDA_OK;
+    if (!x || !weight || !out || !aligned16(x) || !aligned16(weight) || !aligned16(out) ||
+        (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+        return MSDA_ERR_INVALID_ARG;
+    const bool bf16 = out_dtype == MSDA_BF16;
+    CUtensorMap mx, mw, mo;
+    msda_status st = operand_map(mx, x, rows, in_features);
+    if (st == MSDA_OK)
+        st = operand_map(mw, weight, out_features, in_features);
+    if (st == MSDA_OK)
+        st = output_map(mo, out, bf16, rows, out_features);
+    if (st != MSDA_OK)
+        return st;
+    msda_gemm::Params p = {};
+    p.rows = (int)rows;
+    p.N = out_features;
+    p.K = in_features;
+    p.bias = bias;
+    p.epi = msda_gemm::kEpiStore;
+    p.out_bf16 = bf16;
+    return launch_gemm(out_features <= 128 ? 1 : kGemmMaxSub, mx, mw, mo, mo, p,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_query_head(const msda_problem *problem, int32_t in_features, const void *query,
+                            const void *weight, const float *bias, const float *reference_points,
+                            const int64_t *spatial_shapes, float *sampling_locations,
+                            float *attention_weights, msda_stream_t stream)
+{
+    MSDA_TRACE();
+    int64_t rows = 0;
+    int P = 0, LK = 0;
+    msda_status st = head_sizes(problem, rows, P, LK);
+    if (st != MSDA_OK)
+        return st;
+    if (in_features < 8 || in_features % 8 != 0)
+        return MSDA_ERR_INVALID_ARG;
+    if (rows == 0)
+        return MSDA_OK;
+    if (!query || !weight || !aligned16(query) || !aligned16(weight) ||
+        (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) || !ptr_ok(reference_points, rows * 2) ||
+        !spatial_shapes || !aligned16(spatial_shapes) || !ptr_ok(sampling_locations, rows * 2 * P) ||
+        !ptr_ok(attention_weights, rows * P))
+        return MSDA_ERR_INVALID_ARG;
+    CUtensorMap mx, mw, mloc, mattn;
+    st = operand_map(mx, query, rows, in_features);
+    if (st == MSDA_OK)
+        st = operand_map(mw, weight, 3 * (int64_t)P, in_features);
+    if (st == MSDA_OK)
+        st = output_map(mloc, sampling_locations, false, rows, 2 * (int64_t)P);
+    if (st == MSDA_OK)
+        st = output_map(mattn, attention_weights, false, rows, P);
+    if (st != MSDA_OK)
+        return st;
+    msda_gemm::Params p = {};
+    p.rows = (int)rows;
+    p.N = 3 * P;
+    p.K = in_features;
+    p.bias = bias;
+    p.epi = msda_gemm::kEpiHead;
+    p.P = P;
+    p.L = problem->num_levels;
+    p.LK = LK;
+    p.lk_mask = LK - 1;
+    int ks = 0;
+    while ((1 << ks) < problem->num_points)
+        ++ks;
+    p.k_shift = ks;  // L*K is a power of two, so K is one too
+    p.ref = reference_points;
+    p.shapes = spatial_shapes;
+    return launch_gemm(3 * P <= 128 ? 1 : kGemmMaxSub, mx, mw, mloc, mattn, p,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+msda_status msda_query_head_backward(const msda_problem *problem, const float *attention_weights,
+                                     const float *grad_sampling_locations,
+                                     const float *grad_attention_weights, const int64_t *spatial_shapes,
+                                     float *grad_head, float *grad_reference_points, msda_stream_t stream)
+{
+    MSDA_TRACE();
+    int64_t rows = 0;
+    int P = 0, LK = 0;
+    msda_status st = head_sizes(problem, rows, P, LK);
+    if (st != MSDA_OK)
+        return st;
+    if (rows == 0)
+        return MSDA_OK;
+    if (!ptr_ok(attention_weights, rows * P) || !ptr_ok(grad_sampling_locations, rows * 2 * P) ||
+        !ptr_ok(grad_attention_weights, rows * P) || !spatial_shapes || !aligned16(spatial_shapes) ||
+        !ptr_ok(grad_head, rows * 3 * P) || (grad_reference_points && !aligned16(grad_reference_points)))
+        return MSDA_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    st = current_device(dev, sms);
+    if (st != MSDA_OK)
+        return st;
+    int64_t blocks = (rows + 7) / 8;
+    if (blocks > (int64_t)sms * 8)
+        blocks = (int64_t)sms * 8;
+    msda::head_backward_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        rows, P, problem->num_levels, problem->num_points, attention_weights, grad_sampling_locations,
+        grad_attention_weights, spatial_shapes, grad_head, grad_reference_points);
     return cudaGetLastError() == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
 }
 

@@ -232,4 +232,64 @@ __global__ void __launch_bounds__(kSortThreads) sort_queries_kernel(const float2
     }
 }
 
+// ------------------------------------------------ query head: chain rule --
+//
+// Backward of the query head's location / softmax step (cf-1.com/news/4799680
+// §3.2): with loc = ref + off / (W_l, H_l) and A = softmax over each run of
+// L*K logits, the gradient of the head's pre-activations is
+//   grad_off_x = grad_loc_x / W_l,  grad_off_y = grad_loc_y / H_l,
+//   grad_logit_j = A_j * (grad_A_j - sum_{i in run} A_i grad_A_i),
+// and grad_ref = sum over the query's samples of grad_loc.  One warp per
+// query row; L*K a power of two of at most 32 (a run is LK consecutive lanes).
+__global__ void __launch_bounds__(256) head_backward_kernel(int64_t rows, int P, int L, int K,
+                                                            const float *attn, const float *gloc,
+                                                            const float *gattn, const int64_t *shapes,
+                                                            float *ghead, float *gref)
+{
+    __shared__ float Hs[kMaxLevels], Ws[kMaxLevels];
+    if (threadIdx.x < L) {
+        Hs[threadIdx.x] = (float)shapes[2 * threadIdx.x];
+        Ws[threadIdx.x] = (float)shapes[2 * threadIdx.x + 1];
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int LK = L * K;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const float *gl = gloc + r * 2 * P;
+        float *gh = ghead + r * 3 * P;
+        float sx = 0.f, sy = 0.f;
+        for (int h = lane; h < 2 * P; h += 32) {
+            const int l = (h >> 1) / K % L;
+            const float g = __ldg(gl + h);
+            gh[h] = g / ((h & 1) ? Hs[l] : Ws[l]);
+            if (h & 1)
+                sy += g;
+            else
+                sx += g;
+        }
+        for (int j0 = 0; j0 < P; j0 += 32) {
+            const int j = j0 + lane;
+            const float a = j < P ? __ldg(attn + r * P + j) : 0.f;
+            const float g = j < P ? __ldg(gattn + r * P + j) : 0.f;
+            float dot = a * g;
+            for (int o = 1; o < LK; o <<= 1)
+                dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            if (j < P)
+                gh[2 * P + j] = a * (g - dot);
+        }
+        if (gref) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                sx += __shfl_xor_sync(0xffffffffu, sx, o);
+                sy += __shfl_xor_sync(0xffffffffu, sy, o);
+            }
+            if (lane == 0) {
+                gref[2 * r] = sx;
+                gref[2 * r + 1] = sy;
+            }
+        }
+    }
+}
+
 }  // namespace msda
