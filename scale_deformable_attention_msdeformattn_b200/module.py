@@ -1,13 +1,27 @@
 """The attention layer around the core, for callers that want a module.
 
-discosf.com/news/5175395 §3.1 describes the layer: a value projection, an
-output projection, and two linear heads on the query that predict, per head,
-level and point, the two offset components and one attention logit; the
-offsets start at zero and the logit head with Xavier weights.  Here the
-projections and heads are torch linear layers (library GEMMs, outside the
-operator's boundary) and everything between them — locations, softmax,
-sampling, weighted sum and all their gradients — runs in the fused kernels of
-libmsda.so through MSDeformAttnFusedFunction.
+discosf.com/news/5175395 §3.1 describes the layer: a value projection (W'_m of
+the formula, §2.2), an output projection (W_m), and two linear heads on the
+query that predict, per head, level and point, the two offset components and
+one attention logit; the offsets start at zero and the logit head with Xavier
+weights.  cf-1.com/news/4799680 §3.2 turns the head's outputs into sampling
+locations (reference + offset / (W_l, H_l)) and attention weights (a softmax
+over each head's L*K logits).
+
+On the GPU every step runs in libmsda.so, in the mixed precision the
+practical guide recommends (lpnh.cn/news/23513 §4.1: bf16 storage, float32
+accumulation):
+  value_proj   msda_linear on the tensor cores, bf16 output written directly
+               in the core's value layout [B, S, M, D]
+  heads        msda_query_head: one tensor-core GEMM for both heads whose
+               epilogue forms the sampling locations and the softmax (the
+               offsets and logits are never written)
+  core         msda_forward (bf16 value and output rows, float32 accumulation)
+  output_proj  msda_linear, float32 output
+The backward runs msda_backward, msda_query_head_backward (the location and
+softmax chain rule) and, for the projections' input and weight gradients,
+plain float32 matrix products (torch.matmul: library GEMMs).  The parameters
+stay float32 (master weights); the forward reads them rounded to bf16.
 """
 from __future__ import annotations
 
@@ -16,7 +30,66 @@ from typing import Optional
 import torch
 from torch import nn
 
-from .binding import MSDeformAttnFusedFunction
+from . import binding
+
+
+class _LayerFunction(torch.autograd.Function):
+    """The layer's forward and backward through the library's kernels."""
+
+    @staticmethod
+    def forward(ctx, query, reference_points, input_flatten, w_v, b_v, w_h, b_h, w_o, b_o,
+                spatial_shapes, level_start_index, padding_mask, M: int, L: int, K: int):
+        B, Q, C = query.shape
+        S = input_flatten.shape[1]
+        D = C // M
+        bf16 = torch.bfloat16
+        xb = input_flatten.to(bf16).contiguous()
+        qb = query.to(bf16).contiguous()
+        wvb, whb, wob = (w.to(bf16).contiguous() for w in (w_v, w_h, w_o))
+        ref = reference_points.float().contiguous()
+        value = binding.linear(xb.view(B * S, C), wvb, b_v.float().contiguous(),
+                               out_dtype=bf16).view(B, S, M, D)
+        if padding_mask is not None:
+            value = value.masked_fill(padding_mask[:, :, None, None], 0.0)
+        loc, attn = binding.query_head(qb, whb, b_h.float().contiguous(), ref, spatial_shapes, M, K)
+        core = binding.forward(value, spatial_shapes, level_start_index, loc, attn)
+        y = binding.linear(core.view(B * Q, C), wob, b_o.float().contiguous(), out_dtype=torch.float32)
+        ctx.save_for_backward(xb, qb, wvb, whb, wob, value, loc, attn, core, spatial_shapes,
+                              level_start_index,
+                              padding_mask if padding_mask is not None else torch.empty(0))
+        ctx.dims = (B, Q, S, C, M, L, K)
+        ctx.has_mask = padding_mask is not None
+        return y.view(B, Q, C).to(query.dtype)
+
+    @staticmethod
+    def backward(ctx, grad_y):
+        (xb, qb, wvb, whb, wob, value, loc, attn, core, shapes, starts, mask) = ctx.saved_tensors
+        B, Q, S, C, M, L, K = ctx.dims
+        P = M * L * K
+        gy = grad_y.float().reshape(B * Q, C)
+        # output projection y = core W_o^T + b_o
+        g_core = gy @ wob.float()
+        g_wo = gy.t() @ core.view(B * Q, C).float()
+        g_bo = gy.sum(0)
+        # the core (its grad_output rows are stored in the value dtype, bf16)
+        gv, gl, ga = binding.backward(value, shapes, starts, loc, attn,
+                                      g_core.to(torch.bfloat16).view(B, Q, M, C // M))
+        if ctx.has_mask:
+            gv = gv.masked_fill(mask[:, :, None, None], 0.0)
+        # value projection value = x W_v^T + b_v
+        gvf = gv.view(B * S, C)
+        g_x = gvf @ wvb.float()
+        g_wv = gvf.t() @ xb.view(B * S, C).float()
+        g_bv = gvf.sum(0)
+        # the heads: location / softmax chain rule, then the linear layer
+        gh, gref = binding.query_head_backward(attn, gl, ga, shapes,
+                                               want_grad_reference_points=ctx.needs_input_grad[1])
+        ghf = gh.view(B * Q, 3 * P)
+        g_q = ghf @ whb.float()
+        g_wh = ghf.t() @ qb.view(B * Q, C).float()
+        g_bh = ghf.sum(0)
+        return (g_q.view(B, Q, C), gref, g_x.view(B, S, C), g_wv, g_bv, g_wh, g_bh, g_wo, g_bo,
+                None, None, None, None, None, None)
 
 
 class MSDeformAttn(nn.Module):
@@ -24,10 +97,13 @@ class MSDeformAttn(nn.Module):
 
     forward(query [B, Q, C], reference_points [B, Q, 2] normalized (x, y),
     input_flatten [B, S, C], spatial_shapes [L, 2] int64 (H, W),
-    level_start_index [L] int64, padding_mask [B, S] bool or None) -> [B, Q, C].
+    level_start_index [L] int64, padding_mask [B, S] bool or None) -> [B, Q, C]
+    (float32, or the query's dtype).
 
-    One reference point per query, shared by the levels (the fused kernels'
-    form).  Padded keys (padding_mask True) get a zero value row.
+    One reference point per query, shared by the levels.  Padded keys
+    (padding_mask True) get a zero value row.  Sizes the kernels need:
+    C = M * D with D in {8, 16, 32, 64, 128, 256} and C a multiple of 8;
+    L * K a power of two of at most 32; M * L * K a multiple of 32.
     """
 
     def __init__(self, d_model: int = 256, n_levels: int = 4, n_heads: int = 8, n_points: int = 4):
@@ -55,18 +131,15 @@ class MSDeformAttn(nn.Module):
                 level_start_index: torch.Tensor,
                 padding_mask: Optional[torch.Tensor] = None) -> torch.Tensor:
         B, Q, _ = query.shape
-        S = input_flatten.shape[1]
         M, L, K = self.n_heads, self.n_levels, self.n_points
         if reference_points.shape != (B, Q, 2):
             raise ValueError("reference_points must be [B, Q, 2] (one point per query)")
         if spatial_shapes.shape != (L, 2):
             raise ValueError(f"spatial_shapes must be [{L}, 2]")
-        value = self.value_proj(input_flatten)
-        if padding_mask is not None:
-            value = value.masked_fill(padding_mask[..., None], 0.0)
-        value = value.reshape(B, S, M, self.d_model // M).contiguous()
-        offsets = self.sampling_offsets(query).float().reshape(B, Q, M, L, K, 2).contiguous()
-        logits = self.attention_weights(query).float().reshape(B, Q, M, L * K).contiguous()
-        out = MSDeformAttnFusedFunction.apply(value, spatial_shapes, level_start_index,
-                                              reference_points.float().contiguous(), offsets, logits)
-        return self.output_proj(out.reshape(B, Q, self.d_model))
+        # one head GEMM: offset rows (M, L, K, 2) then logit rows (M, L*K)
+        w_h = torch.cat([self.sampling_offsets.weight, self.attention_weights.weight], 0)
+        b_h = torch.cat([self.sampling_offsets.bias, self.attention_weights.bias], 0)
+        return _LayerFunction.apply(query, reference_points, input_flatten, self.value_proj.weight,
+                                    self.value_proj.bias, w_h, b_h, self.output_proj.weight,
+                                    self.output_proj.bias, spatial_shapes, level_start_index,
+                                    padding_mask, M, L, K)

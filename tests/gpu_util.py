@@ -83,14 +83,15 @@ def elem_err(gpu, ref, floor: float = ELEM_FLOOR) -> float:
     return float((np.abs(g - r) / np.maximum(np.abs(r), floor * scale)).max())
 
 
-def assert_close(gpu, ref, tol, what, elem_tol=None):
+def assert_close(gpu, ref, tol, what, elem_tol=None, floor=ELEM_FLOOR):
     """Asserts the normwise error <= tol and the elementwise error <= elem_tol
-    (default: ELEM_TOL for bf16 tensors, else for float32); prints both."""
+    (default: ELEM_TOL for bf16 tensors, else for float32) with the given
+    floor; prints both."""
     e = rel_err(gpu, ref)
     if elem_tol is None:
         is_bf16 = isinstance(gpu, torch.Tensor) and gpu.dtype == torch.bfloat16
         elem_tol = ELEM_TOL["bf16" if is_bf16 else "f32"]
-    ee = elem_err(gpu, ref)
+    ee = elem_err(gpu, ref, floor)
     print(f"  {what}: normwise {e:.2e} elementwise {ee:.2e}")
     assert e <= tol, f"{what}: max relative error {e:.3e} > {tol:.1e}"
     assert ee <= elem_tol, f"{what}: elementwise relative error {ee:.3e} > {elem_tol:.1e}"
