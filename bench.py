@@ -80,6 +80,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-nonfused", action="store_true")
+    ap.add_argument("--layer", action="store_true",
+                    help="time the whole MSDeformAttn layer (tensor-core projections and fused "
+                         "query head around the core), forward + backward, at the workload's "
+                         "shape with C = M*D, beside torch linear layers around the fused core")
     ap.add_argument("--merge-reductions", action="store_true",
                     help="backward merges each tile's grad_value contributions per corner "
                          "row before reducing them (MSDA_MERGE_REDUCTIONS)")
@@ -1135,9 +1139,106 @@ def run_dcn_reference(args):
     return result
 
 
+# ------------------------------------------------------ the whole layer --
+
+def run_layer(args):
+    """One MSDeformAttn layer step (forward + backward through autograd) at
+    the workload's shape, C = M * D: the library's layer (tensor-core
+    value / output projections, fused query head, core) beside the same
+    layer built from torch bf16 linear layers around the fused core (the
+    offsets and logits then make a round trip through HBM).  L2 flushed
+    before each step; CUDA events on the current stream; one GPU."""
+    import torch
+    import torch.nn.functional as F
+    import scale_deformable_attention_msdeformattn_b200 as msda
+
+    w = wl.WORKLOADS[args.workload]
+    B, S, Q, M, D, L, K = w.B, w.S, w.num_queries, w.M, w.D, w.L, w.K
+    C = M * D
+    P = M * L * K
+    dev = torch.device("cuda", 0)
+    torch.manual_seed(0)
+    shapes = torch.tensor(w.levels, dtype=torch.int64, device=dev)
+    starts = torch.from_numpy(wl.level_start_index(w.levels)).to(dev)
+    x = wl.generate(w, with_nonfused=False)
+    ref = torch.from_numpy(x.reference_points).to(dev)
+    layer = msda.MSDeformAttn(d_model=C, n_levels=L, n_heads=M, n_points=K).to(dev)
+    with torch.no_grad():
+        layer.sampling_offsets.weight.normal_(0.0, w.offset_sigma / C ** 0.5)
+        layer.attention_weights.weight.normal_(0.0, w.logit_sigma / C ** 0.5)
+    query = torch.randn(B, Q, C, device=dev, requires_grad=True)
+    feats = torch.randn(B, S, C, device=dev, requires_grad=True)
+    gy = torch.randn(B, Q, C, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def library_step():
+        y = layer(query, ref, feats, shapes, starts)
+        y.backward(gy)
+
+    bf = torch.bfloat16
+
+    def torch_linear_step():
+        # the same layer with torch bf16 linear layers around the fused core
+        value = F.linear(feats.to(bf), layer.value_proj.weight.to(bf), layer.value_proj.bias.to(bf))
+        qb = query.to(bf)
+        off = F.linear(qb, layer.sampling_offsets.weight.to(bf), layer.sampling_offsets.bias.to(bf))
+        logit = F.linear(qb, layer.attention_weights.weight.to(bf), layer.attention_weights.bias.to(bf))
+        core = msda.MSDeformAttnFusedFunction.apply(
+            value.view(B, S, M, D), shapes, starts, ref, off.float().view(B, Q, M, L, K, 2),
+            logit.float().view(B, Q, M, L * K))
+        y = F.linear(core.reshape(B, Q, C), layer.output_proj.weight.to(bf), layer.output_proj.bias.to(bf))
+        y.float().backward(gy)
+
+    def time(step, n):
+        evs = []
+        for i in range(args.warmup + n):
+            flush.fill_(float(i))
+            for t in (query, feats):
+                t.grad = None
+            layer.zero_grad(set_to_none=True)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            e[0].record()
+            step()
+            e[1].record()
+            if i >= args.warmup:
+                evs.append(e)
+        torch.cuda.synchronize()
+        ms = [a.elapsed_time(b) for a, b in evs]
+        return statistics.median(ms), ms
+
+    lib_ms, _ = time(library_step, args.steps)
+    tl_ms, _ = time(torch_linear_step, args.steps)
+    if msda.device_status() != 0:
+        raise SystemExit("kernels reported an error")
+    # bytes the fused head and the value epilogue keep out of HBM: the
+    # offsets + logits (bf16 linear output, then read back as float32 by the
+    # core) and the separate float32 copies of them
+    head_bytes = B * Q * 3 * P * (2 + 2 + 4 + 4)
+    line = {
+        "metric": "MSDeformAttn layer fwd+bwd ms (projections, query head, core)",
+        "value": round(lib_ms, 4), "unit": "ms", "higher_is_better": False,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "dtype": "bf16 operands / f32 accumulate (layer); core bf16 value",
+        "data": "synthetic: seeded offsets / logits heads, random query and features",
+        "config": {"workload": w.name, "B": B, "S": S, "Q": Q, "C": C, "M": M, "L": L, "K": K,
+                   "l2": "flushed before each step"},
+        "torch_linear_layer_ms": round(tl_ms, 4),
+        "speedup_vs_torch_linear_layer": round(tl_ms / lib_ms, 3),
+        "head_hbm_bytes_avoided_per_step": head_bytes,
+        "gpu": torch.cuda.get_device_name(0),
+    }
+    print(json.dumps(line), flush=True)
+    if args.out:
+        with open(args.out, "a") as f:
+            f.write(json.dumps(line) + "\n")
+    return line
+
+
 def main(argv=None):
     args = parse_args(argv)
     dcn = args.workload in wl.DCN_WORKLOADS
+    if args.layer:
+        return run_layer(args)
     if args.impl == "reference":
         return run_dcn_reference(args) if dcn else run_reference(args)
     return run_dcn(args) if dcn else run_ours(args)

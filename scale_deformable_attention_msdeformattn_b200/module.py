@@ -19,9 +19,11 @@ accumulation):
   core         msda_forward (bf16 value and output rows, float32 accumulation)
   output_proj  msda_linear, float32 output
 The backward runs msda_backward, msda_query_head_backward (the location and
-softmax chain rule) and, for the projections' input and weight gradients,
-plain float32 matrix products (torch.matmul: library GEMMs).  The parameters
-stay float32 (master weights); the forward reads them rounded to bf16.
+softmax chain rule), the projections' input gradients through msda_linear
+(bf16 gradient rows against the transposed bf16 weights) and their weight
+gradients as bf16 library matrix products with float32 accumulation
+(torch.matmul).  The parameters stay float32 (master weights); the forward
+reads them rounded to bf16.
 """
 from __future__ import annotations
 
@@ -66,28 +68,31 @@ class _LayerFunction(torch.autograd.Function):
         (xb, qb, wvb, whb, wob, value, loc, attn, core, shapes, starts, mask) = ctx.saved_tensors
         B, Q, S, C, M, L, K = ctx.dims
         P = M * L * K
-        gy = grad_y.float().reshape(B * Q, C)
-        # output projection y = core W_o^T + b_o
-        g_core = gy @ wob.float()
-        g_wo = gy.t() @ core.view(B * Q, C).float()
-        g_bo = gy.sum(0)
-        # the core (its grad_output rows are stored in the value dtype, bf16)
-        gv, gl, ga = binding.backward(value, shapes, starts, loc, attn,
-                                      g_core.to(torch.bfloat16).view(B, Q, M, C // M))
+        bf16 = torch.bfloat16
+        # the layer's gradients in bf16 as its operands (float32 accumulation):
+        # input gradients on the tensor cores through msda_linear with the
+        # transposed weights, weight gradients as library GEMMs
+        gyb = grad_y.to(bf16).reshape(B * Q, C).contiguous()
+        # output projection y = core W_o^T + b_o; the core's grad_output rows
+        # are stored in the value dtype (bf16)
+        g_core = binding.linear(gyb, wob.t().contiguous(), out_dtype=bf16)
+        g_wo = (gyb.t() @ core.view(B * Q, C)).float()
+        g_bo = grad_y.float().sum((0, 1))
+        gv, gl, ga = binding.backward(value, shapes, starts, loc, attn, g_core.view(B, Q, M, C // M))
         if ctx.has_mask:
             gv = gv.masked_fill(mask[:, :, None, None], 0.0)
         # value projection value = x W_v^T + b_v
-        gvf = gv.view(B * S, C)
-        g_x = gvf @ wvb.float()
-        g_wv = gvf.t() @ xb.view(B * S, C).float()
-        g_bv = gvf.sum(0)
+        gvb = gv.view(B * S, C).to(bf16)
+        g_x = binding.linear(gvb, wvb.t().contiguous(), out_dtype=torch.float32)
+        g_wv = (gvb.t() @ xb.view(B * S, C)).float()
+        g_bv = gv.view(B * S, C).sum(0)
         # the heads: location / softmax chain rule, then the linear layer
         gh, gref = binding.query_head_backward(attn, gl, ga, shapes,
                                                want_grad_reference_points=ctx.needs_input_grad[1])
-        ghf = gh.view(B * Q, 3 * P)
-        g_q = ghf @ whb.float()
-        g_wh = ghf.t() @ qb.view(B * Q, C).float()
-        g_bh = ghf.sum(0)
+        ghb = gh.view(B * Q, 3 * P).to(bf16)
+        g_q = binding.linear(ghb, whb.t().contiguous(), out_dtype=torch.float32)
+        g_wh = (ghb.t() @ qb.view(B * Q, C)).float()
+        g_bh = gh.view(B * Q, 3 * P).sum(0)
         return (g_q.view(B, Q, C), gref, g_x.view(B, S, C), g_wv, g_bv, g_wh, g_bh, g_wo, g_bo,
                 None, None, None, None, None, None)
 
