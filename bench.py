@@ -87,6 +87,9 @@ def parse_args(argv=None):
     ap.add_argument("--merge-reductions", action="store_true",
                     help="backward merges each tile's grad_value contributions per corner "
                          "row before reducing them (MSDA_MERGE_REDUCTIONS)")
+    ap.add_argument("--zero", choices=("overlap", "serial"), default="overlap",
+                    help="where the zero-fill of the gradient accumulators runs: on a second "
+                         "stream beside the forward (default), or after it on the launch stream")
     ap.add_argument("--sorted", action="store_true",
                     help="order the queries by the Morton cell of their reference point "
                          "(msda_sort_queries, inside the timed step) and process them in that order")
@@ -304,10 +307,15 @@ def run_ours(args):
     qv = torch.empty((B, S, M, D), dtype=torch.int8, device=dev) if int8 else None
     qs = torch.empty((B, M), dtype=torch.float32, device=dev) if int8 else None
 
+    nbytes = algorithmic_bytes(w)
+    overlap = args.zero == "overlap"
+
     def step(ev, tin=None, o=None):
         # the zero-fill of the gradient accumulators does not depend on the
-        # forward: it runs on a second stream, concurrently with it, and the
-        # backward waits for both
+        # forward: it runs on a second stream beside it and the backward waits
+        # for both (--zero serial puts it after the forward instead: decoder
+        # step 137 against 129 us, but the forward's own time without HBM
+        # shared with the zero-fill's 182 MB)
         tin = tin or t
         o = o or outputs
         stream = torch.cuda.current_stream()  # the capture stream under graph capture
@@ -318,16 +326,22 @@ def run_ours(args):
             msda.quantize_value_s8(tin["value"], value_s8=qv, value_scale=qs)
         value = qv if int8 else tin["value"]
         ev[6].record(stream)
-        side.wait_event(ev[6])
-        with torch.cuda.stream(side):
-            ev[4].record(side)
-            msda.zero_grads(o["grad_value"], o["grad_reference_points"])
-            ev[5].record(side)
         msda.fused_forward(value, tin["spatial_shapes"], tin["level_start_index"],
                            tin["reference_points"], tin["sampling_offsets"],
                            tin["attention_logits"], out=o["out"], query_order=order, value_scale=qs)
+        if overlap:  # enqueued after the forward, whose CTAs take the SMs first
+            side.wait_event(ev[6])
+            with torch.cuda.stream(side):
+                ev[4].record(side)
+                msda.zero_grads(o["grad_value"], o["grad_reference_points"])
+                ev[5].record(side)
         ev[1].record(stream)
-        stream.wait_event(ev[5])
+        if overlap:
+            stream.wait_event(ev[5])
+        else:
+            ev[4].record(stream)
+            msda.zero_grads(o["grad_value"], o["grad_reference_points"])
+            ev[5].record(stream)
         ev[2].record(stream)
         msda.fused_backward(value, tin["spatial_shapes"], tin["level_start_index"],
                             tin["reference_points"], tin["sampling_offsets"],
@@ -367,13 +381,12 @@ def run_ours(args):
 
     fwd = [e[6].elapsed_time(e[1]) for e in evs]
     pre = [e[0].elapsed_time(e[6]) for e in evs]
-    zero = [e[4].elapsed_time(e[5]) for e in evs]  # on the side stream, under the forward
+    zero = [e[4].elapsed_time(e[5]) for e in evs]
     bwd = [e[2].elapsed_time(e[3]) for e in evs]
     stepms = [e[0].elapsed_time(e[3]) for e in evs]
     samples_step = w.samples
     total_ms, value = aggregate_over_ranks(float(sum(stepms)), samples_step, args.steps, world, dev)
     ms_per_step = total_ms / args.steps
-    nbytes = algorithmic_bytes(w)
 
     result = None
     if rank == 0:
@@ -407,13 +420,14 @@ def run_ours(args):
                 "samples_per_step_per_gpu": samples_step,
                 "step": ("msda_sort_queries -> " if args.sorted else "")
                 + ("msda_quantize_value_s8 -> " if int8 else "")
-                + "msda_fused_forward || msda_zero_grads (second stream) -> msda_fused_backward",
+                + ("msda_fused_forward || msda_zero_grads (second stream) -> msda_fused_backward"
+                   if overlap else "msda_fused_forward -> msda_zero_grads -> msda_fused_backward"),
                 "query_order": "Morton cell of the reference point" if args.sorted else "natural",
                 "l2": "flushed between steps (256 MiB write outside the timed events)",
                 "parallelism": f"dp{world} (independent batch per GPU)",
             },
             "fwd_ms": round(fwd_ms, 5),
-            "zero_ms": round(zero_ms, 5),  # overlapped with the forward
+            "zero_ms": round(zero_ms, 5),  # under the forward, or after it (config.step)
             # before the forward: the query sort (--sorted) and the INT8 quantisation
             "pre_ms": round(statistics.mean(pre), 5) if (args.sorted or int8) else None,
 
@@ -451,6 +465,8 @@ def run_ours(args):
                 "merged per tile of consecutive queries of one head"
                 if args.merge_reductions and not args.sorted
                 else "direct (one vector reduction per corner contribution)")
+            result["fwd_alone"] = _time_fwd(msda, t, outputs, flush, min(args.steps, 50),
+                                            qv if int8 else t["value"], qs, order, nbytes, peaks)
             result["warm_l2"] = _time_warm(w, step, min(args.steps, 50))
             result["graph"] = _time_graph(w.samples, step, flush, min(args.steps, 100), 7)
         stats = _input_stats(w, x)
@@ -459,6 +475,16 @@ def run_ours(args):
             touched = step_bytes - 2 * (stats["value_bytes_whole"] - stats["value_bytes_touched"])
             stats["hbm_frac_step_touched"] = round(
                 touched / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
+            # each kernel reads the value tensor once: count its touched sectors
+            untouched = stats["value_bytes_whole"] - stats["value_bytes_touched"]
+            rl = result["roofline"]
+            rl["bytes_per_launch_touched"] = nbytes[dom] - untouched
+            rl["frac_touched"] = round((nbytes[dom] - untouched) / (dom_ms * 1e-3) / 1e9
+                                       / peaks["hbm_gbs"], 4)
+            if "fwd_alone" in result:
+                fa = result["fwd_alone"]
+                fa["frac_touched"] = round((nbytes["fused_forward"] - untouched)
+                                           / (fa["fwd_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
         result["config"]["input_stats"] = stats
         if not args.no_e2e:
             result["e2e"] = _time_e2e(_pinned(x), step, make_outputs, flush, min(args.steps, 50),
@@ -523,6 +549,28 @@ def _time_nonfused(msda, t, w, nbytes, flush, n, value, value_scale=None):
             "fwd_hbm_frac": round(nbytes["forward"] / (fwd * 1e-3) / 1e9 / peak, 4),
             "bwd_hbm_frac": round(nbytes["backward"] / (bwd * 1e-3) / 1e9 / peak, 4),
             "fwd_gsamples_per_s": round(w.samples / (fwd * 1e-3) / 1e9, 4), "launches": n}
+
+
+def _time_fwd(msda, t, o, flush, n, value, value_scale, order, nbytes, peaks):
+    """msda_fused_forward alone (nothing beside it on the GPU, L2 flushed
+    before each launch)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    ts = []
+    for i in range(n + 3):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        flush.fill_(float(i))
+        e[0].record(stream)
+        msda.fused_forward(value, t["spatial_shapes"], t["level_start_index"],
+                           t["reference_points"], t["sampling_offsets"], t["attention_logits"],
+                           out=o["out"], query_order=order, value_scale=value_scale)
+        e[1].record(stream)
+        if i >= 3:
+            ts.append(e)
+    torch.cuda.synchronize()
+    ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ts)
+    return {"fwd_ms": round(ms, 5), "launches": n,
+            "frac": round(nbytes["fused_forward"] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
 
 
 def _time_bwd(msda, t, o, flush, n, value, value_scale, order, merge):
@@ -998,11 +1046,11 @@ def run_dcn(args):
             msda.quantize_value_s8(inp.flatten(1, 2), value_s8=q.flatten(1, 2), value_scale=qs)
             inp = q
         ev[4].record(stream)
-        side.wait_event(ev[4])
+        msda.dcn_forward(inp, tin["offset"], tin["mask"], out=o["out"], value_scale=qs, **geo)
+        side.wait_event(ev[4])  # enqueued after the forward, whose CTAs take the SMs first
         with torch.cuda.stream(side):
             msda.zero_grads(o["grad_input"].flatten(1, 2))
             ev[5].record(side)
-        msda.dcn_forward(inp, tin["offset"], tin["mask"], out=o["out"], value_scale=qs, **geo)
         ev[1].record(stream)
         stream.wait_event(ev[5])
         ev[2].record(stream)

@@ -298,10 +298,11 @@ msda_status launch_zero(float *a, int64_t na, float *b, int64_t nb, cudaStream_t
     msda_status st = current_device(dev, sms);
     if (st != MSDA_OK)
         return st;
+    // grid-stride over at most MSDA_ZERO_CTAS_PER_SM CTAs per SM
     int64_t work = na / 4 > nb ? na / 4 : nb;
     int64_t blocks = (work + 255) / 256;
-    if (blocks > (int64_t)sms * 8)
-        blocks = (int64_t)sms * 8;
+    if (blocks > (int64_t)sms * MSDA_ZERO_CTAS_PER_SM)
+        blocks = (int64_t)sms * MSDA_ZERO_CTAS_PER_SM;
     if (blocks < 1)
         blocks = 1;
     msda::zero_kernel<<<(unsigned)blocks, 256, 0, stream>>>(reinterpret_cast<float4 *>(a), na / 4, b, nb);
@@ -327,12 +328,49 @@ msda_status launch_to_bf16(const float *src, void *dst, int64_t n, cudaStream_t 
 
 // Kernel selection -----------------------------------------------------------
 
+// The forward with rows split over MSDA_FWD_SPLIT lane groups
+// (msda_kernels.cuh, forward_kernel SPLIT), taken for problems whose rows,
+// one lane group each, would not fill one resident wave of the unsplit
+// kernel.  Returns false (nothing launched) when the problem is larger.
+template <typename T, int DD, bool FUSED, bool SHORT>
+bool try_forward_split(KernelArgs &a, cudaStream_t s, msda_status &st)
+{
+    constexpr int rpw0 = msda::forward_rows_per_warp<T, DD>();
+    constexpr int rpw = rpw0 / MSDA_FWD_SPLIT;
+    static_assert(MSDA_FWD_SPLIT >= 1 && rpw >= 1, "split rows must fit a warp");
+    if (MSDA_FWD_SPLIT == 1)
+        return false;
+    int dev = 0, sms = 0;
+    if (current_device(dev, sms) != MSDA_OK)
+        return false;
+    const int64_t warps = (a.rows + rpw0 - 1) / rpw0;
+    if (warps >= (int64_t)sms * msda::kMaxWarpsPerCta * msda::FwdTune<T, SHORT>::kMinCtas)
+        return false;
+    st = launch_rows((const void *)msda::forward_kernel<T, DD, FUSED, false, SHORT, MSDA_FWD_SPLIT>, rpw,
+                     kForwardRecordBytes, a.L * a.K, false, a, s);
+    return true;
+}
+
 // The general kernels (query order, DCN grid) are separate instantiations, so
 // that the plain attention kernels carry none of their branches.
 template <bool FUSED>
 msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 {
     const bool gen = a.order != nullptr || a.dcn != 0 || a.stage != 0;
+    msda_status st = MSDA_OK;
+    if (!gen && p->value_dtype == MSDA_F32) {
+        if ((p->head_dim == 8 && try_forward_split<float, 8, FUSED, false>(a, s, st)) ||
+            (p->head_dim == 16 && try_forward_split<float, 16, FUSED, false>(a, s, st)) ||
+            (p->head_dim == 32 && try_forward_split<float, 32, FUSED, false>(a, s, st)))
+            return st;
+    }
+    if (!gen && p->value_dtype == MSDA_BF16 && a.L * a.K <= 16) {
+        if ((p->head_dim == 8 && try_forward_split<__nv_bfloat16, 8, FUSED, true>(a, s, st)) ||
+            (p->head_dim == 16 && try_forward_split<__nv_bfloat16, 16, FUSED, true>(a, s, st)) ||
+            (p->head_dim == 32 && try_forward_split<__nv_bfloat16, 32, FUSED, true>(a, s, st)) ||
+            (p->head_dim == 64 && try_forward_split<__nv_bfloat16, 64, FUSED, true>(a, s, st)))
+            return st;
+    }
 #define MSDA_FWD_CASE(T, DD)                                                                      \
     case DD:                                                                                       \
         return launch_rows(gen ? (const void *)msda::forward_kernel<T, DD, FUSED, true>          \

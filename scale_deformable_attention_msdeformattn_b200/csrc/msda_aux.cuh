@@ -14,8 +14,17 @@ namespace msda {
 __global__ void zero_kernel(float4 *a, int64_t n4, float *b, int64_t n)
 {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride)
-        a[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // four independent stores per step
+    for (; i + 3 * stride < n4; i += 4 * stride) {
+        a[i] = z;
+        a[i + stride] = z;
+        a[i + 2 * stride] = z;
+        a[i + 3 * stride] = z;
+    }
+    for (; i < n4; i += stride)
+        a[i] = z;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
         b[i] = 0.f;
 }

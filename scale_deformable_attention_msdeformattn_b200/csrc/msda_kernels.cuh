@@ -72,6 +72,12 @@ namespace msda {
 #ifndef MSDA_FWD_MIN_CTAS_BF16_SHORT
 #define MSDA_FWD_MIN_CTAS_BF16_SHORT 3
 #endif
+#ifndef MSDA_ZERO_CTAS_PER_SM         // zero-fill grid: 256-thread CTAs per SM (2 measured
+#define MSDA_ZERO_CTAS_PER_SM 8        // slower beside the decoder's forward: 57 against 48 us)
+#endif
+#ifndef MSDA_FWD_SPLIT               // lane groups per row of the split forward (small problems)
+#define MSDA_FWD_SPLIT 4
+#endif
 #ifndef MSDA_FWD_STAGE_F32           // TMA-staged set-up inputs (see "input staging")
 #define MSDA_FWD_STAGE_F32 0
 #endif
@@ -1174,7 +1180,14 @@ template <bool SHORT> struct FwdTune<S8, SHORT> {
 // GEN = false: the plain attention kernel (natural query order, no DCN grid),
 // with those branches removed at compile time; GEN = true honours
 // KernelArgs::order and KernelArgs::dcn.
-template <typename T, int D, bool FUSED, bool GEN, bool SHORT = false>
+//
+// SPLIT > 1 (plain kernels only): SPLIT lane groups share a row, group ph
+// gathering samples ph*U .. ph*U + U-1, then (ph + SPLIT)*U ..., and the
+// partial sums meet in a shuffle reduction before group 0 stores the row.
+// For problems with too few rows to fill the GPU (the decoder's 300 queries
+// per image), this gives each row SPLIT times the loads in flight and the
+// grid SPLIT times the warps.
+template <typename T, int D, bool FUSED, bool GEN, bool SHORT = false, int SPLIT = 1>
 __global__ void __launch_bounds__(kMaxWarpsPerCta * 32, FwdTune<T, SHORT>::kMinCtas)
 forward_kernel(const KernelArgs a_in)
 {
@@ -1189,6 +1202,8 @@ forward_kernel(const KernelArgs a_in)
     using Raw = typename Lay::Raw;
     constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Lay::kEpv;
     constexpr int U = Tune::kInFlight;  // samples in flight per lane (4 corners each)
+    static_assert(SPLIT == 1 || (!GEN && SPLIT * G <= 32), "row split: plain kernels, G * SPLIT <= 32");
+    constexpr int GS = G * SPLIT;       // lanes of one row
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ Geometry geo;
@@ -1199,14 +1214,14 @@ forward_kernel(const KernelArgs a_in)
     const int P = a.L * a.K;
     const int stride = record_stride(P);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int grp = lane / G, gl = lane % G;
-    const int slot = warp * Lay::kRowsPerWarp + grp;
+    constexpr int RPW = 32 / GS;  // rows per warp
+    const int grp = lane / GS, ph = (lane / G) % SPLIT, gl = lane % G;
+    const int slot = warp * RPW + grp;
     float4 *wa = reinterpret_cast<float4 *>(smem_raw) + slot * stride;
     int4 *off = reinterpret_cast<int4 *>(smem_raw) + a.rows_per_tile * stride + slot * stride;
     const uint64_t pol = stream_policy();
-    constexpr int RPW = Lay::kRowsPerWarp;
-    // staged slices are contiguous rows: not with a query order
-    const int cap = a.order ? 0 : stage_cap(Tune::kStage || a.stage, RPW, P);
+    // staged slices are contiguous rows: not with a query order nor a split
+    const int cap = (a.order || SPLIT > 1) ? 0 : stage_cap(Tune::kStage || a.stage, RPW, P);
     const WarpStage ws = warp_stage(smem_raw + align16((size_t)a.rows_per_tile * stride * 32), warp,
                                     blockDim.x >> 5, cap);
     if (cap) {
@@ -1269,21 +1284,21 @@ forward_kernel(const KernelArgs a_in)
             setup_forward_staged<FUSED>(a, geo, p0, RPW, lane, pol, wa - grp * stride, off - grp * stride,
                                         stride, ws.p + st * cap, ws.z + st * cap);
         else
-            setup_forward_row<G, FUSED>(a, geo, row, active, gl, pol, wa, off);
+            setup_forward_row<GS, FUSED>(a, geo, row, active, lane % GS, pol, wa, off);
         __syncwarp();
+        float acc[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            acc[e] = 0.f;
+        const int64_t bq = row / a.M;
+        const int m = (int)(row - bq * a.M);
+        const int64_t b = bq / a.Q;
         if (active) {
-            const int64_t bq = row / a.M;
-            const int m = (int)(row - bq * a.M);
-            const int64_t b = bq / a.Q;
             // this lane's first vector of head m of batch b, key 0; corner rows
             // are D channels apart
             const Raw *vbase = reinterpret_cast<const Raw *>(static_cast<const T *>(a.value) +
                                                              (b * a.S * a.M + m) * D) + gl;
-            float acc[E];
-#pragma unroll
-            for (int e = 0; e < E; ++e)
-                acc[e] = 0.f;
-            for (int s0 = 0; s0 < P; s0 += U) {
+            for (int s0 = ph * U; s0 < P; s0 += U * SPLIT) {
                 Raw v[U][4][CH];
                 float4 w[U];
                 bool ok[U];
@@ -1321,6 +1336,16 @@ forward_kernel(const KernelArgs a_in)
                         }
                 }
             }
+        }
+        if constexpr (SPLIT > 1) {
+            // the row's partial sums: lanes gl of its SPLIT groups are G apart
+#pragma unroll
+            for (int i = G; i < GS; i <<= 1)
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], i);
+        }
+        if (active && ph == 0) {
             if constexpr (std::is_same<T, S8>::value) {
                 // dequantize once per row, store bf16 (EPV = 8 channels, 16 bytes)
                 static_assert(EPV == 8, "INT8 lanes hold 8 channels");
