@@ -18,7 +18,7 @@
 //                      a STAGES-deep shared-memory ring; completion on a
 //                      "full" mbarrier per stage (transaction bytes);
 //   warp 1             allocates the TMEM columns; one lane issues the MMAs
-//                      (M = 128, N = 128 per sub-tile, K = 16 per instruction,
+//                      (M = 128, N = BN, K = 16 per instruction,
 //                      cta_group::1, kind::f16 with bf16 operands, float32
 //                      accumulation), frees each stage with tcgen05.commit on
 //                      its "empty" barrier and, after a tile's last K block,
@@ -27,9 +27,16 @@
 //                      (its 32 output rows; two warps per lane quarter, each
 //                      taking every other column chunk) 32 columns at a
 //                      time, applies the epilogue, writes 32-row x 128-byte
-//                      boxes into shared memory (128-byte swizzle, double-
-//                      buffered) and stores them with TMA; then it hands the
-//                      accumulator buffer back to the MMA lane.
+//                      boxes into shared memory (128-byte swizzle, one box
+//                      per warp by default) and stores them with TMA; then it
+//                      hands the accumulator buffer back to the MMA lane.
+// Measured on 87040 x 256 -> 256 (bf16 out, B200): the K-block cadence is set
+// by the stage ring (a 16 KB TMA load takes about 1.1 us to land under load,
+// so the ring's depth bounds the MMA rate); one epilogue box per warp instead
+// of two frees 32 KB for two more stages (21.8 -> 19.2 us), the bias from
+// shared memory instead of 32 shuffles per 32 columns takes a third off each
+// box (-> 19.0 us), and one N = 256 MMA instead of two of N = 128 per K step
+// 23.1 -> 21.8 us.
 // With NSUB <= 2 there are two accumulator buffers (2 x BN <= 512 columns),
 // so a tile's epilogue overlaps the next tile's loads and MMAs.
 // No TMA multicast and no clusters: the tensor maps cover this GPU's memory
@@ -57,6 +64,10 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kATileBytes = kBM * kBK * 2;      // 16 KB
 constexpr int kBSubBytes = kSubN * kBK * 2;     // 16 KB
 constexpr int kBoxBytes = 32 * 128;             // one epilogue box: 32 rows x 128 bytes
+#ifndef MSDA_GEMM_EPI_BOXES
+#define MSDA_GEMM_EPI_BOXES 1                       // epilogue boxes per warp (1 or 2)
+#endif
+constexpr int kEpiBoxes = MSDA_GEMM_EPI_BOXES;
 constexpr int kGemmSpinLimit = 1 << 20;
 constexpr int kMaxLevels = 16;
 
@@ -104,13 +115,21 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *b)
 // One potentially blocking test: the thread is suspended until the phase
 // completes or about kTryWaitNs nanoseconds pass, and woken as soon as it
 // completes (no sleep quantum added to the hand-off latency).
-constexpr unsigned kTryWaitNs = 1000;
+#ifndef MSDA_GEMM_TRY_WAIT_NS
+#define MSDA_GEMM_TRY_WAIT_NS 1000
+#endif
+constexpr unsigned kTryWaitNs = MSDA_GEMM_TRY_WAIT_NS;
 __device__ __forceinline__ bool mbar_try(uint64_t *b, unsigned parity)
 {
     uint32_t ok;
-    asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-                 " selp.u32 %0, 1, 0, p;\n}\n"
-                 : "=r"(ok) : "r"(smem_addr(b)), "r"(parity), "n"(kTryWaitNs) : "memory");
+    if constexpr (kTryWaitNs > 0)
+        asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+                     " selp.u32 %0, 1, 0, p;\n}\n"
+                     : "=r"(ok) : "r"(smem_addr(b)), "r"(parity), "n"(kTryWaitNs) : "memory");
+    else
+        asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+                     " selp.u32 %0, 1, 0, p;\n}\n"
+                     : "=r"(ok) : "r"(smem_addr(b)), "r"(parity) : "memory");
     return ok != 0;
 }
 // Bounded wait for the completion of the phase with the given parity: at
@@ -159,15 +178,23 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr)
 }
 
 // Instruction descriptor: kind::f16 with bf16 A and B, float32 D, both
-// K-major, M = 128, N = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kSubN >> 3) << 17) |
-                            ((uint32_t)(kBM >> 4) << 24);
+// K-major, M = 128, N columns (a multiple of 16, at most 256).
+template <int N>
+constexpr uint32_t idesc_bf16()
+{
+    static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+}
 
+// D[128 x N] (+)= A[128 x 16] * B[N x 16]^T; B's N rows are consecutive
+// 128-byte rows (8-row groups 1024 bytes apart), as NSUB 128-row boxes of w
+// stored back to back are.
+template <int N>
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t acc)
 {
     asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
                  " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-                 :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(kIdesc), "r"(acc)
+                 :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc_bf16<N>()), "r"(acc)
                  : "memory");
 }
 // Arrives on `bar` when every MMA this thread issued before has completed.
@@ -202,7 +229,8 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // Shared memory (dynamic, 1024-byte aligned): the stage ring, the epilogue
-// boxes (two per epilogue warp), then the barriers.  Host and device agree.
+// boxes (kEpiBoxes per epilogue warp), then the barriers.  Host and device
+// agree.
 // WRES (weight-resident): the CTA's BN x K block of w (p.w_bytes, at most
 // kWMaxBytes) is loaded once and only x streams through the ring; every tile
 // of the CTA then has the same column tile.  The ring has p.stages stages
@@ -216,7 +244,7 @@ template <int NSUB, bool WRES> struct Cfg {
     static constexpr int kAcc = 2;                                 // TMEM accumulator buffers
     static constexpr int kTmemCols = 2 * kBN;
     static constexpr int kMaxKBlocks = kWMaxBytes / (NSUB * kBSubBytes);  // WRES: K blocks w may have
-    static constexpr int kEpiBytes = kEpiWarps * 2 * kBoxBytes;
+    static constexpr int kEpiBytes = kEpiWarps * kEpiBoxes * kBoxBytes;
     // full, empty per stage; accumulator full / empty; drain; w full
     static constexpr int kBarBytes = 8 * (2 * kMaxStages + 2 * kAcc + 2) + 16;
     // dynamic shared memory for a w area of w_bytes and `stages` stages
@@ -249,14 +277,34 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Adds bias[col .. col + 31] (0 past N) to v: lane i loads element i (one
-// coalesced load for the warp) and the values reach every lane by shuffles.
-__device__ __forceinline__ void add_bias32(const float *bias, int col, int N, int lane, float (&v)[32])
+// bias[col + lane] (0 past N or without a bias): one coalesced load for a
+// warp's 32 columns.
+__device__ __forceinline__ float bias_lane(const float *bias, int col, int N, int lane)
 {
-    const float mine = col + lane < N ? __ldg(bias + col + lane) : 0.f;
+    return (bias && col + lane < N) ? __ldg(bias + col + lane) : 0.f;
+}
+
+// Adds the 32 columns' bias to v: lane i holds element i (bias_lane), the
+// values reach every lane by shuffles.
+__device__ __forceinline__ void add_bias32(float mine, float (&v)[32])
+{
 #pragma unroll
     for (int i = 0; i < 32; ++i)
         v[i] += __shfl_sync(0xffffffffu, mine, i);
+}
+
+// Adds b[0 .. 31] (shared memory, 16-byte aligned; every lane reads the
+// same words, a broadcast) to v.
+__device__ __forceinline__ void add_bias32_smem(const float *b, float (&v)[32])
+{
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(b + i);
+        v[i] += t.x;
+        v[i + 1] += t.y;
+        v[i + 2] += t.z;
+        v[i + 3] += t.w;
+    }
 }
 
 template <int LK>
@@ -306,6 +354,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(wfull + 1);
     // query head: 1 / W_l or 1 / H_l of head column h, at h % (2 L K)
     __shared__ float colscale[2 * 32];
+    // weight-resident: the bias of the CTA's column tile (0 past N), added
+    // from shared memory (a shuffle per column costs the epilogue more than
+    // its whole tensor-memory read)
+    __shared__ __align__(16) float sbias[WRES ? C::kBN : 4];
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -325,6 +377,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
         mbar_init(wfull, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         abort_flag = 0;
+    }
+    if (WRES) {
+        const int nb0 = (blockIdx.x % p.n_tiles) * C::kBN;
+        for (int i = threadIdx.x; i < C::kBN; i += blockDim.x)
+            sbias[i] = (p.bias && nb0 + i < p.N) ? p.bias[nb0 + i] : 0.f;
     }
     if (p.epi == kEpiHead && threadIdx.x < 2 * p.LK) {
         const int j = threadIdx.x, l = ((j >> 1) & p.lk_mask) >> p.k_shift;
@@ -415,12 +472,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                                                  : a_base + kATileBytes;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint64_t ad = smem_desc(a_base + kk * 32);
-#pragma unroll
-                        for (int j = 0; j < NSUB; ++j) {
-                            const uint64_t bd = smem_desc(b_base + j * kBSubBytes + kk * 32);
-                            mma_bf16(d + j * kSubN, ad, bd, (kb > 0 || kk > 0) ? 1u : 0u);
-                        }
+                        // one MMA over all BN columns (the w sub-tiles are
+                        // consecutive rows of one operand)
+                        mma_bf16<C::kBN>(d, smem_desc(a_base + kk * 32), smem_desc(b_base + kk * 32),
+                                         (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(empty + s);  // frees the stage once these MMAs have read it
                 }
@@ -437,10 +492,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
         const int q = warp & 3;                     // TMEM lane quarter
         const int e = warp - 2;                     // epilogue warp index
         const int half = e >> 2;                    // which column chunks of the quarter
-        uint8_t *boxes = epi_smem + e * 2 * kBoxBytes;
+        uint8_t *boxes = epi_smem + e * kEpiBoxes * kBoxBytes;
         int nbox = 0, local = 0;
+        const int step = (p.epi == kEpiStore && p.out_bf16) ? 64 : 32;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
             const int buf = local % C::kAcc, use = local / C::kAcc;
+            const int m0 = (t / p.n_tiles) * kBM, n0 = (t % p.n_tiles) * C::kBN;
+            // this warp's bias values of the tile (chunks c0 = half*step +
+            // 2*step*k, 32 columns each), loaded before the accumulator wait
+            constexpr int kNb = WRES ? 1 : C::kBN / 32 / 2;
+            float bl[kNb];
+#pragma unroll
+            for (int k = 0; k < kNb; ++k) {
+                const int c = half * step + (k / (step / 32)) * 2 * step + (k % (step / 32)) * 32;
+                bl[k] = (!WRES && c < C::kBN) ? bias_lane(p.bias, n0 + c, p.N, lane) : 0.f;
+            }
             const bool ready = __all_sync(0xffffffffu, mbar_wait(acc_full + buf, use & 1) &&
                                                            !*(volatile int *)&abort_flag);
             if (!ready) {
@@ -451,7 +517,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                 break;
             }
             tc_fence_after();
-            const int m0 = (t / p.n_tiles) * kBM, n0 = (t % p.n_tiles) * C::kBN;
             const int row0 = m0 + 32 * q;           // first row of this warp
             const int r = row0 + lane;
             const uint32_t tbase = tmem + buf * C::kBN + ((uint32_t)(32 * q) << 16);
@@ -460,9 +525,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                 rx = __ldg(p.ref + 2 * (int64_t)r);
                 ry = __ldg(p.ref + 2 * (int64_t)r + 1);
             }
-            const int step = (p.epi == kEpiStore && p.out_bf16) ? 64 : 32;
 #pragma unroll 1
-            for (int c0 = half * step; c0 < C::kBN && n0 + c0 < p.N; c0 += 2 * step) {
+            for (int c0 = half * step, kc = 0; c0 < C::kBN && n0 + c0 < p.N; c0 += 2 * step, ++kc) {
                 float v[32], v2[32];
                 tmem_ld32(tbase + c0, v);
                 if (step == 64)
@@ -471,11 +535,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                 uint4 chunks[8];
                 const CUtensorMap *map = &map_o0;
                 int x = col;
+                // this chunk's bias values (kc < kNb: registers, no dynamic index)
+                float b0 = 0.f, b1 = 0.f;
+#pragma unroll
+                for (int k = 0; k < kNb; ++k) {
+                    if (k == kc * (step / 32))
+                        b0 = bl[k];
+                    if (step == 64 && k == kc * 2 + 1)
+                        b1 = bl[k];
+                }
                 if (p.epi == kEpiStore) {
-                    if (p.bias) {
-                        add_bias32(p.bias, col, p.N, lane, v);
+                    if (WRES) {
+                        if (p.bias) {
+                            add_bias32_smem(sbias + c0, v);
+                            if (step == 64)
+                                add_bias32_smem(sbias + c0 + 32, v2);
+                        }
+                    } else if (p.bias) {
+                        add_bias32(b0, v);
                         if (step == 64)
-                            add_bias32(p.bias, col + 32, p.N, lane, v2);
+                            add_bias32(b1, v2);
                     }
                     if (step == 64) {
 #pragma unroll
@@ -495,8 +574,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                     }
                 } else {
                     // query head: a 32-column chunk is all offsets or whole runs of logits
-                    if (p.bias)
-                        add_bias32(p.bias, col, p.N, lane, v);
+                    if (WRES)
+                        add_bias32_smem(sbias + c0, v);
+                    else if (p.bias)
+                        add_bias32(b0, v);
                     if (col < 2 * p.P) {
                         const int cmask = 2 * p.LK - 1;
 #pragma unroll
@@ -516,11 +597,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                     }
                     pack_f32(v, chunks);
                 }
-                // stage the box (double buffer: the store issued two boxes ago
-                // must have finished reading it) and store it with TMA
-                uint8_t *box = boxes + (nbox & 1) * kBoxBytes;
+                // stage the box (kEpiBoxes buffers: the store issued kEpiBoxes
+                // boxes ago must have finished reading it) and store it with TMA
+                uint8_t *box = boxes + (nbox % kEpiBoxes) * kBoxBytes;
                 if (lane == 0)
-                    tma_store_wait_read<1>();
+                    tma_store_wait_read<kEpiBoxes - 1>();
                 __syncwarp();
                 box_put_row(box, lane, chunks);
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
