@@ -332,8 +332,10 @@ msda_status launch_to_bf16(const float *src, void *dst, int64_t n, cudaStream_t 
 // (msda_kernels.cuh, forward_kernel SPLIT), taken for problems whose rows,
 // one lane group each, would not fill one resident wave of the unsplit
 // kernel.  Returns false (nothing launched) when the problem is larger.
+// The general kernels split on the same rule, so that a query order never
+// changes a row's summation order.
 template <typename T, int DD, bool FUSED, bool SHORT>
-bool try_forward_split(KernelArgs &a, cudaStream_t s, msda_status &st)
+bool try_forward_split(KernelArgs &a, bool gen, cudaStream_t s, msda_status &st)
 {
     constexpr int rpw0 = msda::forward_rows_per_warp<T, DD>();
     constexpr int rpw = rpw0 / MSDA_FWD_SPLIT;
@@ -346,8 +348,9 @@ bool try_forward_split(KernelArgs &a, cudaStream_t s, msda_status &st)
     const int64_t warps = (a.rows + rpw0 - 1) / rpw0;
     if (warps >= (int64_t)sms * msda::kMaxWarpsPerCta * msda::FwdTune<T, SHORT>::kMinCtas)
         return false;
-    st = launch_rows((const void *)msda::forward_kernel<T, DD, FUSED, false, SHORT, MSDA_FWD_SPLIT>, rpw,
-                     kForwardRecordBytes, a.L * a.K, false, a, s);
+    st = launch_rows(gen ? (const void *)msda::forward_kernel<T, DD, FUSED, true, SHORT, MSDA_FWD_SPLIT>
+                         : (const void *)msda::forward_kernel<T, DD, FUSED, false, SHORT, MSDA_FWD_SPLIT>,
+                     rpw, kForwardRecordBytes, a.L * a.K, false, a, s);
     return true;
 }
 
@@ -358,17 +361,18 @@ msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
 {
     const bool gen = a.order != nullptr || a.dcn != 0 || a.stage != 0;
     msda_status st = MSDA_OK;
-    if (!gen && p->value_dtype == MSDA_F32) {
-        if ((p->head_dim == 8 && try_forward_split<float, 8, FUSED, false>(a, s, st)) ||
-            (p->head_dim == 16 && try_forward_split<float, 16, FUSED, false>(a, s, st)) ||
-            (p->head_dim == 32 && try_forward_split<float, 32, FUSED, false>(a, s, st)))
+    // (staged inputs, a per-call option, need whole rows per lane group)
+    if (!a.stage && p->value_dtype == MSDA_F32) {
+        if ((p->head_dim == 8 && try_forward_split<float, 8, FUSED, false>(a, gen, s, st)) ||
+            (p->head_dim == 16 && try_forward_split<float, 16, FUSED, false>(a, gen, s, st)) ||
+            (p->head_dim == 32 && try_forward_split<float, 32, FUSED, false>(a, gen, s, st)))
             return st;
     }
-    if (!gen && p->value_dtype == MSDA_BF16 && a.L * a.K <= 16) {
-        if ((p->head_dim == 8 && try_forward_split<__nv_bfloat16, 8, FUSED, true>(a, s, st)) ||
-            (p->head_dim == 16 && try_forward_split<__nv_bfloat16, 16, FUSED, true>(a, s, st)) ||
-            (p->head_dim == 32 && try_forward_split<__nv_bfloat16, 32, FUSED, true>(a, s, st)) ||
-            (p->head_dim == 64 && try_forward_split<__nv_bfloat16, 64, FUSED, true>(a, s, st)))
+    if (!a.stage && p->value_dtype == MSDA_BF16 && a.L * a.K <= 16) {
+        if ((p->head_dim == 8 && try_forward_split<__nv_bfloat16, 8, FUSED, true>(a, gen, s, st)) ||
+            (p->head_dim == 16 && try_forward_split<__nv_bfloat16, 16, FUSED, true>(a, gen, s, st)) ||
+            (p->head_dim == 32 && try_forward_split<__nv_bfloat16, 32, FUSED, true>(a, gen, s, st)) ||
+            (p->head_dim == 64 && try_forward_split<__nv_bfloat16, 64, FUSED, true>(a, gen, s, st)))
             return st;
     }
 #define MSDA_FWD_CASE(T, DD)                                                                      \

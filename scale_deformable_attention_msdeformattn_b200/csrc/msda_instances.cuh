@@ -18,11 +18,13 @@
     MSDA_FWD_D(PFX, T, 8, SHORT) MSDA_FWD_D(PFX, T, 16, SHORT) MSDA_FWD_D(PFX, T, 32, SHORT) \
     MSDA_FWD_D(PFX, T, 64, SHORT) MSDA_FWD_D(PFX, T, 128, SHORT) MSDA_FWD_D(PFX, T, 256, SHORT)
 
-// forward_kernel<T, D, FUSED, false, SHORT, SPLIT>: rows split over SPLIT
-// lane groups (plain kernels, head dims whose rows leave room in a warp)
+// forward_kernel<T, D, FUSED, GEN, SHORT, SPLIT>: rows split over SPLIT
+// lane groups (head dims whose rows leave room in a warp)
 #define MSDA_FWD_SPLIT_D(PFX, T, D, SHORT, SPLIT)                                                   \
     PFX template __global__ void forward_kernel<T, D, false, false, SHORT, SPLIT>(const KernelArgs); \
-    PFX template __global__ void forward_kernel<T, D, true, false, SHORT, SPLIT>(const KernelArgs);
+    PFX template __global__ void forward_kernel<T, D, false, true, SHORT, SPLIT>(const KernelArgs);  \
+    PFX template __global__ void forward_kernel<T, D, true, false, SHORT, SPLIT>(const KernelArgs);  \
+    PFX template __global__ void forward_kernel<T, D, true, true, SHORT, SPLIT>(const KernelArgs);
 #define MSDA_FWD_SPLIT_INSTANCES(PFX)                                                             \
     MSDA_FWD_SPLIT_D(PFX, float, 8, false, MSDA_FWD_SPLIT)                                         \
     MSDA_FWD_SPLIT_D(PFX, float, 16, false, MSDA_FWD_SPLIT)                                        \

@@ -1181,7 +1181,7 @@ template <bool SHORT> struct FwdTune<S8, SHORT> {
 // with those branches removed at compile time; GEN = true honours
 // KernelArgs::order and KernelArgs::dcn.
 //
-// SPLIT > 1 (plain kernels only): SPLIT lane groups share a row, group ph
+// SPLIT > 1: SPLIT lane groups share a row, group ph
 // gathering samples ph*U .. ph*U + U-1, then (ph + SPLIT)*U ..., and the
 // partial sums meet in a shuffle reduction before group 0 stores the row.
 // For problems with too few rows to fill the GPU (the decoder's 300 queries
@@ -1202,7 +1202,7 @@ forward_kernel(const KernelArgs a_in)
     using Raw = typename Lay::Raw;
     constexpr int G = Lay::kG, CH = Lay::kCh, E = Lay::kLaneElems, EPV = Lay::kEpv;
     constexpr int U = Tune::kInFlight;  // samples in flight per lane (4 corners each)
-    static_assert(SPLIT == 1 || (!GEN && SPLIT * G <= 32), "row split: plain kernels, G * SPLIT <= 32");
+    static_assert(SPLIT == 1 || SPLIT * G <= 32, "row split: G * SPLIT <= 32");
     constexpr int GS = G * SPLIT;       // lanes of one row
 
     extern __shared__ __align__(16) unsigned char smem_raw[];

@@ -44,6 +44,11 @@ LINEAR = [
     (300, 136, 600, True, "f32"),
     (4099, 256, 256, True, "bf16"),
     (255, 64, 40, False, "bf16"),
+    # w too large to stay in shared memory (more than 4 K blocks at 256
+    # output columns, more than 8 at 128): w streams through the ring with x
+    (513, 320, 256, True, "f32"),
+    (1000, 384, 256, False, "f32"),
+    (300, 576, 104, True, "bf16"),
 ]
 
 
