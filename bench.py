@@ -48,9 +48,9 @@ L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 # hash of the CUDA sources it was taken from and is reported only while those
 # sources are unchanged.  Filled from the summaries under profiles/.
 NCU_TRAFFIC = {
-    # profiles/detr_encoder_f32_fused_kernels.md: 107.66 MB read + 18.59 MB written
-    ("fused_backward", "detr_encoder_f32"): {"bytes": 126254080, "csrc": "9bfe38b88dbda604"},
-    ("fused_forward", "detr_encoder_f32"): {"bytes": 60058880, "csrc": "9bfe38b88dbda604"},
+    # profiles/detr_encoder_f32_fused_kernels.md: mean of two launches, DRAM read + write
+    ("fused_backward", "detr_encoder_f32"): {"bytes": 127103488, "csrc": "82b094a66de9ae01"},
+    ("fused_forward", "detr_encoder_f32"): {"bytes": 59862656, "csrc": "82b094a66de9ae01"},
     # profiles/dcnv3_stage1_f32_kernels.md: 122.08 MB read + 18.45 MB written
     ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 140523776, "csrc": "9bfe38b88dbda604"},
     ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 72899072, "csrc": "9bfe38b88dbda604"},
