@@ -51,9 +51,15 @@ NCU_TRAFFIC = {
     # profiles/detr_encoder_f32_fused_kernels.md: mean of two launches, DRAM read + write
     ("fused_backward", "detr_encoder_f32"): {"bytes": 127103488, "csrc": "82b094a66de9ae01"},
     ("fused_forward", "detr_encoder_f32"): {"bytes": 59862656, "csrc": "82b094a66de9ae01"},
-    # profiles/dcnv3_stage1_f32_kernels.md: 122.08 MB read + 18.45 MB written
-    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 140523776, "csrc": "9bfe38b88dbda604"},
-    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 72899072, "csrc": "9bfe38b88dbda604"},
+    # profiles/detr_decoder_bf16_kernels.md: DRAM read + write of one launch
+    ("fused_backward", "detr_decoder_bf16"): {"bytes": 138262272, "csrc": "82b094a66de9ae01"},
+    ("fused_forward", "detr_decoder_bf16"): {"bytes": 51268096, "csrc": "82b094a66de9ae01"},
+    # profiles/stress_1080p_k8_bf16_fused_kernels.md: DRAM read + write of one launch
+    ("fused_backward", "stress_1080p_k8_bf16"): {"bytes": 925939712, "csrc": "82b094a66de9ae01"},
+    ("fused_forward", "stress_1080p_k8_bf16"): {"bytes": 381244928, "csrc": "82b094a66de9ae01"},
+    # profiles/dcnv3_stage1_f32_kernels.md: DRAM read + write of one launch
+    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 143730688, "csrc": "82b094a66de9ae01"},
+    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 73360896, "csrc": "82b094a66de9ae01"},
 }
 
 

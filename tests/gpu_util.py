@@ -83,6 +83,11 @@ def elem_err(gpu, ref, floor: float = ELEM_FLOOR) -> float:
     return float((np.abs(g - r) / np.maximum(np.abs(r), floor * scale)).max())
 
 
+# (what, normwise error, elementwise error) of every assert_close call, for
+# the run's summary table (tests/conftest.py)
+RECORDS = []
+
+
 def assert_close(gpu, ref, tol, what, elem_tol=None, floor=ELEM_FLOOR):
     """Asserts the normwise error <= tol and the elementwise error <= elem_tol
     (default: ELEM_TOL for bf16 tensors, else for float32) with the given
@@ -93,6 +98,7 @@ def assert_close(gpu, ref, tol, what, elem_tol=None, floor=ELEM_FLOOR):
         elem_tol = ELEM_TOL["bf16" if is_bf16 else "f32"]
     ee = elem_err(gpu, ref, floor)
     print(f"  {what}: normwise {e:.2e} elementwise {ee:.2e}")
+    RECORDS.append((what, e, ee))
     assert e <= tol, f"{what}: max relative error {e:.3e} > {tol:.1e}"
     assert ee <= elem_tol, f"{what}: elementwise relative error {ee:.3e} > {elem_tol:.1e}"
     return e

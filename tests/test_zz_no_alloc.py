@@ -85,10 +85,10 @@ def test_noalloc_matches_workspace_backward(spec):
         # against the oracle: grad_value is its float64 sum rounded to bf16 up
         # to one rounding step (at most 2^-7 of the value), the other
         # gradients at the workload's bounds
-        assert_close(gv, bf16_round(o_gv), 2.0 ** -7, f"call {call}: grad_value vs rounded oracle",
+        assert_close(gv, bf16_round(o_gv), 2.0 ** -7, f"no-alloc call {call}: grad_value vs rounded oracle",
                      elem_tol=2.0 ** -7)
-        assert_close(gl, o_gl, TOL[w.dtype], f"call {call}: grad_loc vs oracle")
-        assert_close(ga, o_ga, TOL[w.dtype], f"call {call}: grad_attn vs oracle")
+        assert_close(gl, o_gl, TOL[w.dtype], f"no-alloc call {call}: grad_loc vs oracle")
+        assert_close(ga, o_ga, TOL[w.dtype], f"no-alloc call {call}: grad_attn vs oracle")
 
     code = ctypes.c_int32(-1)
     assert lib.msda_get_device_status(_stream(), ctypes.byref(code)) == 0 and code.value == 0
