@@ -58,6 +58,11 @@ def _load():
             lib.msda_oracle_softmax.argtypes = [D, P, P]
             lib.msda_oracle_fused_chain.argtypes = [D, P, P, P, P, P, P, P]
             lib.msda_oracle_quantize_value_s8.argtypes = [D, P, P, P]
+            lib.msda_oracle_quantize_value_e4m3.argtypes = [D, P, P, P]
+            lib.msda_oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.msda_oracle_e4m3_encode.restype = ctypes.c_ubyte
+            lib.msda_oracle_e4m3_decode.argtypes = [ctypes.c_ubyte]
+            lib.msda_oracle_e4m3_decode.restype = ctypes.c_double
             DD = ctypes.POINTER(_DcnDims)
             lib.msda_oracle_dcn_forward.argtypes = [DD, P, P, P, P]
             lib.msda_oracle_dcn_backward.argtypes = [DD, P, P, P, P, P, P, P]
@@ -66,7 +71,8 @@ def _load():
             lib.msda_oracle_linear_backward.argtypes = [I, I, I, P, P, P, P, P, P]
             for f in ("msda_oracle_forward", "msda_oracle_backward", "msda_oracle_sampling_locations",
                       "msda_oracle_softmax", "msda_oracle_fused_chain",
-                      "msda_oracle_quantize_value_s8", "msda_oracle_dcn_forward",
+                      "msda_oracle_quantize_value_s8", "msda_oracle_quantize_value_e4m3",
+                      "msda_oracle_dcn_forward",
                       "msda_oracle_dcn_backward", "msda_oracle_linear",
                       "msda_oracle_linear_backward"):
                 getattr(lib, f).restype = None
@@ -203,6 +209,48 @@ def quantize_value_s8(value):
 def dequantize_value_s8(q, scale):
     """q * scale in float64 (exact), [B,S,M,D]: the value the operator samples."""
     return np.asarray(q, np.float64) * np.asarray(scale, np.float64)[:, None, :, None]
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 codes (uint8) of float32 values (finite), elementwise: the
+    nearest representable value, ties to the even mantissa, clipped to +-448."""
+    lib = _load()
+    x = np.asarray(x, np.float32)
+    return np.array([lib.msda_oracle_e4m3_encode(float(v)) for v in x.ravel()], np.uint8).reshape(x.shape)
+
+
+_e4m3_table = None
+
+
+def e4m3_decode(c) -> np.ndarray:
+    """The float64 values of E4M3 codes (NaN codes give NaN)."""
+    global _e4m3_table
+    if _e4m3_table is None:
+        lib = _load()
+        _e4m3_table = np.array([lib.msda_oracle_e4m3_decode(i) for i in range(256)], np.float64)
+    return _e4m3_table[np.asarray(c, np.uint8)]
+
+
+def quantize_value_e4m3(value):
+    """FP8 (E4M3) value storage: (codes uint8 [B,S,M,D], scale float32 [B,M])
+    with one absmax scale per (batch, head), amax / 448.  `value` is float32,
+    or bfloat16 bit patterns (uint16), widened exactly to float32."""
+    v = np.asarray(value)
+    if v.dtype == np.uint16:
+        v = (v.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    B, S, M, D = v.shape
+    d = _Dims(B, S, 0, M, D, 0, 0)
+    q = np.empty(v.shape, np.uint8)
+    scale = np.empty((B, M), np.float32)
+    _load().msda_oracle_quantize_value_e4m3(ctypes.byref(d), _p(v), _p(q), _p(scale))
+    return q, scale
+
+
+def dequantize_value_e4m3(q, scale):
+    """decode(q) * scale in float64 (exact), [B,S,M,D]: the value the operator
+    samples."""
+    return e4m3_decode(q) * np.asarray(scale, np.float64)[:, None, :, None]
 
 
 def dcn_output_size(H: int, W: int, kernel, stride=(1, 1), pad=(0, 0), dil=(1, 1)):

@@ -333,6 +333,86 @@ void msda_oracle_quantize_value_s8(const oracle_dims *d, const float *value, int
 }
 
 /*
+ * FP8 value storage, the other low-precision format of the same note
+ * ([csdn] §4).  Format: the E4M3 encoding of the OCP 8-bit floating-point
+ * specification (v1.0): bit 7 the sign, bits 6..3 a biased exponent (bias 7),
+ * bits 2..0 a mantissa; exponent field e > 0 encodes (1 + m/8) * 2^(e - 7),
+ * e = 0 encodes the subnormals (m/8) * 2^-6; S.1111.111 is NaN and there is no
+ * infinity, so the largest finite magnitude is S.1111.110 = 1.75 * 2^8 = 448.
+ * Reading taken (listed with the others): the INT8 scheme above with 448 in
+ * place of 127 -- scale = amax / 448 (1 when amax == 0), x = value / scale in
+ * float32, the code the E4M3 value nearest to x (ties to the even mantissa),
+ * magnitudes above 448 clipped to 448 ("satfinite"); the sign of x is kept
+ * when x rounds to zero.
+ */
+
+/* The E4M3 code of the float x (finite), from the definition above: the
+ * representable magnitudes around |x| are multiples of the quantum 2^(E-3)
+ * of |x|'s binade E (E >= -6; the subnormals share the quantum 2^-9). */
+unsigned char msda_oracle_e4m3_encode(float x)
+{
+    const unsigned char sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0)
+        return (unsigned char)(sign | 0x7E);
+    int E = -6;                               /* binade: 2^E <= a < 2^(E+1) */
+    if (a >= ldexp(1.0, -6)) {
+        (void)frexp(a, &E);                   /* a = f * 2^E, f in [0.5, 1) */
+        E -= 1;
+    }
+    const double quantum = ldexp(1.0, E - 3);
+    double r = nearbyint(a / quantum);        /* a / quantum is exact; half to even */
+    /* r counts quanta of binade E: subnormals 0..8, normals 8..16 (16 carries
+     * into the next binade, whose mantissa is then 0) */
+    if (a < ldexp(1.0, -6)) {                 /* subnormal range */
+        if (r >= 8.0)
+            return (unsigned char)(sign | (1 << 3));      /* rounds up to 2^-6 */
+        return (unsigned char)(sign | (unsigned)r);
+    }
+    if (r >= 16.0) {
+        E += 1;
+        r = 8.0;
+    }
+    if (E > 8 || (E == 8 && r > 14.0))        /* beyond 448: clip */
+        return (unsigned char)(sign | 0x7E);
+    return (unsigned char)(sign | ((unsigned)(E + 7) << 3) | (unsigned)(r - 8.0));
+}
+
+/* The value of an E4M3 code (NaN codes return NaN). */
+double msda_oracle_e4m3_decode(unsigned char c)
+{
+    const int e = (c >> 3) & 15, m = c & 7;
+    const double sgn = (c & 0x80) ? -1.0 : 1.0;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        return sgn * ldexp((double)m, -9);
+    return sgn * ldexp(8.0 + m, e - 10);
+}
+
+void msda_oracle_quantize_value_e4m3(const oracle_dims *d, const float *value, unsigned char *q,
+                                     float *scale)
+{
+    for (int64_t b = 0; b < d->B; ++b)
+        for (int64_t m = 0; m < d->M; ++m) {
+            float amax = 0.0f;
+            for (int64_t s = 0; s < d->S; ++s)
+                for (int64_t c = 0; c < d->D; ++c) {
+                    const float a = fabsf(value[((b * d->S + s) * d->M + m) * d->D + c]);
+                    if (a > amax)
+                        amax = a;
+                }
+            const float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+            scale[b * d->M + m] = sc;
+            for (int64_t s = 0; s < d->S; ++s)
+                for (int64_t c = 0; c < d->D; ++c) {
+                    const int64_t i = ((b * d->S + s) * d->M + m) * d->D + c;
+                    q[i] = msda_oracle_e4m3_encode(value[i] / sc);
+                }
+        }
+}
+
+/*
  * DCNv3 core ([discosf] §4.2): for output pixel p0 = (i, j) of image n and
  * group g,
  *   y[n,i,j,g,:] = sum_k m[n,i,j,g,k] * x_g(p0 + p_k + dp[n,i,j,g,k])

@@ -15,6 +15,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_dcn as dcn_pins
+from tests import test_oracle_fp8 as fp8_pins
 from tests import test_oracle_linear as linear_pins
 from tests import test_oracle_pins as pins
 
@@ -98,6 +99,22 @@ DCN_PIN_CHECKS = [
 ]
 
 
+FP8_MUTATIONS = {
+    "e4m3_exponent_bias_8": ("((unsigned)(E + 7) << 3)", "((unsigned)(E + 8) << 3)"),
+    "e4m3_ties_away_from_zero": ("double r = nearbyint(a / quantum);", "double r = round(a / quantum);"),
+    "e4m3_overflow_to_nan": ("    if (a >= 448.0)\n        return (unsigned char)(sign | 0x7E);",
+                             "    if (a >= 448.0)\n        return (unsigned char)(sign | 0x7F);"),
+    "e4m3_scale_127": ("amax > 0.0f ? amax / 448.0f : 1.0f", "amax > 0.0f ? amax / 127.0f : 1.0f"),
+}
+
+FP8_PIN_CHECKS = [
+    lambda o: fp8_pins.test_spec_values(),
+    lambda o: fp8_pins.test_every_code_round_trips(),
+    lambda o: fp8_pins.test_ties_and_neighbours_match_brute_force(),
+    lambda o: fp8_pins.test_matches_torch_float8_conversion(),
+    lambda o: fp8_pins.test_quantiser_scale_and_error_bound(),
+]
+
 LINEAR_PIN_CHECKS = [
     linear_pins.test_golden_worked_linear,
     linear_pins.test_identity_and_zero_weights,
@@ -114,24 +131,30 @@ def _swapped(lib_path):
     lib = ctypes.CDLL(lib_path)
     for name in ("msda_oracle_forward", "msda_oracle_backward", "msda_oracle_sampling_locations",
                  "msda_oracle_softmax", "msda_oracle_fused_chain", "msda_oracle_dcn_forward",
-                 "msda_oracle_dcn_backward", "msda_oracle_linear", "msda_oracle_linear_backward"):
+                 "msda_oracle_dcn_backward", "msda_oracle_linear", "msda_oracle_linear_backward",
+                 "msda_oracle_e4m3_encode", "msda_oracle_e4m3_decode",
+                 "msda_oracle_quantize_value_e4m3"):
         f, ref = getattr(lib, name), getattr(saved, name)
         f.argtypes, f.restype = ref.argtypes, ref.restype
     oracle._lib = lib
+    saved_table, oracle._e4m3_table = oracle._e4m3_table, None
     try:
         yield
     finally:
         oracle._lib = saved
+        oracle._e4m3_table = saved_table
 
 
-ALL_MUTATIONS = {**MUTATIONS, **DCN_MUTATIONS, **LINEAR_MUTATIONS}
+ALL_MUTATIONS = {**MUTATIONS, **DCN_MUTATIONS, **LINEAR_MUTATIONS, **FP8_MUTATIONS}
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(DCN_MUTATIONS) + sorted(LINEAR_MUTATIONS))
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(DCN_MUTATIONS) + sorted(LINEAR_MUTATIONS)
+                         + sorted(FP8_MUTATIONS))
 def test_planted_mistake_is_caught(name, tmp_path):
     old, new = ALL_MUTATIONS[name]
     checks = (PIN_CHECKS if name in MUTATIONS else
-              DCN_PIN_CHECKS if name in DCN_MUTATIONS else LINEAR_PIN_CHECKS)
+              DCN_PIN_CHECKS if name in DCN_MUTATIONS else
+              LINEAR_PIN_CHECKS if name in LINEAR_MUTATIONS else FP8_PIN_CHECKS)
     src = open(SRC).read()
     assert src.count(old) == 1, name
     mutated = tmp_path / "mut.c"
