@@ -113,8 +113,8 @@ def parse_args(argv=None):
 def algorithmic_bytes(w: wl.Workload) -> dict:
     """Each tensor of a launch touched once (inputs read, outputs written)."""
     B, S, Q, M, D, L, K = w.B, w.S, w.num_queries, w.M, w.D, w.L, w.K
-    e = {"f32": 4, "bf16": 2, "s8": 1}[w.dtype]       # value element
-    er = {"f32": 4, "bf16": 2, "s8": 2}[w.dtype]      # output / grad_output element
+    e = {"f32": 4, "bf16": 2, "s8": 1, "e4m3": 1}[w.dtype]       # value element
+    er = {"f32": 4, "bf16": 2, "s8": 2, "e4m3": 2}[w.dtype]      # output / grad_output element
     value = B * S * M * D * e
     rowd = B * Q * M * D * er
     samples = B * Q * M * L * K
@@ -127,7 +127,7 @@ def algorithmic_bytes(w: wl.Workload) -> dict:
     fused_fwd = value + loc + attn + ref + rowd             # offsets, logits, ref -> out
     fused_bwd = rowd + value + loc + attn + ref + gvalue + loc + attn + ref
     # INT8 storage: the bf16 source read once, the codes written once
-    quantize = B * S * M * D * 3 if w.dtype == "s8" else 0
+    quantize = B * S * M * D * 3 if w.dtype in ("s8", "e4m3") else 0
     return {"forward": fwd, "backward": bwd, "fused_forward": fused_fwd,
             "fused_backward": fused_bwd, "zero_grads": gvalue + ref, "quantize": quantize}
 
@@ -309,8 +309,14 @@ def run_ours(args):
 
     side = torch.cuda.Stream(device=dev)
     order = torch.empty(B * Q, dtype=torch.int32, device=dev) if args.sorted else None
-    int8 = w.dtype == "s8"
-    qv = torch.empty((B, S, M, D), dtype=torch.int8, device=dev) if int8 else None
+    # one-byte value storage: the step's value arrives as bf16 and is stored
+    # as INT8 or FP8 codes with a (batch, head) scale
+    int8 = w.dtype in ("s8", "e4m3")
+    qdtype, quantize = ((torch.int8, lambda v, q, sc: msda.quantize_value_s8(v, value_s8=q, value_scale=sc))
+                        if w.dtype == "s8" else
+                        (torch.float8_e4m3fn,
+                         lambda v, q, sc: msda.quantize_value_e4m3(v, value_e4m3=q, value_scale=sc)))
+    qv = torch.empty((B, S, M, D), dtype=qdtype, device=dev) if int8 else None
     qs = torch.empty((B, M), dtype=torch.float32, device=dev) if int8 else None
 
     nbytes = algorithmic_bytes(w)
@@ -328,8 +334,8 @@ def run_ours(args):
         ev[0].record(stream)
         if order is not None:
             msda.sort_queries(tin["reference_points"], query_order=order)
-        if int8:  # the step's value arrives as bf16 and is stored as INT8
-            msda.quantize_value_s8(tin["value"], value_s8=qv, value_scale=qs)
+        if int8:  # the step's value arrives as bf16 and is stored in one byte
+            quantize(tin["value"], qv, qs)
         value = qv if int8 else tin["value"]
         ev[6].record(stream)
         msda.fused_forward(value, tin["spatial_shapes"], tin["level_start_index"],
@@ -416,7 +422,8 @@ def run_ours(args):
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": {"f32": "f32", "bf16": "bf16 value / f32 accumulate",
-                      "s8": "int8 value (per batch-head scale) / bf16 rows / f32 accumulate"}[w.dtype],
+                      "s8": "int8 value (per batch-head scale) / bf16 rows / f32 accumulate",
+                      "e4m3": "fp8 e4m3 value (per batch-head scale) / bf16 rows / f32 accumulate"}[w.dtype],
             "data": "synthetic: seeded SplitMix64 + Box-Muller draws of the workload's shapes "
                     "and distributions (no dataset)",
             "config": {
@@ -425,7 +432,7 @@ def run_ours(args):
                 "offset_sigma_px": w.offset_sigma, "logit_sigma": w.logit_sigma,
                 "samples_per_step_per_gpu": samples_step,
                 "step": ("msda_sort_queries -> " if args.sorted else "")
-                + ("msda_quantize_value_s8 -> " if int8 else "")
+                + (f"msda_quantize_value_{w.dtype} -> " if int8 else "")
                 + ("msda_fused_forward || msda_zero_grads (second stream) -> msda_fused_backward"
                    if overlap else "msda_fused_forward -> msda_zero_grads -> msda_fused_backward"),
                 "query_order": "Morton cell of the reference point" if args.sorted else "natural",
@@ -458,7 +465,7 @@ def run_ours(args):
         }
         if want_nonfused:
             if int8:
-                msda.quantize_value_s8(t["value"], value_s8=qv, value_scale=qs)
+                quantize(t["value"], qv, qs)
             result["nonfused"] = _time_nonfused(msda, t, w, nbytes, flush, min(args.steps, 50),
                                                 qv if int8 else t["value"], qs)
         if world == 1:
@@ -684,7 +691,7 @@ def _input_stats(w: wl.Workload, x: wl.Inputs, max_queries: int = 4096) -> dict:
         start = x.level_start_index[None, None, None, :, None]
         b = np.arange(w.B)[:, None, None, None, None]
         m = np.arange(w.M)[None, None, :, None, None]
-        elt = {"f32": 4, "bf16": 2, "s8": 1}[w.dtype]
+        elt = {"f32": 4, "bf16": 2, "s8": 1, "e4m3": 1}[w.dtype]
         row_bytes = w.D * elt
         rows = []
         for dy in (0, 1):

@@ -33,7 +33,8 @@
  *     move in 32-byte vectors).  The library keeps no pointer after the call
  *     returns and allocates no memory.
  *   - value, output and grad_output hold value_dtype elements (float32 or
- *     bfloat16; with MSDA_S8 value, output and grad_output are bfloat16);
+ *     bfloat16; with MSDA_S8 or MSDA_E4M3 value, output and grad_output are
+ *     bfloat16);
  *     every other floating-point tensor is float32.  Accumulation is float32.
  *   - Locations and offsets are (x, y) pairs; spatial_shapes rows are (H, W).
  *   - spatial_shapes [L,2] and level_start_index [L] are int64 device arrays.
@@ -102,7 +103,14 @@ typedef enum msda_dtype {
      * and grad_output are bfloat16; grad_value is the gradient with respect
      * to the dequantized value (float32, or bf16 with MSDA_GRAD_VALUE_BF16).
      * msda_quantize_value_s8 produces q and the scales. */
-    MSDA_S8 = 2
+    MSDA_S8 = 2,
+    /* FP8 value storage (the same note's low-precision storage): value is one
+     * E4M3 code per element (the OCP 8-bit floating-point E4M3 encoding:
+     * sign, 4 exponent bits with bias 7, 3 mantissa bits, largest finite
+     * 448, no infinity) with one float32 scale per (batch, head) in
+     * msda_problem.value_scale; otherwise as MSDA_S8.
+     * msda_quantize_value_e4m3 produces the codes and the scales. */
+    MSDA_E4M3 = 3
 } msda_dtype;
 
 /* msda_problem.flags */
@@ -162,7 +170,7 @@ typedef struct msda_problem {
      * detected (the rows of queries missing from the order are not written).
      * Read by the kernels on the stream: it must stay valid until they end. */
     const int32_t *query_order;
-    /* MSDA_S8 value only (ignored otherwise, required then): device array
+    /* MSDA_S8 / MSDA_E4M3 value only (ignored otherwise, required then): device array
      * [B, M] float32, 4-byte aligned, the dequantization scale of each
      * (batch, head).  Read by the kernels on the stream. */
     const float *value_scale;
@@ -312,6 +320,25 @@ MSDA_API msda_status msda_backward_noalloc(const msda_problem *problem, const vo
 MSDA_API msda_status msda_quantize_value_s8(const msda_problem *problem, const void *value,
                                             void *value_s8, float *value_scale,
                                             msda_stream_t stream);
+
+/*
+ * FP8 value storage for MSDA_E4M3 (the same note): for each (batch b, head m)
+ *   amax  = max over keys s and channels d of |value[b, s, m, d]|
+ *   scale = amax / 448 (float32 division), 1 when amax = 0
+ *   code  = the E4M3 value nearest to value / scale (float32 division), ties
+ *           to the even mantissa, magnitudes above 448 clipped to 448, the
+ *           sign kept when the quotient rounds to zero
+ *   value        [B, S, M, D]  problem->value_dtype (MSDA_F32 or MSDA_BF16),
+ *                              finite, 16-byte aligned
+ *   value_e4m3   [B, S, M, D]  one byte per element, written, 32-byte aligned
+ *   value_scale  [B, M]        float32, written (also used as scratch)
+ * D must be a multiple of 8.  Four operations on `stream`, as
+ * msda_quantize_value_s8.  Non-finite inputs give unspecified codes and
+ * scales.
+ */
+MSDA_API msda_status msda_quantize_value_e4m3(const msda_problem *problem, const void *value,
+                                              void *value_e4m3, float *value_scale,
+                                              msda_stream_t stream);
 
 /*
  * Processing order that keeps spatially close queries together (the optional

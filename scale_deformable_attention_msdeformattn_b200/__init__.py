@@ -22,6 +22,7 @@ from .binding import (  # noqa: F401
     fused_forward,
     linear,
     ms_deform_attn,
+    quantize_value_e4m3,
     quantize_value_s8,
     query_head,
     query_head_backward,

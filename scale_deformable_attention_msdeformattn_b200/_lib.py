@@ -21,6 +21,7 @@ MSDA_ERR_DEVICE_BOUNDS = 6
 MSDA_F32 = 0
 MSDA_BF16 = 1
 MSDA_S8 = 2
+MSDA_E4M3 = 3
 
 MSDA_GRAD_VALUE_BF16 = 1 << 0
 MSDA_ACCUMULATE_GRADS = 1 << 1
@@ -81,6 +82,7 @@ _SIGNATURES = {
     "msda_backward_noalloc": [_PROB, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "msda_sort_queries": [_PROB, _P, _P, _P],
     "msda_quantize_value_s8": [_PROB, _P, _P, _P, _P],
+    "msda_quantize_value_e4m3": [_PROB, _P, _P, _P, _P],
     "msda_dcn_output_size": [_DCN, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)],
     "msda_dcn_forward": [_DCN, _P, _P, _P, _P, _P],
     "msda_dcn_backward": [_DCN, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],

@@ -65,12 +65,15 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None, device=None):
     return t
 
 
-_DTYPES = {torch.float32: _lib.MSDA_F32, torch.bfloat16: _lib.MSDA_BF16, torch.int8: _lib.MSDA_S8}
+_DTYPES = {torch.float32: _lib.MSDA_F32, torch.bfloat16: _lib.MSDA_BF16, torch.int8: _lib.MSDA_S8,
+           torch.float8_e4m3fn: _lib.MSDA_E4M3}
+# one-byte value storage: codes times a (batch, head) scale (value_scale)
+_SCALED = (torch.int8, torch.float8_e4m3fn)
 
 
 def _row_dtype(value: torch.Tensor):
-    """dtype of output / grad_output: value's, bfloat16 for INT8 value."""
-    return torch.bfloat16 if value.dtype == torch.int8 else value.dtype
+    """dtype of output / grad_output: value's, bfloat16 for one-byte value."""
+    return torch.bfloat16 if value.dtype in _SCALED else value.dtype
 
 
 def _problem(value: torch.Tensor, Q: int, L: int, K: int, flags: int = 0,
@@ -79,12 +82,13 @@ def _problem(value: torch.Tensor, Q: int, L: int, K: int, flags: int = 0,
     if value.dim() != 4:
         raise ValueError("value must be [B, S, M, D]")
     if value.dtype not in _DTYPES:
-        raise TypeError("value must be float32, bfloat16 or int8 (with value_scale)")
+        raise TypeError("value must be float32, bfloat16, int8 or float8_e4m3fn (with value_scale)")
     B, S, M, D = value.shape
     prob = _lib.Problem(B, S, Q, M, D, L, K, _DTYPES[value.dtype], flags)
-    if value.dtype == torch.int8:
+    if value.dtype in _SCALED:
         if value_scale is None:
-            raise ValueError("int8 value needs value_scale [B, M] (see quantize_value_s8)")
+            raise ValueError("one-byte value needs value_scale [B, M] "
+                             "(see quantize_value_s8, quantize_value_e4m3)")
         _need(value_scale, "value_scale", torch.float32, (B, M), value.device)
         prob.value_scale = _ptr(value_scale)
     if query_order is not None:
@@ -110,7 +114,7 @@ def forward(value: torch.Tensor, spatial_shapes: torch.Tensor, level_start_index
             query_order: Optional[torch.Tensor] = None,
             value_scale: Optional[torch.Tensor] = None) -> torch.Tensor:
     """msda_forward: returns out [B, Q, M, D] in value's dtype (bfloat16 for
-    int8 value, which needs value_scale [B, M]).  query_order: optional int32
+    one-byte value, which needs value_scale [B, M]).  query_order: optional int32
     [B*Q] processing order (see sort_queries)."""
     _need(value, "value", None)
     L = _geometry(value, spatial_shapes, level_start_index)
@@ -346,6 +350,29 @@ def quantize_value_s8(value: torch.Tensor, value_s8: Optional[torch.Tensor] = No
     return value_s8, value_scale
 
 
+def quantize_value_e4m3(value: torch.Tensor, value_e4m3: Optional[torch.Tensor] = None,
+                        value_scale: Optional[torch.Tensor] = None):
+    """msda_quantize_value_e4m3: (float8_e4m3fn value [B, S, M, D], float32
+    scale [B, M]) from a float32 or bfloat16 value, one absmax scale per
+    (batch, head), amax / 448; pass both to the other calls
+    (value_scale=...)."""
+    _need(value, "value", None)
+    if value.dim() != 4 or value.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("value must be a float32 or bfloat16 [B, S, M, D] tensor")
+    B, S, M, D = value.shape
+    if value_e4m3 is None:
+        value_e4m3 = torch.empty((B, S, M, D), dtype=torch.float8_e4m3fn, device=value.device)
+    if value_scale is None:
+        value_scale = torch.empty((B, M), dtype=torch.float32, device=value.device)
+    _need(value_e4m3, "value_e4m3", torch.float8_e4m3fn, (B, S, M, D), value.device)
+    _need(value_scale, "value_scale", torch.float32, (B, M), value.device)
+    prob = _lib.Problem(B, S, 1, M, D, 1, 1, _DTYPES[value.dtype], 0)
+    st = _lib.load().msda_quantize_value_e4m3(ctypes.byref(prob), _ptr(value), _ptr(value_e4m3),
+                                              _ptr(value_scale), _stream())
+    _check(st, "msda_quantize_value_e4m3")
+    return value_e4m3, value_scale
+
+
 def _pair(v):
     return (int(v), int(v)) if isinstance(v, int) else (int(v[0]), int(v[1]))
 
@@ -354,13 +381,14 @@ def _dcn_problem(input: torch.Tensor, kernel, stride, pad, dilation, flags=0, va
     if input.dim() != 5:
         raise ValueError("input must be [N, H, W, G, C]")
     if input.dtype not in _DTYPES:
-        raise TypeError("input must be float32, bfloat16 or int8 (with value_scale)")
+        raise TypeError("input must be float32, bfloat16, int8 or float8_e4m3fn (with value_scale)")
     N, H, W, G, C = input.shape
     (kh, kw), (sh, sw), (ph, pw), (dh, dw) = _pair(kernel), _pair(stride), _pair(pad), _pair(dilation)
     prob = _lib.DcnProblem(N, H, W, G, C, kh, kw, sh, sw, ph, pw, dh, dw, _DTYPES[input.dtype], flags)
-    if input.dtype == torch.int8:
+    if input.dtype in _SCALED:
         if value_scale is None:
-            raise ValueError("int8 input needs value_scale [N, G] (see quantize_value_s8)")
+            raise ValueError("one-byte input needs value_scale [N, G] "
+                             "(see quantize_value_s8, quantize_value_e4m3)")
         _need(value_scale, "value_scale", torch.float32, (N, G), input.device)
         prob.value_scale = _ptr(value_scale)
     ho, wo = ctypes.c_int64(0), ctypes.c_int64(0)

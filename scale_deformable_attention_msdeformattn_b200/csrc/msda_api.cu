@@ -42,7 +42,9 @@ bool is_supported_head_dim(int d)
     return d == 8 || d == 16 || d == 32 || d == 64 || d == 128 || d == 256;
 }
 
-size_t elem_bytes(int32_t dtype) { return dtype == MSDA_BF16 ? 2 : (dtype == MSDA_S8 ? 1 : 4); }
+bool scaled_dtype(int32_t dtype) { return dtype == MSDA_S8 || dtype == MSDA_E4M3; }
+
+size_t elem_bytes(int32_t dtype) { return dtype == MSDA_BF16 ? 2 : (scaled_dtype(dtype) ? 1 : 4); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
@@ -65,9 +67,9 @@ msda_status check_problem(const msda_problem *p)
     if (p->batch < 0 || p->num_queries < 0 || p->num_keys < 1 || p->num_heads < 1 ||
         p->num_levels < 1 || p->num_points < 1 || p->head_dim < 1)
         return MSDA_ERR_INVALID_ARG;
-    if (p->value_dtype != MSDA_F32 && p->value_dtype != MSDA_BF16 && p->value_dtype != MSDA_S8)
+    if (p->value_dtype != MSDA_F32 && p->value_dtype != MSDA_BF16 && !scaled_dtype(p->value_dtype))
         return MSDA_ERR_INVALID_ARG;
-    if (p->value_dtype == MSDA_S8 &&
+    if (scaled_dtype(p->value_dtype) &&
         (!p->value_scale || (reinterpret_cast<uintptr_t>(p->value_scale) & 3u)))
         return MSDA_ERR_INVALID_ARG;
     if (p->flags & ~(uint32_t)(MSDA_GRAD_VALUE_BF16 | MSDA_ACCUMULATE_GRADS | MSDA_STAGE_INPUTS |
@@ -404,10 +406,15 @@ msda_status launch_forward(const msda_problem *p, KernelArgs &a, cudaStream_t s)
             MSDA_FWD_CASE_BF16(64) MSDA_FWD_CASE_BF16(128) MSDA_FWD_CASE_BF16(256)
         }
 #undef MSDA_FWD_CASE_BF16
-    } else {
+    } else if (p->value_dtype == MSDA_S8) {
         switch (p->head_dim) {
             MSDA_FWD_CASE(msda::S8, 8) MSDA_FWD_CASE(msda::S8, 16) MSDA_FWD_CASE(msda::S8, 32)
             MSDA_FWD_CASE(msda::S8, 64) MSDA_FWD_CASE(msda::S8, 128) MSDA_FWD_CASE(msda::S8, 256)
+        }
+    } else {
+        switch (p->head_dim) {
+            MSDA_FWD_CASE(msda::E4M3, 8) MSDA_FWD_CASE(msda::E4M3, 16) MSDA_FWD_CASE(msda::E4M3, 32)
+            MSDA_FWD_CASE(msda::E4M3, 64) MSDA_FWD_CASE(msda::E4M3, 128) MSDA_FWD_CASE(msda::E4M3, 256)
         }
     }
 #undef MSDA_FWD_CASE
@@ -455,10 +462,15 @@ msda_status launch_backward(const msda_problem *p, KernelArgs &a, cudaStream_t s
             MSDA_BWD_CASE(__nv_bfloat16, 32) MSDA_BWD_CASE(__nv_bfloat16, 64)
             MSDA_BWD_CASE(__nv_bfloat16, 128) MSDA_BWD_CASE(__nv_bfloat16, 256)
         }
-    } else {
+    } else if (p->value_dtype == MSDA_S8) {
         switch (p->head_dim) {
             MSDA_BWD_CASE(msda::S8, 8) MSDA_BWD_CASE(msda::S8, 16) MSDA_BWD_CASE(msda::S8, 32)
             MSDA_BWD_CASE(msda::S8, 64) MSDA_BWD_CASE(msda::S8, 128) MSDA_BWD_CASE(msda::S8, 256)
+        }
+    } else {
+        switch (p->head_dim) {
+            MSDA_BWD_CASE(msda::E4M3, 8) MSDA_BWD_CASE(msda::E4M3, 16) MSDA_BWD_CASE(msda::E4M3, 32)
+            MSDA_BWD_CASE(msda::E4M3, 64) MSDA_BWD_CASE(msda::E4M3, 128) MSDA_BWD_CASE(msda::E4M3, 256)
         }
     }
 #undef MSDA_BWD_CASE
@@ -481,7 +493,7 @@ KernelArgs base_args(const msda_problem *p, const void *value, const int64_t *sh
     a.withhold_copy = (p->flags & MSDA_TEST_WITHHOLD_COPY) ? 1 : 0;
     a.stage = (p->flags & MSDA_STAGE_INPUTS) ? 1 : 0;
     a.order = (p->batch * p->num_queries > 0) ? p->query_order : nullptr;
-    a.scale = p->value_dtype == MSDA_S8 ? p->value_scale : nullptr;
+    a.scale = scaled_dtype(p->value_dtype) ? p->value_scale : nullptr;
     return a;
 }
 
@@ -1028,10 +1040,11 @@ msda_status msda_backward_noalloc(const msda_problem *problem, const void *value
     return launch_to_bf16(acc, grad_value, z.value, s);
 }
 
-msda_status msda_quantize_value_s8(const msda_problem *problem, const void *value, void *value_s8,
-                                   float *value_scale, msda_stream_t stream)
+// Per-(b, m) absmax, scale = amax / qmax, then the codes: the INT8 and FP8
+// storage entry points differ only in qmax and the quantising kernel.
+static msda_status quantize_value(const msda_problem *problem, const void *value, void *codes,
+                                  float *value_scale, bool e4m3, msda_stream_t stream)
 {
-    MSDA_TRACE();
     msda_status st = check_problem(problem);
     if (st != MSDA_OK)
         return st;
@@ -1042,7 +1055,7 @@ msda_status msda_quantize_value_s8(const msda_problem *problem, const void *valu
     const int64_t n = B * S * M * (int64_t)D;
     if (B == 0)
         return MSDA_OK;
-    if (!ptr_ok(value, n) || !vec_ptr_ok(value_s8, n) || !value_scale ||
+    if (!ptr_ok(value, n) || !vec_ptr_ok(codes, n) || !value_scale ||
         (reinterpret_cast<uintptr_t>(value_scale) & 3u) || D % 8 != 0)
         return MSDA_ERR_INVALID_ARG;
     int dev = 0, sms = 0;
@@ -1065,21 +1078,45 @@ msda_status msda_quantize_value_s8(const msda_problem *problem, const void *valu
     int64_t qblocks = (n / 8 + 255) / 256;
     if (qblocks > (int64_t)sms * 8)
         qblocks = (int64_t)sms * 8;
+    const float qmax = e4m3 ? 448.f : 127.f;
+    uint2 *q = static_cast<uint2 *>(codes);
     if (problem->value_dtype == MSDA_F32) {
         const float *v = static_cast<const float *>(value);
         msda::absmax_kernel<float><<<(unsigned)(chunks * bm), 256, 0, s>>>(v, S, M, D, (int)chunks, amax);
-        msda::s8_scale_kernel<<<(unsigned)((bm + 255) / 256), 256, 0, s>>>(value_scale, bm);
-        msda::quantize_s8_kernel<float><<<(unsigned)qblocks, 256, 0, s>>>(
-            v, value_scale, n / 8, S, M, D, static_cast<uint2 *>(value_s8));
+        msda::quant_scale_kernel<<<(unsigned)((bm + 255) / 256), 256, 0, s>>>(value_scale, bm, qmax);
+        if (e4m3)
+            msda::quantize_e4m3_kernel<float><<<(unsigned)qblocks, 256, 0, s>>>(v, value_scale, n / 8, S, M,
+                                                                              D, q);
+        else
+            msda::quantize_s8_kernel<float><<<(unsigned)qblocks, 256, 0, s>>>(v, value_scale, n / 8, S, M, D,
+                                                                            q);
     } else {
         const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(value);
         msda::absmax_kernel<__nv_bfloat16><<<(unsigned)(chunks * bm), 256, 0, s>>>(v, S, M, D, (int)chunks,
                                                                                   amax);
-        msda::s8_scale_kernel<<<(unsigned)((bm + 255) / 256), 256, 0, s>>>(value_scale, bm);
-        msda::quantize_s8_kernel<__nv_bfloat16><<<(unsigned)qblocks, 256, 0, s>>>(
-            v, value_scale, n / 8, S, M, D, static_cast<uint2 *>(value_s8));
+        msda::quant_scale_kernel<<<(unsigned)((bm + 255) / 256), 256, 0, s>>>(value_scale, bm, qmax);
+        if (e4m3)
+            msda::quantize_e4m3_kernel<__nv_bfloat16><<<(unsigned)qblocks, 256, 0, s>>>(
+                v, value_scale, n / 8, S, M, D, q);
+        else
+            msda::quantize_s8_kernel<__nv_bfloat16><<<(unsigned)qblocks, 256, 0, s>>>(
+                v, value_scale, n / 8, S, M, D, q);
     }
     return cudaGetLastError() == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
+}
+
+msda_status msda_quantize_value_s8(const msda_problem *problem, const void *value, void *value_s8,
+                                   float *value_scale, msda_stream_t stream)
+{
+    MSDA_TRACE();
+    return quantize_value(problem, value, value_s8, value_scale, false, stream);
+}
+
+msda_status msda_quantize_value_e4m3(const msda_problem *problem, const void *value, void *value_e4m3,
+                                     float *value_scale, msda_stream_t stream)
+{
+    MSDA_TRACE();
+    return quantize_value(problem, value, value_e4m3, value_scale, true, stream);
 }
 
 msda_status msda_sort_queries(const msda_problem *problem, const float *points, int32_t *query_order,

@@ -100,12 +100,14 @@ __global__ void __launch_bounds__(256) absmax_kernel(const T *v, int64_t S, int 
     }
 }
 
-__global__ void s8_scale_kernel(float *scale, int64_t n)
+// scale = amax / qmax in place (1 when amax = 0): qmax 127 for INT8, 448 for
+// FP8 E4M3.
+__global__ void quant_scale_kernel(float *scale, int64_t n, float qmax)
 {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) {
         const float amax = scale[i];
-        scale[i] = amax > 0.f ? __fdiv_rn(amax, 127.f) : 1.f;
+        scale[i] = amax > 0.f ? __fdiv_rn(amax, qmax) : 1.f;
     }
 }
 
@@ -127,6 +129,31 @@ __global__ void quantize_s8_kernel(const T *v, const float *scale, int64_t n8, i
             int r = __float2int_rn(__fdiv_rn(f[e], sc));  // half to even
             r = r > 127 ? 127 : (r < -127 ? -127 : r);
             w[e >> 2] |= ((uint32_t)r & 0xffu) << (8 * (e & 3));
+        }
+        q[i] = make_uint2(w[0], w[1]);
+    }
+}
+
+// FP8 storage: the E4M3 code nearest to value / scale (the division in
+// float32, round to nearest even, magnitudes above 448 clipped to 448, the
+// sign kept on zero), eight channels per thread step.
+template <typename T>
+__global__ void quantize_e4m3_kernel(const T *v, const float *scale, int64_t n8, int64_t S, int M, int D,
+                                     uint2 *q)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
+        const int64_t row = i * 8 / D;  // (b * S + s) * M + m
+        const int64_t m = row % M, b = row / ((int64_t)S * M);
+        const float sc = __ldg(scale + b * M + m);
+        float f[8];
+        load8(v + i * 8, f);
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(
+                make_float2(__fdiv_rn(f[e], sc), __fdiv_rn(f[e + 1], sc)), __NV_SATFINITE, __NV_E4M3);
+            w[e >> 2] |= (uint32_t)c << (8 * (e & 3));
         }
         q[i] = make_uint2(w[0], w[1]);
     }

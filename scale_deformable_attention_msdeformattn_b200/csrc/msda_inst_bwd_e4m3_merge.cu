@@ -1,0 +1,6 @@
+// msda_inst_bwd_e4m3_merge.cu -- explicit instantiations of the operator kernels: backward, FP8 (E4M3) value, merged reductions.
+#include "msda_instances.cuh"
+
+namespace msda {
+MSDA_BWD_INSTANCES(, E4M3, true)
+}  // namespace msda

@@ -50,4 +50,6 @@
     MSDA_FWD_INSTANCES(PFX, S8, false) MSDA_FWD_SPLIT_INSTANCES(PFX)                             \
     MSDA_BWD_INSTANCES(PFX, float, true) MSDA_BWD_INSTANCES(PFX, float, false)                   \
     MSDA_BWD_INSTANCES(PFX, __nv_bfloat16, true) MSDA_BWD_INSTANCES(PFX, __nv_bfloat16, false)   \
-    MSDA_BWD_INSTANCES(PFX, S8, true) MSDA_BWD_INSTANCES(PFX, S8, false)
+    MSDA_BWD_INSTANCES(PFX, S8, true) MSDA_BWD_INSTANCES(PFX, S8, false)                         \
+    MSDA_FWD_INSTANCES(PFX, E4M3, false)                                                         \
+    MSDA_BWD_INSTANCES(PFX, E4M3, true) MSDA_BWD_INSTANCES(PFX, E4M3, false)

@@ -35,6 +35,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include <type_traits>
@@ -262,6 +263,7 @@ __device__ __forceinline__ void st_vec(U8 *p, const U8 &v)
 template <typename T> struct Elem;
 template <> struct Elem<float> {
     static constexpr int kBytes = 4;
+    static constexpr bool kScaled = false;  // stored codes times a (batch, head) scale
     template <int NW> __device__ __forceinline__ static void widen(const uint32_t *u, float *f)
     {
 #pragma unroll
@@ -277,6 +279,7 @@ template <> struct Elem<float> {
 };
 template <> struct Elem<__nv_bfloat16> {
     static constexpr int kBytes = 2;
+    static constexpr bool kScaled = false;
     // bf16 -> f32 is exact: the bf16 bits are the top half of the float.
     template <int NW> __device__ __forceinline__ static void widen(const uint32_t *u, float *f)
     {
@@ -303,6 +306,7 @@ struct S8 {
 };
 template <> struct Elem<S8> {
     static constexpr int kBytes = 1;
+    static constexpr bool kScaled = true;
     // Exact: byte b (offset to b + 128 by the xor) is placed in the low
     // mantissa bits of the float 2^23, which is then subtracted with the
     // offset.
@@ -318,10 +322,38 @@ template <> struct Elem<S8> {
     }
 };
 
+// FP8 value storage: an OCP E4M3 code per channel (sign, 4 exponent bits with
+// bias 7, 3 mantissa bits), dequantized by the (batch, head) scale of
+// KernelArgs::scale.  Never written by the operator kernels.
+struct E4M3 {
+    uint8_t bits;
+};
+template <> struct Elem<E4M3> {
+    static constexpr int kBytes = 1;
+    static constexpr bool kScaled = true;
+    // Exact: every E4M3 value is a half, and every half a float.  Byte k of a
+    // word is element k (the low byte of each 16-bit pair is the pair's .x).
+    template <int NW> __device__ __forceinline__ static void widen(const uint32_t *u, float *f)
+    {
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+                    (__nv_fp8x2_storage_t)((u[i] >> (16 * h)) & 0xffffu), __NV_E4M3);
+                const float2 v = __half22float2(__half2(r));
+                f[4 * i + 2 * h] = v.x;
+                f[4 * i + 2 * h + 1] = v.y;
+            }
+        }
+    }
+};
+
 // Element type of output and grad_output rows: the value type, except bf16
-// rows for INT8 value.
+// rows for one-byte (INT8, FP8) value.
 template <typename T> struct RowOf { using type = T; };
 template <> struct RowOf<S8> { using type = __nv_bfloat16; };
+template <> struct RowOf<E4M3> { using type = __nv_bfloat16; };
 
 // Lane layout of one row of D channels with VB-byte lane vectors.
 template <typename T, int D, int VB> struct Layout {
@@ -352,6 +384,7 @@ template <typename T, int D, int VB> struct Layout {
 // type.
 template <typename T> struct BwdVB { static constexpr int kVB = MSDA_BWD_VB; };
 template <> struct BwdVB<S8> { static constexpr int kVB = 8; };
+template <> struct BwdVB<E4M3> { static constexpr int kVB = 8; };
 template <typename T> struct BwdMinCtas { static constexpr int kN = MSDA_BWD_MIN_CTAS; };
 template <> struct BwdMinCtas<float> { static constexpr int kN = MSDA_BWD_MIN_CTAS_F32; };
 
@@ -1176,6 +1209,7 @@ template <bool SHORT> struct FwdTune<S8, SHORT> {
                          kMinCtas = MSDA_FWD_MIN_CTAS_S8;
     static constexpr bool kStage = false;
 };
+template <bool SHORT> struct FwdTune<E4M3, SHORT> : FwdTune<S8, SHORT> {};
 
 // GEN = false: the plain attention kernel (natural query order, no DCN grid),
 // with those branches removed at compile time; GEN = true honours
@@ -1346,9 +1380,9 @@ forward_kernel(const KernelArgs a_in)
                     acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], i);
         }
         if (active && ph == 0) {
-            if constexpr (std::is_same<T, S8>::value) {
+            if constexpr (Elem<T>::kScaled) {
                 // dequantize once per row, store bf16 (EPV = 8 channels, 16 bytes)
-                static_assert(EPV == 8, "INT8 lanes hold 8 channels");
+                static_assert(EPV == 8, "one-byte lanes hold 8 channels");
                 const float sc = __ldg(a.scale + b * a.M + m);
 #pragma unroll
                 for (int e = 0; e < E; ++e)
@@ -1671,8 +1705,8 @@ backward_kernel(const KernelArgs a_in)
         }
         const int64_t base = row * P;
         float dot = 0.f, ref_gx = 0.f, ref_gy = 0.f;  // fused: per-owner partial sums
-        float vsc = 1.f;  // INT8 value: the dot products are in quantized units
-        if constexpr (std::is_same<T, S8>::value)
+        float vsc = 1.f;  // one-byte value: the dot products are in code units
+        if constexpr (Elem<T>::kScaled)
             vsc = active ? __ldg(a.scale + b * a.M + m) : 0.f;
         for (int c0 = 0; c0 < Pp; c0 += C) {
             float part[C][3];
@@ -1704,7 +1738,7 @@ backward_kernel(const KernelArgs a_in)
                 const unsigned inm = __float_as_uint(r.w);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    d[c] = (inm & (1u << c)) ? (std::is_same<T, S8>::value ? d[c] * vsc : d[c])
+                    d[c] = (inm & (1u << c)) ? (Elem<T>::kScaled ? d[c] * vsc : d[c])
                                              : 0.f;  // corners outside the map read 0
                 const float fx = r.x, fy = r.y, A = r.z, ex = 1.f - fx, ey = 1.f - fy;
                 const float w[4] = {ex * ey, fx * ey, ex * fy, fx * fy};

@@ -108,7 +108,7 @@ class Workload:
     M: int
     D: int
     K: int
-    dtype: str               # value / output dtype: "f32", "bf16", or "s8" (int8 value
+    dtype: str               # value / output dtype: "f32", "bf16", "s8" or "e4m3" (one-byte value
                              # quantised from the bf16 draw; output, grad_output bf16)
     ref: str                 # "pixel_centre" | "uniform" | "uniform_inner"
     offset_sigma: float      # pixels of the sampled level
@@ -157,6 +157,11 @@ WORKLOADS: Dict[str, Workload] = {
                  None, 8, 32, 4, "s8", "pixel_centre", 2.0, 1.0),
         Workload("stress_1080p_k8_s8", 4, 2, ((135, 240), (68, 120), (34, 60), (17, 30)),
                  None, 8, 32, 8, "s8", "pixel_centre", 8.0, 2.0),
+        # FP8 (E4M3) value storage on the same draws
+        Workload("encoder_1024_e4m3", 3, 4, ((128, 128), (64, 64), (32, 32), (16, 16)),
+                 None, 8, 32, 4, "e4m3", "pixel_centre", 2.0, 1.0),
+        Workload("stress_1080p_k8_e4m3", 4, 2, ((135, 240), (68, 120), (34, 60), (17, 30)),
+                 None, 8, 32, 8, "e4m3", "pixel_centre", 8.0, 2.0),
     ]
 }
 
@@ -180,8 +185,8 @@ class Inputs:
     """All arrays are host numpy arrays in the operator's row-major layouts.
 
     value_bits is the stored value tensor: float32 array for "f32", uint16
-    bfloat16 bit patterns for "bf16" and for "s8" (the source that is then
-    quantised to int8).  Everything else is float32.
+    bfloat16 bit patterns for "bf16" and for "s8" / "e4m3" (the source that is
+    then quantised to one byte).  Everything else is float32.
     """
     workload: Workload
     value: np.ndarray            # [B, S, M, D] float32 or uint16 (bf16 bits)
@@ -208,7 +213,7 @@ def _widen(a: np.ndarray) -> np.ndarray:
 
 
 def _store(x: np.ndarray, dtype: str) -> np.ndarray:
-    if dtype in ("bf16", "s8"):  # s8: the bf16 source of the quantised value
+    if dtype in ("bf16", "s8", "e4m3"):  # s8, e4m3: the bf16 source of the quantised value
         return to_bf16_bits(x)
     return x.astype(np.float32)
 

@@ -28,7 +28,7 @@ ELEM_FLOOR = 1e-3
 
 
 def value_tensor(arr: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
-    if dtype in ("bf16", "s8"):  # s8 workloads carry the bf16 source
+    if dtype in ("bf16", "s8", "e4m3"):  # one-byte workloads carry the bf16 source
         return torch.from_numpy(arr.view(np.int16)).to(device).view(torch.bfloat16)
     return torch.from_numpy(arr).to(device)
 
