@@ -48,18 +48,16 @@ L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 # hash of the CUDA sources it was taken from and is reported only while those
 # sources are unchanged.  Filled from the summaries under profiles/.
 NCU_TRAFFIC = {
-    # profiles/detr_encoder_f32_fused_kernels.md: mean of two launches, DRAM read + write
-    ("fused_backward", "detr_encoder_f32"): {"bytes": 127103488, "csrc": "82b094a66de9ae01"},
-    ("fused_forward", "detr_encoder_f32"): {"bytes": 59862656, "csrc": "82b094a66de9ae01"},
-    # profiles/detr_decoder_bf16_kernels.md: DRAM read + write of one launch
-    ("fused_backward", "detr_decoder_bf16"): {"bytes": 138262272, "csrc": "82b094a66de9ae01"},
-    ("fused_forward", "detr_decoder_bf16"): {"bytes": 51268096, "csrc": "82b094a66de9ae01"},
-    # profiles/stress_1080p_k8_bf16_fused_kernels.md: DRAM read + write of one launch
-    ("fused_backward", "stress_1080p_k8_bf16"): {"bytes": 925939712, "csrc": "82b094a66de9ae01"},
-    ("fused_forward", "stress_1080p_k8_bf16"): {"bytes": 381244928, "csrc": "82b094a66de9ae01"},
-    # profiles/dcnv3_stage1_f32_kernels.md: DRAM read + write of one launch
-    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 143730688, "csrc": "82b094a66de9ae01"},
-    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 73360896, "csrc": "82b094a66de9ae01"},
+    # DRAM read + write per launch (the mean of the launches captured), from
+    # the counter captures listed in the profiles/ summaries
+    ("fused_backward", "detr_encoder_f32"): {"bytes": 126671488, "csrc": "1a0b45d13ae30d65"},
+    ("fused_forward", "detr_encoder_f32"): {"bytes": 59487616, "csrc": "1a0b45d13ae30d65"},
+    ("fused_backward", "detr_decoder_bf16"): {"bytes": 132766720, "csrc": "1a0b45d13ae30d65"},
+    ("fused_forward", "detr_decoder_bf16"): {"bytes": 51133440, "csrc": "1a0b45d13ae30d65"},
+    ("fused_backward", "stress_1080p_k8_bf16"): {"bytes": 924305664, "csrc": "1a0b45d13ae30d65"},
+    ("fused_forward", "stress_1080p_k8_bf16"): {"bytes": 384668160, "csrc": "1a0b45d13ae30d65"},
+    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 141031936, "csrc": "1a0b45d13ae30d65"},
+    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 72917504, "csrc": "1a0b45d13ae30d65"},
 }
 
 
@@ -499,6 +497,18 @@ def run_ours(args):
                 fa["frac_touched"] = round((nbytes["fused_forward"] - untouched)
                                            / (fa["fwd_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
         result["config"]["input_stats"] = stats
+        if dom == "fused_backward":
+            # the backward's own ceiling: its grad_value reductions (one float32
+            # row of D channels per in-map corner) go through the L2's
+            # reduction units, whose rate a reduction-only probe kernel
+            # measured on B200: 6.1 TB/s of payload (red.global.add.v4.f32 at
+            # random 128-byte rows of an L2-resident float32 array)
+            red_bytes = stats["in_map_corners_per_sample"] * w.samples * w.D * 4
+            ach = red_bytes / (bwd_ms * 1e-3) / 1e9
+            result["roofline"]["l2_reduction"] = {
+                "bytes_per_launch": int(red_bytes), "achieved": round(ach, 1), "ceiling": 6100.0,
+                "unit": "GB/s", "frac": round(ach / 6100.0, 4),
+                "ceiling_source": "reduction-only probe kernel on B200 (not part of this bench)"}
         if not args.no_e2e:
             result["e2e"] = _time_e2e(_pinned(x), step, make_outputs, flush, min(args.steps, 50),
                                       w.samples, dev, 7)
@@ -677,9 +687,18 @@ def _input_stats(w: wl.Workload, x: wl.Inputs, max_queries: int = 4096) -> dict:
     inside = (px > -1) & (px < size)
     full_out = ~(inside[..., 0] & inside[..., 1])
     any_out = ((lo < 0) | (lo + 1 > size - 1)).any(axis=-1)
+    # corners the backward reduces into grad_value: the in-map corners of the
+    # samples that are taken
+    in_map = np.zeros(full_out.shape)
+    for dy in (0, 1):
+        for dx in (0, 1):
+            cx, cy = lo[..., 0] + dx, lo[..., 1] + dy
+            in_map += (cx >= 0) & (cx < size[..., 0]) & (cy >= 0) & (cy < size[..., 1])
+    in_map[full_out] = 0
     out = {"samples_counted": int(full_out.size),
            "fully_outside": round(float(full_out.mean()), 4),
-           "any_corner_outside": round(float(any_out.mean()), 4)}
+           "any_corner_outside": round(float(any_out.mean()), 4),
+           "in_map_corners_per_sample": round(float(in_map.mean()), 4)}
     if w.samples <= (4 << 20):
         loc = (x.reference_points.astype(np.float64)[:, :, None, None, None, :]
                + x.sampling_offsets.astype(np.float64) / wh[None, None, None, :, None, :])
@@ -767,7 +786,46 @@ def _time_e2e(hin, step, make_outputs, flush, n, samples, dev, nev):
     return {"value": round(samples / (ms * 1e-3) / 1e9, 4), "unit": UNIT,
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": n, "copies": "pinned host buffers; input and result copies on their own streams, "
-                                  "overlapping the neighbouring steps' kernels"}
+                                  "overlapping the neighbouring steps' kernels",
+            "link_gbs": _link_bandwidth(hin, hout, sets[0][0], sets[0][1], s_in, s_out)}
+
+
+def _link_bandwidth(hin, hout, din, dout, s_in, s_out, reps: int = 5) -> dict:
+    """The host link alone, with the step's own buffers: GB/s of the input
+    copies (host to device), of the result copies (device to host), and of
+    both at once on their two streams (each direction's bytes over the
+    common time), the medians of `reps` rounds: the ceiling the e2e leg's
+    copies can reach."""
+    import torch
+
+    def timed(h2d: bool, d2h: bool) -> float:
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record()
+            s_in.wait_event(a)
+            s_out.wait_event(a)
+            if h2d:
+                with torch.cuda.stream(s_in):
+                    for k in hin:
+                        din[k].copy_(hin[k], non_blocking=True)
+            if d2h:
+                with torch.cuda.stream(s_out):
+                    for k in hout:
+                        hout[k].copy_(dout[k], non_blocking=True)
+            torch.cuda.current_stream().wait_stream(s_in)
+            torch.cuda.current_stream().wait_stream(s_out)
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e-3)
+        return statistics.median(ts)
+
+    nin = sum(v.numel() * v.element_size() for v in hin.values())
+    nout = sum(v.numel() * v.element_size() for v in hout.values())
+    t_in, t_out, t_both = timed(True, False), timed(False, True), timed(True, True)
+    return {"h2d": round(nin / t_in / 1e9, 1), "d2h": round(nout / t_out / 1e9, 1),
+            "both_h2d": round(nin / t_both / 1e9, 1), "both_d2h": round(nout / t_both / 1e9, 1)}
 
 
 # ------------------------------------------------------- the oracle legs --
