@@ -87,3 +87,33 @@ def test_checked_build_int8_and_dcn(checked_lib):
     assert_close(gx, rgx, 1e-5, "checked int8 dcn grad_input")
     assert_close(goff, rgoff, 1e-5, "checked int8 dcn grad_offset")
     assert_close(gm, rgm, 1e-5, "checked int8 dcn grad_mask")
+
+
+def test_checked_build_fp8_decoder(checked_lib):
+    """FP8 value on the decoder's shape (rows split over lane groups in the
+    forward) through the four operator calls."""
+    w = wl.custom("chk_fp8_decoder", 2, [(100, 167), (50, 84), (25, 42), (13, 21)], 300, 8, 32, 4,
+                  "e4m3", "uniform_inner", 4.0, 1.0, index=901)
+    x = wl.generate(w)
+    t = upload(x)
+    q, s = msda.quantize_value_e4m3(t["value"])
+    geo = (t["spatial_shapes"], t["level_start_index"])
+    out = msda.forward(q, *geo, t["sampling_locations"], t["attention_weights"], value_scale=s)
+    gv, gl, ga = msda.backward(q, *geo, t["sampling_locations"], t["attention_weights"],
+                               t["grad_output"], value_scale=s)
+    fout = msda.fused_forward(q, *geo, t["reference_points"], t["sampling_offsets"],
+                              t["attention_logits"], value_scale=s)
+    fgv, fgref, fgoff, fglog = msda.fused_backward(q, *geo, t["reference_points"], t["sampling_offsets"],
+                                                   t["attention_logits"], t["grad_output"], value_scale=s)
+    assert msda.device_status() == 0
+    rq, rs = oracle.quantize_value_e4m3(x.value)
+    x.value = oracle.dequantize_value_e4m3(rq, rs)  # the oracle samples decode(code) * scale
+    r = oracle_nonfused(x)
+    for g, ref, what, tol in zip((out, gv, gl, ga), r, ("out", "grad_value", "grad_loc", "grad_attn"),
+                                 (1e-2, 1e-5, 1e-5, 1e-5)):
+        assert_close(g, ref, tol, f"checked fp8 decoder {what}")
+    rf = oracle_fused(x)
+    for g, ref, what, tol in zip((fout, fgv, fgref, fgoff, fglog), (rf[0],) + rf[2:],
+                                 ("out", "grad_value", "grad_ref", "grad_off", "grad_logits"),
+                                 (1e-2, 1e-5, 1e-5, 1e-5, 1e-5)):
+        assert_close(g, ref, tol, f"checked fp8 decoder fused {what}")
