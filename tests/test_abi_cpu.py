@@ -181,3 +181,63 @@ def test_dcn_checks(lib):
     assert n.value == 2 * 56 * 56 * 4 * 16 * 4
     assert lib.msda_dcn_backward(ctypes.byref(pb), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
                                  16, None) == _lib.MSDA_ERR_INVALID_ARG
+
+
+def test_fp8_checks(lib):
+    """MSDA_E4M3 needs a 4-byte aligned value_scale; the FP8 quantiser takes a
+    float32 / bf16 source, 32-byte aligned codes and a scale array."""
+    p = _prob(value_dtype=_lib.MSDA_E4M3)
+    assert _fwd(lib, p) == _lib.MSDA_ERR_INVALID_ARG
+    p.value_scale = ctypes.c_void_p(0x100002)
+    assert _fwd(lib, p) == _lib.MSDA_ERR_INVALID_ARG
+    src = _prob(value_dtype=_lib.MSDA_E4M3)
+    src.value_scale = FAKE
+    assert lib.msda_quantize_value_e4m3(ctypes.byref(src), FAKE, FAKE, FAKE, None) == \
+        _lib.MSDA_ERR_INVALID_ARG
+    f32 = _prob()
+    assert lib.msda_quantize_value_e4m3(ctypes.byref(f32), FAKE, MISALIGNED, FAKE, None) == \
+        _lib.MSDA_ERR_INVALID_ARG
+    assert lib.msda_quantize_value_e4m3(ctypes.byref(f32), FAKE, FAKE, None, None) == \
+        _lib.MSDA_ERR_INVALID_ARG
+    empty = _prob(batch=0)
+    assert lib.msda_quantize_value_e4m3(ctypes.byref(empty), None, None, None, None) == _lib.MSDA_OK
+
+
+def test_dense_layer_checks(lib):
+    """msda_linear, msda_query_head and msda_query_head_backward reject bad
+    sizes and pointers before anything is enqueued; empty inputs are a no-op."""
+    F32, BF16 = _lib.MSDA_F32, _lib.MSDA_BF16
+    bad, unsupported, ok = _lib.MSDA_ERR_INVALID_ARG, _lib.MSDA_ERR_UNSUPPORTED, _lib.MSDA_OK
+
+    def linear(rows=100, k=16, n=16, x=FAKE, w=FAKE, b=None, out=FAKE, dt=F32):
+        return lib.msda_linear(rows, k, n, x, w, b, out, dt, None)
+
+    assert linear(k=12) == bad                        # in_features a multiple of 8
+    assert linear(k=0) == bad
+    assert linear(n=20) == bad                        # out_features a multiple of 8
+    assert linear(dt=_lib.MSDA_S8) == bad             # float32 or bf16 output only
+    assert linear(rows=-1) == bad
+    assert linear(rows=0, x=None, w=None, out=None) == ok
+    assert linear(x=MISALIGNED) == bad
+    assert linear(out=None, dt=BF16) == bad
+    assert linear(b=ctypes.c_void_p(0x100002)) == bad  # bias 4-byte aligned
+
+    def head(p, k=256, q=FAKE, ref=FAKE, loc=FAKE, attn=FAKE):
+        return lib.msda_query_head(ctypes.byref(p), k, q, FAKE, None, ref, FAKE, loc, attn, None)
+
+    def head_bwd(p, gh=FAKE):
+        return lib.msda_query_head_backward(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, gh, None, None)
+
+    good = _prob(num_heads=8, num_levels=4, num_points=4)          # L*K = 16, P = 128
+    assert head(good, k=12) == bad
+    assert head(good, q=MISALIGNED) == bad
+    assert head(good, loc=None) == bad
+    assert head_bwd(good, gh=MISALIGNED) == bad
+    # L*K a power of two of at most 32, M*L*K a multiple of 32
+    for p in (_prob(num_heads=32, num_levels=3, num_points=1), _prob(num_heads=1, num_levels=2, num_points=2),
+              _prob(num_heads=1, num_levels=4, num_points=16)):
+        assert head(p) == unsupported
+        assert head_bwd(p) == unsupported
+    empty = _prob(batch=0, num_heads=8, num_levels=4, num_points=4)
+    assert head(empty, q=None, ref=None, loc=None, attn=None) == ok
+    assert head_bwd(empty, gh=None) == ok
