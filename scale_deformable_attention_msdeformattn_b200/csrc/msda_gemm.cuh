@@ -24,8 +24,9 @@
 //                      its "empty" barrier and, after a tile's last K block,
 //                      commits the tile's accumulator buffer to the epilogue;
 //   warps 2..9         epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31
-//                      (its 32 output rows; two warps per lane quarter, each
-//                      taking every other column chunk) 32 columns at a
+//                      (its 32 output rows; kEpiWarps / 4 warps per lane
+//                      quarter, two by default, each taking every
+//                      kEpiParts-th column chunk) 32 columns at a
 //                      time, applies the epilogue, writes 32-row x 128-byte
 //                      boxes into shared memory (128-byte swizzle, one box
 //                      per warp by default) and stores them with TMA; then it
@@ -36,7 +37,8 @@
 // of two frees 32 KB for two more stages (21.8 -> 19.2 us), the bias from
 // shared memory instead of 32 shuffles per 32 columns takes a third off each
 // box (-> 19.0 us), and one N = 256 MMA instead of two of N = 128 per K step
-// 23.1 -> 21.8 us.
+// 23.1 -> 21.8 us.  Twelve epilogue warps instead of eight: no change
+// (19.3 us; query head 42.7 against 43.5 us).
 // With NSUB <= 2 there are two accumulator buffers (2 x BN <= 512 columns),
 // so a tile's epilogue overlaps the next tile's loads and MMAs.
 // No TMA multicast and no clusters: the tensor maps cover this GPU's memory
@@ -59,7 +61,12 @@ namespace msda_gemm {
 constexpr int kBM = 128;           // rows per tile (TMEM lanes)
 constexpr int kBK = 64;            // K per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kSubN = 128;         // columns per MMA (and per TMA box of w)
-constexpr int kEpiWarps = 8;
+#ifndef MSDA_GEMM_EPI_WARPS
+#define MSDA_GEMM_EPI_WARPS 8                       // epilogue warps (a multiple of 4)
+#endif
+constexpr int kEpiWarps = MSDA_GEMM_EPI_WARPS;
+constexpr int kEpiParts = kEpiWarps / 4;          // epilogue warps per TMEM lane quarter
+static_assert(kEpiWarps % 4 == 0, "epilogue warps come in lane quarters");
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kATileBytes = kBM * kBK * 2;      // 16 KB
 constexpr int kBSubBytes = kSubN * kBK * 2;     // 16 KB
@@ -491,20 +498,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;                     // TMEM lane quarter
         const int e = warp - 2;                     // epilogue warp index
-        const int half = e >> 2;                    // which column chunks of the quarter
+        const int part = e >> 2;                    // which column chunks of the quarter
         uint8_t *boxes = epi_smem + e * kEpiBoxes * kBoxBytes;
         int nbox = 0, local = 0;
         const int step = (p.epi == kEpiStore && p.out_bf16) ? 64 : 32;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
             const int buf = local % C::kAcc, use = local / C::kAcc;
             const int m0 = (t / p.n_tiles) * kBM, n0 = (t % p.n_tiles) * C::kBN;
-            // this warp's bias values of the tile (chunks c0 = half*step +
-            // 2*step*k, 32 columns each), loaded before the accumulator wait
-            constexpr int kNb = WRES ? 1 : C::kBN / 32 / 2;
+            // this warp's bias values of the tile (chunks c0 = part*step +
+            // kEpiParts*step*k, 32 columns each), loaded before the
+            // accumulator wait
+            constexpr int kNb = WRES ? 1 : (C::kBN / 32 + kEpiParts - 1) / kEpiParts;
             float bl[kNb];
 #pragma unroll
             for (int k = 0; k < kNb; ++k) {
-                const int c = half * step + (k / (step / 32)) * 2 * step + (k % (step / 32)) * 32;
+                const int c = part * step + (k / (step / 32)) * kEpiParts * step + (k % (step / 32)) * 32;
                 bl[k] = (!WRES && c < C::kBN) ? bias_lane(p.bias, n0 + c, p.N, lane) : 0.f;
             }
             const bool ready = __all_sync(0xffffffffu, mbar_wait(acc_full + buf, use & 1) &&
@@ -526,7 +534,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                 ry = __ldg(p.ref + 2 * (int64_t)r + 1);
             }
 #pragma unroll 1
-            for (int c0 = half * step, kc = 0; c0 < C::kBN && n0 + c0 < p.N; c0 += 2 * step, ++kc) {
+            for (int c0 = part * step, kc = 0; c0 < C::kBN && n0 + c0 < p.N; c0 += kEpiParts * step, ++kc) {
                 float v[32], v2[32];
                 tmem_ld32(tbase + c0, v);
                 if (step == 64)
