@@ -229,10 +229,9 @@ msda_status launch_rows(const void *kernel, int rpw, size_t record_bytes, int pa
     return MSDA_OK;
 }
 
-// Shared-memory budget of one CTA of the merged backward: float32 value runs
-// three CTAs per SM (its register budget), the others two.
-constexpr size_t kMergeSmemBudgetF32 = 72 * 1024;
-constexpr size_t kMergeSmemBudget = 108 * 1024;
+// Shared-memory budget of one CTA of the merged backward: every value type
+// runs three CTAs per SM (the backward's register budget).
+constexpr size_t kMergeSmemBudget = 72 * 1024;
 
 // Launches the merged backward (tiles of one head of merge_qb consecutive
 // queries of one batch; msda_kernels.cuh "merged reductions") as a
@@ -435,8 +434,7 @@ msda_status launch_backward_td(const msda_problem *p, KernelArgs &a, cudaStream_
         const void *k = gen ? (const void *)msda::backward_kernel<T, D, FUSED, true, true>
                             : (const void *)msda::backward_kernel<T, D, FUSED, false, true>;
         bool fits = false;
-        const size_t budget = std::is_same<T, float>::value ? kMergeSmemBudgetF32 : kMergeSmemBudget;
-        msda_status st = launch_merge(k, rpw, rec, pp, D, budget, a, p, s, fits);
+        msda_status st = launch_merge(k, rpw, rec, pp, D, kMergeSmemBudget, a, p, s, fits);
         if (st != MSDA_OK || fits)
             return st;
     }

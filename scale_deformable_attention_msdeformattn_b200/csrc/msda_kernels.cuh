@@ -100,8 +100,11 @@ namespace msda {
 #ifndef MSDA_BWD_MIN_CTAS_F32       // backward CTAs per SM (register budget) by value type
 #define MSDA_BWD_MIN_CTAS_F32 3
 #endif
-#ifndef MSDA_BWD_MIN_CTAS
-#define MSDA_BWD_MIN_CTAS 2
+#ifndef MSDA_BWD_MIN_CTAS_BF16
+#define MSDA_BWD_MIN_CTAS_BF16 3
+#endif
+#ifndef MSDA_BWD_MIN_CTAS            // one-byte (INT8, FP8) value
+#define MSDA_BWD_MIN_CTAS 3
 #endif
 #ifndef MSDA_MERGE_FLUSH_CHAINS      // merged backward: slot lists a lane group walks together
 #define MSDA_MERGE_FLUSH_CHAINS 1
@@ -233,11 +236,13 @@ struct alignas(32) U8 {
 };
 
 template <int VB> struct RawOf;
+template <> struct RawOf<4> { using type = uint32_t; };
 template <> struct RawOf<8> { using type = uint2; };
 template <> struct RawOf<16> { using type = uint4; };
 template <> struct RawOf<32> { using type = U8; };
 
 // Read-only vector load of `value` (L1-cached).
+__device__ __forceinline__ uint32_t ld_vec(const uint32_t *p) { return __ldg(p); }
 __device__ __forceinline__ uint2 ld_vec(const uint2 *p) { return __ldg(p); }
 __device__ __forceinline__ uint4 ld_vec(const uint4 *p) { return __ldg(p); }
 __device__ __forceinline__ U8 ld_vec(const U8 *p)
@@ -366,7 +371,7 @@ template <typename T, int D, int VB> struct Layout {
     static constexpr int kCh = kNvec / kG;                   // vectors per lane
     static constexpr int kRowsPerWarp = 32 / kG;
     static constexpr int kLaneElems = kCh * kEpv;            // channels per lane
-    static_assert(kVB == 8 || kVB == 16 || kVB == 32, "vector size");
+    static_assert(kVB == 4 || kVB == 8 || kVB == 16 || kVB == 32, "vector size");
     static_assert(kNvec >= 1 && kNvec % kG == 0, "unsupported head_dim");
     __device__ __forceinline__ static void widen(const Raw &r, float *f)
     {
@@ -382,11 +387,28 @@ template <typename T, int D, int VB> struct Layout {
 
 // Lane vector width and resident CTAs per SM of the backward for each value
 // type.
+// bf16 backward: 8-byte lanes, so that a lane's float32 gradient channels
+// are one 16-byte vector and the G lanes of a row reduce whole 128-byte
+// lines (16-byte lanes split each D = 32 row into two 64-byte reductions;
+// measured on the fused backward alone, µs: 1024^2 1194 -> 1055, 1080p K=8
+// 2048 -> 1899, decoder 70.8 -> 67.6; with 3 CTAs per SM, which the smaller
+// register need then allows: 985, 1692, 59.5)
+#ifndef MSDA_BWD_VB_BF16
+#define MSDA_BWD_VB_BF16 8
+#endif
 template <typename T> struct BwdVB { static constexpr int kVB = MSDA_BWD_VB; };
-template <> struct BwdVB<S8> { static constexpr int kVB = 8; };
-template <> struct BwdVB<E4M3> { static constexpr int kVB = 8; };
+template <> struct BwdVB<__nv_bfloat16> { static constexpr int kVB = MSDA_BWD_VB_BF16; };
+// One-byte (INT8, FP8) value backward: 4-byte lanes for the same reason as
+// bf16's 8-byte ones (whole-line reductions), at 3 CTAs per SM (fused
+// backward alone, µs: 1024^2 INT8 1196 -> 996, 1080p K=8 FP8 2024 -> 1713).
+#ifndef MSDA_BWD_VB_1B
+#define MSDA_BWD_VB_1B 4
+#endif
+template <> struct BwdVB<S8> { static constexpr int kVB = MSDA_BWD_VB_1B; };
+template <> struct BwdVB<E4M3> { static constexpr int kVB = MSDA_BWD_VB_1B; };
 template <typename T> struct BwdMinCtas { static constexpr int kN = MSDA_BWD_MIN_CTAS; };
 template <> struct BwdMinCtas<float> { static constexpr int kN = MSDA_BWD_MIN_CTAS_F32; };
+template <> struct BwdMinCtas<__nv_bfloat16> { static constexpr int kN = MSDA_BWD_MIN_CTAS_BF16; };
 
 template <int G>
 __device__ __forceinline__ float group_sum(float v)
