@@ -50,14 +50,14 @@ L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 NCU_TRAFFIC = {
     # DRAM read + write per launch (the mean of the launches captured), from
     # the counter captures listed in the profiles/ summaries
-    ("fused_backward", "detr_encoder_f32"): {"bytes": 126671488, "csrc": "6c528b367b52484c"},
-    ("fused_forward", "detr_encoder_f32"): {"bytes": 59487616, "csrc": "6c528b367b52484c"},
-    ("fused_backward", "detr_decoder_bf16"): {"bytes": 132766720, "csrc": "6c528b367b52484c"},
-    ("fused_forward", "detr_decoder_bf16"): {"bytes": 51133440, "csrc": "6c528b367b52484c"},
-    ("fused_backward", "stress_1080p_k8_bf16"): {"bytes": 924305664, "csrc": "6c528b367b52484c"},
-    ("fused_forward", "stress_1080p_k8_bf16"): {"bytes": 384668160, "csrc": "6c528b367b52484c"},
-    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 141031936, "csrc": "6c528b367b52484c"},
-    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 72917504, "csrc": "6c528b367b52484c"},
+    ("fused_backward", "detr_encoder_f32"): {"bytes": 126669824, "csrc": "8f2eaf4fa1f3588a"},
+    ("fused_forward", "detr_encoder_f32"): {"bytes": 59208448, "csrc": "8f2eaf4fa1f3588a"},
+    ("fused_backward", "detr_decoder_bf16"): {"bytes": 135612160, "csrc": "8f2eaf4fa1f3588a"},
+    ("fused_forward", "detr_decoder_bf16"): {"bytes": 51015424, "csrc": "8f2eaf4fa1f3588a"},
+    ("fused_backward", "stress_1080p_k8_bf16"): {"bytes": 913981184, "csrc": "8f2eaf4fa1f3588a"},
+    ("fused_forward", "stress_1080p_k8_bf16"): {"bytes": 384010752, "csrc": "8f2eaf4fa1f3588a"},
+    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 141286400, "csrc": "8f2eaf4fa1f3588a"},
+    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 73070336, "csrc": "8f2eaf4fa1f3588a"},
 }
 
 
