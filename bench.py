@@ -26,6 +26,7 @@ import glob
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -50,29 +51,37 @@ L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 NCU_TRAFFIC = {
     # DRAM read + write per launch (the mean of the launches captured), from
     # the counter captures listed in the profiles/ summaries
-    ("fused_backward", "detr_encoder_f32"): {"bytes": 126669824, "csrc": "8f2eaf4fa1f3588a"},
-    ("fused_forward", "detr_encoder_f32"): {"bytes": 59208448, "csrc": "8f2eaf4fa1f3588a"},
-    ("fused_backward", "detr_decoder_bf16"): {"bytes": 135612160, "csrc": "8f2eaf4fa1f3588a"},
-    ("fused_forward", "detr_decoder_bf16"): {"bytes": 51015424, "csrc": "8f2eaf4fa1f3588a"},
-    ("fused_backward", "stress_1080p_k8_bf16"): {"bytes": 913981184, "csrc": "8f2eaf4fa1f3588a"},
-    ("fused_forward", "stress_1080p_k8_bf16"): {"bytes": 384010752, "csrc": "8f2eaf4fa1f3588a"},
-    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 141286400, "csrc": "8f2eaf4fa1f3588a"},
-    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 73070336, "csrc": "8f2eaf4fa1f3588a"},
+    ("fused_backward", "detr_encoder_f32"): {"bytes": 126669824, "csrc": "76997acc56ab4bc7"},
+    ("fused_forward", "detr_encoder_f32"): {"bytes": 59208448, "csrc": "76997acc56ab4bc7"},
+    ("fused_backward", "detr_decoder_bf16"): {"bytes": 135612160, "csrc": "76997acc56ab4bc7"},
+    ("fused_forward", "detr_decoder_bf16"): {"bytes": 51015424, "csrc": "76997acc56ab4bc7"},
+    ("fused_backward", "stress_1080p_k8_bf16"): {"bytes": 913981184, "csrc": "76997acc56ab4bc7"},
+    ("fused_forward", "stress_1080p_k8_bf16"): {"bytes": 384010752, "csrc": "76997acc56ab4bc7"},
+    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 141286400, "csrc": "76997acc56ab4bc7"},
+    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 73070336, "csrc": "76997acc56ab4bc7"},
 }
 
 
+def _code_only(text: str) -> str:
+    """C++ source without its comments and blank lines (a comment edit keeps
+    the hash)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def csrc_hash() -> str:
-    """Hash of the sources the operator kernels are compiled and launched
-    from (every file of csrc/ except the dense-layer GEMM header, which none
-    of them includes)."""
+    """Hash of the code the operator kernels are compiled and launched from:
+    every file of csrc/ except the dense-layer GEMM header (which none of
+    them includes), comments left out."""
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "scale_deformable_attention_msdeformattn_b200",
                                            "csrc", "*"))):
         if os.path.basename(p) == "msda_gemm.cuh":
             continue
-        with open(p, "rb") as f:
+        with open(p, encoding="utf-8") as f:
             h.update(os.path.basename(p).encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -5,11 +5,12 @@
 //
 // Work decomposition.  A "row" is one (b, q, m) triple; rows are numbered
 // r = (b * Q + q) * M + m.  A group of G lanes owns one row; each lane owns
-// one vector of VB bytes (16 or 32: 4 or 8 float32, 8 or 16 bf16 channels) of
-// the head_dim axis, so a corner of a sample is one fully used G*VB-byte row
+// one vector of VB bytes (4 to 32, by value type and direction) of the
+// head_dim axis, so a corner of a sample is one fully used G*VB-byte row
 // segment of `value` (128 bytes for D = 32 float32).  A warp carries 32 / G
 // rows, a CTA up to 8 warps (fewer when the per-row shared-memory records
-// would not fit).
+// would not fit); rows too few to fill the GPU are split over several lane
+// groups in the forward (SPLIT).
 //
 // Per tile of rows there are two phases:
 //   1. set-up: the group's lanes turn the row's L*K samples into records in
@@ -23,14 +24,18 @@
 //      the group with a reduce-scatter of shuffles (each lane ends up owning
 //      one sample's results), and scatters A * w_c * g into the float32
 //      grad_value with 16-byte vector reductions (red.global.add.v4.f32), laid
-//      out so that every reduction fills whole 32-byte L2 sectors.
+//      out so that a row's lanes reduce whole 128-byte lines (one L2 request
+//      per line: the backward's lanes carry 4 float32 gradient channels).
 //
 // Floor decisions.  The pixel coordinate x = loc_x * W - 0.5 and its floor are
-// taken in float64 with the same operations, in the same order, as the
-// defining formula (fused: loc = ref + off / W first, then loc * W - 0.5), so
-// the corner choice is exactly that of the formula evaluated in double
-// precision; the fractional parts are then rounded to float32 and everything
-// else runs in float32.
+// taken in float64 so that the corner choice is exactly that of the defining
+// formula evaluated in double precision: non-fused fma(loc, W, -0.5) rounds
+// as the formula does (loc * W is exact); fused fma(ref, W, off) - 0.5
+// differs from the formula's chain (loc = ref + off / W, then loc * W - 0.5)
+// by far less than the distance to an integer unless x lies within 1e-9 of
+// one or the magnitudes are large, and there the chain itself is evaluated.
+// The fractional parts are then rounded to float32 and everything else runs
+// in float32.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -85,7 +90,7 @@ namespace msda {
 #ifndef MSDA_FWD_STAGE_BF16
 #define MSDA_FWD_STAGE_BF16 0
 #endif
-#ifndef MSDA_FWD_VB_S8               // INT8 value: bytes per lane vector
+#ifndef MSDA_FWD_VB_S8               // one-byte (INT8, FP8) value: bytes per lane vector
 #define MSDA_FWD_VB_S8 8
 #endif
 #ifndef MSDA_FWD_INFLIGHT_S8          // INT8: one sample in flight, 3 CTAs per SM (measured
@@ -146,7 +151,7 @@ struct KernelArgs {
     int withhold_copy;      // testing: arm the input copies but never issue them
     int stage;              // forward: stage set-up inputs by bulk copies (general kernels)
     const int32_t *order;   // optional processing order of the B*Q queries
-    const float *scale;     // INT8 value: dequantization scale per (batch, head)
+    const float *scale;     // one-byte value: dequantization scale per (batch, head)
     // DCNv3 core (non-fused kernels): levels are the kh kernel rows, points
     // the kw kernel columns, all on the one H x W map; the pixel coordinate
     // of sample (l, k) of output pixel q = (i, j) is the convolution grid
