@@ -145,7 +145,14 @@ typedef enum msda_dtype {
                                           the copy but never issue it, so
                                           their bounded wait runs out and
                                           they report MSDA_ERR_DEVICE_TIMEOUT
-                                          (and finish on direct loads) */
+                                          (and finish on direct loads);
+                                          msda_query_head's tensor-core
+                                          kernel arms each CTA's first
+                                          operand stage without loading it:
+                                          its waits run out (about a second
+                                          each), it reports the same status,
+                                          writes no output, frees its tensor
+                                          memory and returns */
 
 /* Sizes of one call.  S = sum_l H_l * W_l. */
 typedef struct msda_problem {

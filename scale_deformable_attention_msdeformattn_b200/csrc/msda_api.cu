@@ -1215,6 +1215,7 @@ msda_status msda_query_head(const msda_problem *problem, int32_t in_features, co
     p.k_shift = ks;  // L*K is a power of two, so K is one too
     p.ref = reference_points;
     p.shapes = spatial_shapes;
+    p.withhold = (problem->flags & MSDA_TEST_WITHHOLD_COPY) ? 1 : 0;
     return launch_gemm(3 * P <= 128 ? 1 : MSDA_GEMM_HEAD_SUB, mx, mw, mloc, mattn, p,
                        reinterpret_cast<cudaStream_t>(stream));
 }

@@ -101,6 +101,7 @@ struct Params {
     const int64_t *shapes;    // [L, 2] (H, W), device
     int stages;               // stage ring depth (<= kMaxStages)
     int w_bytes;              // weight-resident: bytes of the w area
+    int withhold;             // testing: arm the CTA's first stage without loading it
     int *status;
 };
 
@@ -430,6 +431,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ C
                     }
                     uint8_t *a_tile = smem + s * C::kStageBytes;
                     mbar_expect_tx(full + s, (unsigned)C::kStageBytes);
+                    if (p.withhold && g == 0)
+                        continue;  // the stage never fills: the MMA lane's wait runs out
                     tma_load_2d(a_tile, &map_x, kb * kBK, m0, full + s);
                     if (!WRES) {
 #pragma unroll
