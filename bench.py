@@ -51,14 +51,14 @@ L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 NCU_TRAFFIC = {
     # DRAM read + write per launch (the mean of the launches captured), from
     # the counter captures listed in the profiles/ summaries
-    ("fused_backward", "detr_encoder_f32"): {"bytes": 126669824, "csrc": "76997acc56ab4bc7"},
-    ("fused_forward", "detr_encoder_f32"): {"bytes": 59208448, "csrc": "76997acc56ab4bc7"},
-    ("fused_backward", "detr_decoder_bf16"): {"bytes": 135612160, "csrc": "76997acc56ab4bc7"},
-    ("fused_forward", "detr_decoder_bf16"): {"bytes": 51015424, "csrc": "76997acc56ab4bc7"},
-    ("fused_backward", "stress_1080p_k8_bf16"): {"bytes": 913981184, "csrc": "76997acc56ab4bc7"},
-    ("fused_forward", "stress_1080p_k8_bf16"): {"bytes": 384010752, "csrc": "76997acc56ab4bc7"},
-    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 141286400, "csrc": "76997acc56ab4bc7"},
-    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 73070336, "csrc": "76997acc56ab4bc7"},
+    ("fused_backward", "detr_encoder_f32"): {"bytes": 126197632, "csrc": "9ceaf8a65da5ceee"},
+    ("fused_forward", "detr_encoder_f32"): {"bytes": 59481600, "csrc": "9ceaf8a65da5ceee"},
+    ("fused_backward", "detr_decoder_bf16"): {"bytes": 132292352, "csrc": "9ceaf8a65da5ceee"},
+    ("fused_forward", "detr_decoder_bf16"): {"bytes": 51024640, "csrc": "9ceaf8a65da5ceee"},
+    ("fused_backward", "stress_1080p_k8_bf16"): {"bytes": 914386688, "csrc": "9ceaf8a65da5ceee"},
+    ("fused_forward", "stress_1080p_k8_bf16"): {"bytes": 381361664, "csrc": "9ceaf8a65da5ceee"},
+    ("dcn_backward", "dcnv3_stage1_f32"): {"bytes": 140071168, "csrc": "9ceaf8a65da5ceee"},
+    ("dcn_forward", "dcnv3_stage1_f32"): {"bytes": 73025024, "csrc": "9ceaf8a65da5ceee"},
 }
 
 
