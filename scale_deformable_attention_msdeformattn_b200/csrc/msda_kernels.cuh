@@ -49,8 +49,10 @@ namespace msda {
 
 // Tuning knobs (compile-time).  The forward gathers float32 rows with 16-byte
 // lane vectors, one sample in flight per lane and 4 CTAs per SM, and bf16
-// rows with 16-byte vectors and four samples in flight; the backward uses
-// 16-byte vectors (whole-sector grad_value reductions, more rows per warp).
+// rows with 16-byte vectors and four samples in flight; the backward sizes
+// its lanes by value type (float32 16 B, bf16 8 B, one-byte types 4 B) so
+// that a row's float32 gradient is one whole 128-byte line per reduction
+// request (D = 32), with 3 CTAs per SM.
 // Bulk-copy staging of the set-up inputs measured slower everywhere with
 // these layouts; it stays available per call (MSDA_STAGE_INPUTS, general
 // kernels) and by these switches.
@@ -1486,7 +1488,7 @@ template <int G> struct BwdChunk { static constexpr int kC = G < 4 ? G : 4; };
 //   2. after a CTA barrier, groups of FG lanes take the occupied slots, walk
 //      each list summing A * w_c * g (the weights are recomputed from the
 //      record, the row's grad_output read from shared memory) and reduce the
-//      sum into grad_value with one whole-sector vector reduction per lane;
+//      sum into grad_value with one vector reduction per lane (a row is a whole line);
 //      each walked slot is reset for the next tile;
 //   3. a second barrier closes the tile.
 // The table has at least as many slots as the tile has contributions, so a
