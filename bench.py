@@ -515,13 +515,15 @@ def run_ours(args):
             # the backward's own ceiling: its grad_value reductions (one float32
             # row of D channels per in-map corner) go through the L2's
             # reduction units, whose rate a reduction-only probe kernel
-            # measured on B200: 6.1 TB/s of payload (red.global.add.v4.f32 at
-            # random 128-byte rows of an L2-resident float32 array)
+            # measured on B200: 6.4 TB/s of payload (red.global.add.v4.f32 at
+            # random 128-byte rows of an L2-resident float32 array the size of
+            # the encoder's grad_value; bulk reductions from shared memory
+            # reach the same rate)
             red_bytes = stats["in_map_corners_per_sample"] * w.samples * w.D * 4
             ach = red_bytes / (bwd_ms * 1e-3) / 1e9
             result["roofline"]["l2_reduction"] = {
-                "bytes_per_launch": int(red_bytes), "achieved": round(ach, 1), "ceiling": 6100.0,
-                "unit": "GB/s", "frac": round(ach / 6100.0, 4),
+                "bytes_per_launch": int(red_bytes), "achieved": round(ach, 1), "ceiling": 6400.0,
+                "unit": "GB/s", "frac": round(ach / 6400.0, 4),
                 "ceiling_source": "reduction-only probe kernel on B200 (not part of this bench)"}
         if not args.no_e2e:
             result["e2e"] = _time_e2e(_pinned(x), step, make_outputs, flush, min(args.steps, 50),
