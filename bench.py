@@ -111,6 +111,10 @@ def parse_args(argv=None):
     ap.add_argument("--sorted", action="store_true",
                     help="order the queries by the Morton cell of their reference point "
                          "(msda_sort_queries, inside the timed step) and process them in that order")
+    ap.add_argument("--headline", choices=("graph", "launched"), default="graph",
+                    help="what `value` times: the step replayed from a CUDA graph captured once "
+                         "(default), or the step's calls launched one by one from the host; the "
+                         "other is reported beside it")
     ap.add_argument("--out", default=None, help="also append the JSON line to this file")
     a = ap.parse_args(argv)
     if a.warmup < 3:
@@ -389,6 +393,7 @@ def run_ours(args):
     if msda.device_status() != 0:
         raise SystemExit("kernels reported inconsistent geometry")
 
+    # K launched steps: the per-kernel times (events between the calls)
     evs = events(args.steps)
     clocks = ClockSampler(local)
     barrier()
@@ -401,7 +406,13 @@ def run_ours(args):
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     barrier()
+
+    # K replays of the same step from a CUDA graph: the step without the
+    # host's launch gaps
+    graphms = _graph_steps(step, 7, flush, args.steps, barrier)
     clocks.stop()
+    if msda.device_status() != 0:
+        raise SystemExit("kernels reported inconsistent geometry")
 
     fwd = [e[6].elapsed_time(e[1]) for e in evs]
     pre = [e[0].elapsed_time(e[6]) for e in evs]
@@ -409,7 +420,12 @@ def run_ours(args):
     bwd = [e[2].elapsed_time(e[3]) for e in evs]
     stepms = [e[0].elapsed_time(e[3]) for e in evs]
     samples_step = w.samples
-    total_ms, value = aggregate_over_ranks(float(sum(stepms)), samples_step, args.steps, world, dev)
+    l_total_ms, l_value = aggregate_over_ranks(float(sum(stepms)), samples_step, args.steps, world, dev)
+    g_total_ms, g_value = aggregate_over_ranks(float(sum(graphms)), samples_step, args.steps, world, dev)
+    if args.headline == "graph":
+        total_ms, value, headms = g_total_ms, g_value, graphms
+    else:
+        total_ms, value, headms = l_total_ms, l_value, stepms
     ms_per_step = total_ms / args.steps
 
     result = None
@@ -449,6 +465,9 @@ def run_ours(args):
                    if overlap else "msda_fused_forward -> msda_zero_grads -> msda_fused_backward"),
                 "query_order": "Morton cell of the reference point" if args.sorted else "natural",
                 "l2": "flushed between steps (256 MiB write outside the timed events)",
+                "timing": ("the step replayed from a CUDA graph captured once (both streams), events "
+                           "around each replay" if args.headline == "graph" else
+                           "the step's calls launched one by one, events around each step"),
                 "parallelism": f"dp{world} (independent batch per GPU)",
             },
             "fwd_ms": round(fwd_ms, 5),
@@ -458,7 +477,14 @@ def run_ours(args):
 
             "bwd_ms": round(bwd_ms, 5),
             "fwd_gsamples_per_s": round(samples_step / (fwd_ms * 1e-3) / 1e9, 4),
-            "step_ms_p10_p50_p90": [round(float(np.percentile(stepms, p)), 5) for p in (10, 50, 90)],
+            "step_ms_p10_p50_p90": [round(float(np.percentile(headms, p)), 5) for p in (10, 50, 90)],
+            # the other way of timing the same step (config.timing names the headline's)
+            ("launched" if args.headline == "graph" else "graph"): {
+                "value": round(l_value if args.headline == "graph" else g_value, 4), "unit": UNIT,
+                "ms_per_step": round((l_total_ms if args.headline == "graph" else g_total_ms)
+                                     / args.steps, 5),
+                "step_ms_p10_p50_p90": [round(float(np.percentile(
+                    stepms if args.headline == "graph" else graphms, p)), 5) for p in (10, 50, 90)]},
             "hbm_frac_step": round(step_bytes / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
             "roofline": {
                 "kernel": dom,
@@ -493,7 +519,6 @@ def run_ours(args):
             result["fwd_alone"] = _time_fwd(msda, t, outputs, flush, min(args.steps, 50),
                                             qv if int8 else t["value"], qs, order, nbytes, peaks)
             result["warm_l2"] = _time_warm(w, step, min(args.steps, 50))
-            result["graph"] = _time_graph(w.samples, step, flush, min(args.steps, 100), 7)
         stats = _input_stats(w, x)
         if "value_bytes_touched" in stats:
             # the value tensor counted by the sectors the gathers touch instead of whole
@@ -639,10 +664,10 @@ def _time_bwd(msda, t, o, flush, n, value, value_scale, order, merge):
             "bwd_ms": round(ms, 5), "launches": n}
 
 
-def _time_graph(samples, step, flush, n, nev):
-    """The step captured once into a CUDA graph (its two streams included) and
-    replayed n times, L2 flushed before each replay outside the graph; events
-    around each replay.  Removes the host's launch cost from the step."""
+def _capture_step(step, nev):
+    """The step captured once into a CUDA graph (its second stream included,
+    through the step's own fork and join events), after one more run on the
+    capture stream."""
     import torch
     stream = torch.cuda.current_stream()
     cap = torch.cuda.Stream()
@@ -651,25 +676,37 @@ def _time_graph(samples, step, flush, n, nev):
     with torch.cuda.stream(cap):
         step([torch.cuda.Event() for _ in range(nev)])  # once more on the capture stream
         torch.cuda.synchronize()
-        with torch.cuda.graph(g, stream=cap):
+        # thread-local capture: calls other threads make meanwhile (a process
+        # group's watchdog) neither break the capture nor fail
+        with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
             step([torch.cuda.Event() for _ in range(nev)])
     stream.wait_stream(cap)
+    return g
+
+
+def _graph_steps(step, nev, flush, n, barrier):
+    """n replays of the step from a CUDA graph captured once (both streams),
+    the L2 flushed before each outside the timed events, bracketed by a
+    barrier and a synchronize like the launched steps; the replays' event
+    times in ms."""
+    import torch
+    g = _capture_step(step, nev)
     for i in range(3):
         flush.fill_(float(i))
         g.replay()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    barrier()
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
     for i, (a, b) in enumerate(evs):
         flush.fill_(float(i))
-        a.record(stream)
+        a.record(cur)
         g.replay()
-        b.record(stream)
+        b.record(cur)
     torch.cuda.synchronize()
-    ms = [a.elapsed_time(b) for a, b in evs]
-    med = float(np.median(ms))
+    barrier()
     del g
-    return {"ms_per_step_median": round(med, 5), "ms_per_step_mean": round(float(np.mean(ms)), 5),
-            "value": round(samples / (float(np.mean(ms)) * 1e-3) / 1e9, 4), "unit": UNIT, "steps": n,
-            "l2": "flushed before each replay"}
+    return [a.elapsed_time(b) for a, b in evs]
 
 
 def _time_warm(w, step, n):
@@ -1169,9 +1206,15 @@ def run_dcn(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    graphms = _graph_steps(step, 6, flush, args.steps, lambda: dist.barrier() if world > 1 else None)
     clocks.stop()
     stepms = [e[0].elapsed_time(e[3]) for e in evs]
-    total_ms, value = aggregate_over_ranks(float(sum(stepms)), w.samples, args.steps, world, dev)
+    l_total_ms, l_value = aggregate_over_ranks(float(sum(stepms)), w.samples, args.steps, world, dev)
+    g_total_ms, g_value = aggregate_over_ranks(float(sum(graphms)), w.samples, args.steps, world, dev)
+    if args.headline == "graph":
+        total_ms, value, headms = g_total_ms, g_value, graphms
+    else:
+        total_ms, value, headms = l_total_ms, l_value, stepms
     result = None
     if rank == 0:
         peaks = _peaks()
@@ -1196,9 +1239,18 @@ def run_dcn(args):
                        "step": ("msda_quantize_value_s8 -> " if int8 else "")
                        + "msda_dcn_forward || msda_zero_grads (second stream) -> msda_dcn_backward",
                        "l2": "flushed between steps (256 MiB write outside the timed events)",
+                       "timing": ("the step replayed from a CUDA graph captured once (both streams), "
+                                  "events around each replay" if args.headline == "graph" else
+                                  "the step's calls launched one by one, events around each step"),
                        "parallelism": f"dp{world} (independent batch per GPU)"},
             "fwd_ms": round(fwd_ms, 5), "bwd_ms": round(bwd_ms, 5),
-            "step_ms_p10_p50_p90": [round(float(np.percentile(stepms, p)), 5) for p in (10, 50, 90)],
+            "step_ms_p10_p50_p90": [round(float(np.percentile(headms, p)), 5) for p in (10, 50, 90)],
+            ("launched" if args.headline == "graph" else "graph"): {
+                "value": round(l_value if args.headline == "graph" else g_value, 4), "unit": UNIT,
+                "ms_per_step": round((l_total_ms if args.headline == "graph" else g_total_ms)
+                                     / args.steps, 5),
+                "step_ms_p10_p50_p90": [round(float(np.percentile(
+                    stepms if args.headline == "graph" else graphms, p)), 5) for p in (10, 50, 90)]},
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -1208,8 +1260,6 @@ def run_dcn(args):
             "gpu_launches": (3 + (3 if int8 else 0)) * args.steps,
             "clocks": clocks.summary(),
         }
-        if world == 1:
-            result["graph"] = _time_graph(w.samples, step, flush, min(args.steps, 100), 6)
         if not args.no_e2e and world == 1:
             hin = {k: v.cpu().pin_memory() for k, v in t.items()}
             result["e2e"] = _time_e2e(hin, step, make_outputs, flush, min(args.steps, 50), w.samples,
