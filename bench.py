@@ -234,6 +234,27 @@ def rank_workload(base: wl.Workload, rank: int) -> wl.Workload:
     return base if rank == 0 else wl.dataclasses.replace(base, index=base.index + 1000 * rank)
 
 
+def _other_timing(headline: str, graph_ok: bool, steps: int, launched, graph) -> dict:
+    """The JSON entry of the step timing that is not the headline: value,
+    ms per step and percentiles of (value, total ms, per-step ms)."""
+    if not graph_ok:
+        return {"graph": {"unavailable": "CUDA graph capture failed; the launched steps are the headline"}}
+    key, (v, total, ms) = ("launched", launched) if headline == "graph" else ("graph", graph)
+    return {key: {"value": round(v, 4), "unit": UNIT, "ms_per_step": round(total / steps, 5),
+                  "step_ms_p10_p50_p90": [round(float(np.percentile(ms, p)), 5) for p in (10, 50, 90)]}}
+
+
+def _all_ranks(ok: bool, world: int, device=None) -> bool:
+    """Whether ok holds on every rank (a MIN all-reduce when world > 1)."""
+    if world == 1:
+        return ok
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([1 if ok else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return bool(t.item())
+
+
 def aggregate_over_ranks(total_ms: float, samples_per_rank_step: int, steps: int, world: int,
                          device=None):
     """Max over ranks of the timed duration (ms) and the whole-job throughput
@@ -409,7 +430,7 @@ def run_ours(args):
 
     # K replays of the same step from a CUDA graph: the step without the
     # host's launch gaps
-    graphms = _graph_steps(step, 7, flush, args.steps, barrier)
+    graphms = _graph_steps(step, 7, flush, args.steps, barrier, lambda ok: _all_ranks(ok, world, dev))
     clocks.stop()
     if msda.device_status() != 0:
         raise SystemExit("kernels reported inconsistent geometry")
@@ -421,6 +442,9 @@ def run_ours(args):
     stepms = [e[0].elapsed_time(e[3]) for e in evs]
     samples_step = w.samples
     l_total_ms, l_value = aggregate_over_ranks(float(sum(stepms)), samples_step, args.steps, world, dev)
+    graph_ok = graphms is not None
+    if not graph_ok:  # no graph: the launched steps are the headline
+        args.headline, graphms = "launched", stepms
     g_total_ms, g_value = aggregate_over_ranks(float(sum(graphms)), samples_step, args.steps, world, dev)
     if args.headline == "graph":
         total_ms, value, headms = g_total_ms, g_value, graphms
@@ -479,12 +503,8 @@ def run_ours(args):
             "fwd_gsamples_per_s": round(samples_step / (fwd_ms * 1e-3) / 1e9, 4),
             "step_ms_p10_p50_p90": [round(float(np.percentile(headms, p)), 5) for p in (10, 50, 90)],
             # the other way of timing the same step (config.timing names the headline's)
-            ("launched" if args.headline == "graph" else "graph"): {
-                "value": round(l_value if args.headline == "graph" else g_value, 4), "unit": UNIT,
-                "ms_per_step": round((l_total_ms if args.headline == "graph" else g_total_ms)
-                                     / args.steps, 5),
-                "step_ms_p10_p50_p90": [round(float(np.percentile(
-                    stepms if args.headline == "graph" else graphms, p)), 5) for p in (10, 50, 90)]},
+            **_other_timing(args.headline, graph_ok, args.steps, (l_value, l_total_ms, stepms),
+                            (g_value, g_total_ms, graphms)),
             "hbm_frac_step": round(step_bytes / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
             "roofline": {
                 "kernel": dom,
@@ -684,13 +704,20 @@ def _capture_step(step, nev):
     return g
 
 
-def _graph_steps(step, nev, flush, n, barrier):
+def _graph_steps(step, nev, flush, n, barrier, agree):
     """n replays of the step from a CUDA graph captured once (both streams),
     the L2 flushed before each outside the timed events, bracketed by a
     barrier and a synchronize like the launched steps; the replays' event
-    times in ms."""
+    times in ms, or None (on every rank) when the capture failed on any:
+    agree(ok) returns whether it succeeded on all ranks."""
     import torch
-    g = _capture_step(step, nev)
+    try:
+        g = _capture_step(step, nev)
+    except RuntimeError as e:
+        print(f"CUDA graph capture failed ({e}); the launched steps stand", file=sys.stderr)
+        g = None
+    if not agree(g is not None):
+        return None
     for i in range(3):
         flush.fill_(float(i))
         g.replay()
@@ -1206,9 +1233,13 @@ def run_dcn(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    graphms = _graph_steps(step, 6, flush, args.steps, lambda: dist.barrier() if world > 1 else None)
+    graphms = _graph_steps(step, 6, flush, args.steps, lambda: dist.barrier() if world > 1 else None,
+                           lambda ok: _all_ranks(ok, world, dev))
     clocks.stop()
     stepms = [e[0].elapsed_time(e[3]) for e in evs]
+    graph_ok = graphms is not None
+    if not graph_ok:
+        args.headline, graphms = "launched", stepms
     l_total_ms, l_value = aggregate_over_ranks(float(sum(stepms)), w.samples, args.steps, world, dev)
     g_total_ms, g_value = aggregate_over_ranks(float(sum(graphms)), w.samples, args.steps, world, dev)
     if args.headline == "graph":
@@ -1245,12 +1276,8 @@ def run_dcn(args):
                        "parallelism": f"dp{world} (independent batch per GPU)"},
             "fwd_ms": round(fwd_ms, 5), "bwd_ms": round(bwd_ms, 5),
             "step_ms_p10_p50_p90": [round(float(np.percentile(headms, p)), 5) for p in (10, 50, 90)],
-            ("launched" if args.headline == "graph" else "graph"): {
-                "value": round(l_value if args.headline == "graph" else g_value, 4), "unit": UNIT,
-                "ms_per_step": round((l_total_ms if args.headline == "graph" else g_total_ms)
-                                     / args.steps, 5),
-                "step_ms_p10_p50_p90": [round(float(np.percentile(
-                    stepms if args.headline == "graph" else graphms, p)), 5) for p in (10, 50, 90)]},
+            **_other_timing(args.headline, graph_ok, args.steps, (l_value, l_total_ms, stepms),
+                            (g_value, g_total_ms, graphms)),
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4),

@@ -1,6 +1,7 @@
 """Host logic of multi-GPU runs, exercised with gloo ranks on the CPU: the
-weak-scaling workload split and the max-over-ranks timing, and the reference
-arm under torchrun (only rank 0 reports).  No GPU is used."""
+weak-scaling workload split, the max-over-ranks timing, the ranks'
+agreement on the CUDA-graph timing, and the reference arm under torchrun
+(only rank 0 reports).  No GPU is used."""
 import json
 import os
 import socket
@@ -30,7 +31,9 @@ def _worker(rank, world, port, times, out):
     try:
         w = bench.rank_workload(wl.WORKLOADS["tiny_f32"], rank)
         total, value = bench.aggregate_over_ranks(times[rank], w.samples, 10, world)
-        out[rank] = (total, value, w.seed)
+        # the graph-capture agreement: false on every rank if false on any
+        agreed = (bench._all_ranks(True, world), bench._all_ranks(rank == 0, world))
+        out[rank] = (total, value, w.seed, agreed)
     finally:
         dist.destroy_process_group()
 
@@ -51,9 +54,10 @@ def test_max_over_ranks_and_weak_scaling_split():
         res = dict(out)
     samples = 1 * 16 * 2 * 2 * 2  # tiny workload: B*Q*M*L*K
     for r in range(world):
-        total, value, seed = res[r]
+        total, value, seed, agreed = res[r]
         assert total == 5.0  # the slowest rank sets the time
         assert abs(value - world * samples * 10 / 5e-3 / 1e9) < 1e-12
+        assert agreed == (True, False)  # a capture failed on one rank: every rank falls back
     assert res[0][2] != res[1][2]  # every rank draws its own batch
 
 
