@@ -1,14 +1,14 @@
-"""bench.py's host-side arithmetic on the CPU: algorithmic bytes against the
-survey's table for the encoder shape, the out-of-map statistics against a
-closed form, the touched-bytes count against brute force, and the clock
-summary's reason decoding."""
+"""bench.py's host-side arithmetic on the CPU: algorithmic bytes against
+hand counts for the encoder and decoder shapes, the out-of-map statistics against a
+closed form, the touched-bytes count against brute force, the clock
+summary's reason decoding and the headline timing's entries."""
 import numpy as np
 
 import bench
 from scale_deformable_attention_msdeformattn_b200 import workloads as wl
 
 
-def test_algorithmic_bytes_match_the_survey_table():
+def test_algorithmic_bytes_match_hand_counts():
     # encoder float32: forward 79.65 MB, backward 136.54 MB (value + loc + A +
     # out; grad_out + value + loc + A + grad_value + grad_loc + grad_attn)
     nb = bench.algorithmic_bytes(wl.WORKLOADS["detr_encoder_f32"])
@@ -88,3 +88,18 @@ def test_dcn_workload_sizes_agree_with_the_oracle_and_the_library():
     x1, x2 = wl.generate_dcn(w), wl.generate_dcn(w)
     assert np.array_equal(x1.offset, x2.offset) and np.array_equal(x1.mask, x2.mask)
     np.testing.assert_allclose(x1.mask.sum(-1), 1.0, rtol=1e-5)
+
+
+def test_headline_timing_and_the_other_entry():
+    """`value` times the graph-replayed step by default; the line carries the
+    launched step beside it, or says that the capture failed."""
+    assert bench.parse_args([]).headline == "graph"
+    launched = (7.4, 38.0, [0.38, 0.37, 0.39])
+    graph = (7.7, 37.0, [0.37, 0.37, 0.37])
+    e = bench._other_timing("graph", True, 100, launched, graph)
+    assert set(e) == {"launched"} and e["launched"]["value"] == 7.4
+    assert e["launched"]["ms_per_step"] == 0.38 and e["launched"]["step_ms_p10_p50_p90"][1] == 0.38
+    e = bench._other_timing("launched", True, 100, launched, graph)
+    assert set(e) == {"graph"} and e["graph"]["value"] == 7.7
+    e = bench._other_timing("launched", False, 100, launched, launched)
+    assert "unavailable" in e["graph"]
